@@ -1,0 +1,442 @@
+/*
+ * sla_oracle.c -- plain, slow, fp64 CPU oracle of the SageSLA attention
+ * forward (Sparse-Linear Attention with a SageAttention-style INT8 sparse
+ * part).  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the CPU
+ * baseline leg of the benchmark call it; the product library never does, and
+ * it shares no code with the CUDA path.
+ *
+ * What it computes, per (b, h), in the order the method defines it:
+ *
+ *  1. Pooled block means of Q and K over the valid tokens of each block
+ *     (query blocks of blk_q tokens, key blocks of blk_k tokens; the last block
+ *     of a sequence may be partial and uses its own token count).
+ *  2. Block importance s_IJ = qbar_I . kbar_J.  The pages keep "the top k% most
+ *     important key-value pairs" ("TurboDiffusion技术架构解析", §2.1, SLA
+ *     formula) without naming the criterion; the pooled dot product is the
+ *     reading taken here.  The dot product is accumulated in channel order
+ *     with one fused multiply-add per channel (one rounding per step).
+ *  3. Selection: per query block, the first k_sel key blocks in the order
+ *     (score descending, block index ascending); k_sel = floor(topk * n_kb +
+ *     1e-4) clamped to [0, n_kb]; the selected list is reported ascending.
+ *  4. INT8 quantisation (SageAttention style, "清华开源TurboDiffusion加速框架"
+ *     section "SageAttention与稀疏计算": FP16 -> INT8 on the tensor cores).
+ *     K is smoothed by its per-channel mean over all N tokens; per block
+ *     scale = amax / 127 in fp32; code = clamp(rint_even(x / scale), -127,
+ *     127), every step in IEEE fp32 so that a GPU can reproduce it exactly.
+ *  5. Sparse branch: for every query row, exact softmax attention
+ *     softmax(q k^T / sqrt(d)) v ("TurboDiffusion技术架构解析", §2.1, standard
+ *     attention formula) restricted to the tokens of the selected key blocks;
+ *     with quantisation on, the logits are (qhat . khat) * s_q * s_k / sqrt(d).
+ *  6. Linear branch over the remaining (unselected) key blocks: kernelised
+ *     linear attention phi(Q)(phi(K)^T V) ("TurboDiffusion技术架构解析", §2.1,
+ *     linear attention formula, phi = elu+1 or ReLU), normalised by
+ *     phi(q) . sum phi(k); computed in state form: h_J = phi(K_J)^T V_J,
+ *     z_J = sum of phi(K_J) rows, H_I = sum over unselected J of h_J.  A zero
+ *     denominator gives a zero output.  phi acts on the raw bf16 Q and K.
+ *  7. O = O_sparse + O_linear.
+ *
+ * Precision: fp64 everywhere except the quantisation step, which is specified
+ * in fp32.  Build with -ffp-contract=off and without -ffast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+static float bf32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* k_sel = floor(topk * n_kb + 1e-4), clamped to [0, n_kb]. */
+int orc_topk_count(int n_kb, double topk)
+{
+    double x = floor(topk * (double)n_kb + 1e-4);
+    if (x < 0.0) x = 0.0;
+    if (x > (double)n_kb) x = (double)n_kb;
+    return (int)x;
+}
+
+/* mean[J][c] = (sum of x[t][c] over the valid tokens t of block J) / count */
+static void pool_head(const uint16_t *x, int N, int d, int blk, double *mean)
+{
+    int nb = (N + blk - 1) / blk;
+    for (int J = 0; J < nb; ++J) {
+        int t0 = J * blk, t1 = t0 + blk < N ? t0 + blk : N;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int t = t0; t < t1; ++t) s += bf(x[(size_t)t * d + c]);
+            mean[(size_t)J * d + c] = s / (double)(t1 - t0);
+        }
+    }
+}
+
+void orc_pool(const uint16_t *x, int BH, int N, int d, int blk, double *mean)
+{
+    int nb = (N + blk - 1) / blk;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh)
+        pool_head(x + (size_t)bh * N * d, N, d, blk, mean + (size_t)bh * nb * d);
+}
+
+typedef struct { double s; int j; } scored;
+
+/* order: score descending, then block index ascending */
+static int cmp_scored(const void *a, const void *b)
+{
+    const scored *x = (const scored *)a, *y = (const scored *)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+static int cmp_int(const void *a, const void *b)
+{
+    int x = *(const int *)a, y = *(const int *)b;
+    return (x > y) - (x < y);
+}
+
+/* Scores and selection for one head.  idx: [n_qb][k_sel] ascending.
+ * scores (nullable): [n_qb][n_kb]. */
+static void mask_head(const uint16_t *q, const uint16_t *k, int N, int d, int blk_q, int blk_k,
+                      int k_sel, int32_t *idx, uint32_t *bitmap, double *scores)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int words = (n_kb + 31) / 32;
+    double *qm = (double *)malloc(sizeof(double) * (size_t)n_qb * d);
+    double *km = (double *)malloc(sizeof(double) * (size_t)n_kb * d);
+    scored *row = (scored *)malloc(sizeof(scored) * (size_t)n_kb);
+    int *pick = (int *)malloc(sizeof(int) * (size_t)(n_kb + 1));
+    pool_head(q, N, d, blk_q, qm);
+    pool_head(k, N, d, blk_k, km);
+    for (int I = 0; I < n_qb; ++I) {
+        for (int J = 0; J < n_kb; ++J) {
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s = fma(qm[(size_t)I * d + c], km[(size_t)J * d + c], s);
+            row[J].s = s;
+            row[J].j = J;
+            if (scores) scores[(size_t)I * n_kb + J] = s;
+        }
+        qsort(row, (size_t)n_kb, sizeof(scored), cmp_scored);
+        for (int r = 0; r < k_sel; ++r) pick[r] = row[r].j;
+        qsort(pick, (size_t)k_sel, sizeof(int), cmp_int);
+        for (int r = 0; r < k_sel; ++r) idx[(size_t)I * k_sel + r] = pick[r];
+        if (bitmap) {
+            uint32_t *w = bitmap + (size_t)I * words;
+            memset(w, 0, sizeof(uint32_t) * (size_t)words);
+            for (int r = 0; r < k_sel; ++r) w[pick[r] >> 5] |= 1u << (pick[r] & 31);
+        }
+    }
+    free(qm); free(km); free(row); free(pick);
+}
+
+void orc_block_mask(const uint16_t *q, const uint16_t *k, int BH, int N, int d, int blk_q,
+                    int blk_k, double topk, int32_t *idx, uint32_t *bitmap, double *scores)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int k_sel = orc_topk_count(n_kb, topk);
+    int words = (n_kb + 31) / 32;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh)
+        mask_head(q + (size_t)bh * N * d, k + (size_t)bh * N * d, N, d, blk_q, blk_k, k_sel,
+                  idx + (size_t)bh * n_qb * k_sel, bitmap ? bitmap + (size_t)bh * n_qb * words : NULL,
+                  scores ? scores + (size_t)bh * n_qb * n_kb : NULL);
+}
+
+/* Symmetric per-block INT8 code of x with scale s (both fp32). */
+static int8_t code8(float x, float s)
+{
+    if (s == 0.0f) return 0;
+    float r = rintf(x / s);
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/* Quantise one head.  K is smoothed by its fp32-rounded per-channel mean. */
+static void quant_head(const uint16_t *q, const uint16_t *k, int N, int d, int blk_q, int blk_k,
+                       int8_t *q8, int8_t *k8, float *sq, float *sk, float *kmean)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    float *mu = (float *)malloc(sizeof(float) * (size_t)d);
+    for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        for (int t = 0; t < N; ++t) s += bf(k[(size_t)t * d + c]);
+        mu[c] = (float)(s / (double)N);
+        if (kmean) kmean[c] = mu[c];
+    }
+    for (int I = 0; I < n_qb; ++I) {
+        int t0 = I * blk_q, t1 = t0 + blk_q < N ? t0 + blk_q : N;
+        float amax = 0.0f;
+        for (size_t e = (size_t)t0 * d; e < (size_t)t1 * d; ++e) amax = fmaxf(amax, fabsf(bf32(q[e])));
+        float s = amax / 127.0f;
+        sq[I] = s;
+        for (size_t e = (size_t)t0 * d; e < (size_t)t1 * d; ++e) q8[e] = code8(bf32(q[e]), s);
+    }
+    for (int J = 0; J < n_kb; ++J) {
+        int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+        float amax = 0.0f;
+        for (int t = t0; t < t1; ++t)
+            for (int c = 0; c < d; ++c) amax = fmaxf(amax, fabsf(bf32(k[(size_t)t * d + c]) - mu[c]));
+        float s = amax / 127.0f;
+        sk[J] = s;
+        for (int t = t0; t < t1; ++t)
+            for (int c = 0; c < d; ++c) k8[(size_t)t * d + c] = code8(bf32(k[(size_t)t * d + c]) - mu[c], s);
+    }
+    free(mu);
+}
+
+void orc_quantize(const uint16_t *q, const uint16_t *k, int BH, int N, int d, int blk_q, int blk_k,
+                  int8_t *q8, int8_t *k8, float *sq, float *sk, float *kmean)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+#pragma omp parallel for schedule(dynamic)
+    for (int bh = 0; bh < BH; ++bh)
+        quant_head(q + (size_t)bh * N * d, k + (size_t)bh * N * d, N, d, blk_q, blk_k,
+                   q8 + (size_t)bh * N * d, k8 + (size_t)bh * N * d, sq + (size_t)bh * n_qb,
+                   sk + (size_t)bh * n_kb, kmean ? kmean + (size_t)bh * d : NULL);
+}
+
+/* phi = elu+1 (0) or ReLU (1) */
+static double phi_f(double x, int phi)
+{
+    if (phi == 1) return x > 0.0 ? x : 0.0;
+    return x > 0.0 ? x + 1.0 : exp(x);
+}
+
+/* Linear-attention states of one head: h[J][c][e] = sum_t phi(k_tc) v_te,
+ * z[J][c] = sum_t phi(k_tc), over the valid tokens t of key block J. */
+static void states_head(const uint16_t *k, const uint16_t *v, int N, int d, int blk_k, int phi,
+                        double *h, double *z)
+{
+    int n_kb = (N + blk_k - 1) / blk_k;
+    double *pk = (double *)malloc(sizeof(double) * (size_t)d);
+    double *vv = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int J = 0; J < n_kb; ++J) {
+        double *hJ = h + (size_t)J * d * d, *zJ = z + (size_t)J * d;
+        memset(hJ, 0, sizeof(double) * (size_t)d * d);
+        memset(zJ, 0, sizeof(double) * (size_t)d);
+        int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+        for (int t = t0; t < t1; ++t) {
+            for (int c = 0; c < d; ++c) pk[c] = phi_f(bf(k[(size_t)t * d + c]), phi);
+            for (int e = 0; e < d; ++e) vv[e] = bf(v[(size_t)t * d + e]);
+            for (int c = 0; c < d; ++c) {
+                zJ[c] += pk[c];
+                for (int e = 0; e < d; ++e) hJ[(size_t)c * d + e] += pk[c] * vv[e];
+            }
+        }
+    }
+    free(pk); free(vv);
+}
+
+void orc_states(const uint16_t *k, const uint16_t *v, int N, int d, int blk_k, int phi,
+                double *h, double *z)
+{
+    states_head(k, v, N, d, blk_k, phi, h, z);
+}
+
+/* H_I = sum of h_J and Z_I = sum of z_J over the key blocks J not selected by
+ * query block I (sel: ascending list of k_sel block indices). */
+static void unselected_state(const int32_t *sel, int k_sel, int n_kb, int d, const double *h,
+                             const double *z, double *HI, double *ZI)
+{
+    memset(HI, 0, sizeof(double) * (size_t)d * d);
+    memset(ZI, 0, sizeof(double) * (size_t)d);
+    int r = 0;
+    for (int J = 0; J < n_kb; ++J) {
+        if (r < k_sel && sel[r] == J) { ++r; continue; }
+        const double *hJ = h + (size_t)J * d * d, *zJ = z + (size_t)J * d;
+        for (size_t e = 0; e < (size_t)d * d; ++e) HI[e] += hJ[e];
+        for (int c = 0; c < d; ++c) ZI[c] += zJ[c];
+    }
+}
+
+/* One output row i of one head: sparse part os[d], linear part ol[d].
+ * sel: the k_sel selected key blocks of i's query block; HI/ZI: its
+ * unselected state; work: scratch of k_sel*blk_k + d doubles. */
+static void row_out(int i, const uint16_t *q, const uint16_t *k, const uint16_t *v, int N, int d,
+                    int blk_q, int blk_k, int k_sel, const int32_t *sel, int phi, int quant,
+                    const int8_t *q8, const int8_t *k8, const float *sq, const float *sk,
+                    const double *HI, const double *ZI, double *os, double *ol, double *work)
+{
+    int I = i / blk_q;
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+    /* ---- sparse branch: exact softmax over the selected blocks' tokens ---- */
+    int nk = 0;
+    double mx = -INFINITY;
+    for (int r = 0; r < k_sel; ++r) {
+        int J = sel[r];
+        int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+        for (int j = t0; j < t1; ++j) {
+            double l;
+            if (quant) {
+                int64_t acc = 0;
+                for (int c = 0; c < d; ++c)
+                    acc += (int64_t)q8[(size_t)i * d + c] * (int64_t)k8[(size_t)j * d + c];
+                l = (double)acc * (double)sq[I] * (double)sk[J] * inv_sqrt_d;
+            } else {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c) acc += bf(q[(size_t)i * d + c]) * bf(k[(size_t)j * d + c]);
+                l = acc * inv_sqrt_d;
+            }
+            work[nk++] = l;
+            if (l > mx) mx = l;
+        }
+    }
+    for (int e = 0; e < d; ++e) os[e] = 0.0;
+    if (nk > 0) {
+        double den = 0.0;
+        int n = 0;
+        for (int r = 0; r < k_sel; ++r) {
+            int J = sel[r];
+            int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+            for (int j = t0; j < t1; ++j) {
+                double p = exp(work[n++] - mx);
+                den += p;
+                for (int e = 0; e < d; ++e) os[e] += p * bf(v[(size_t)j * d + e]);
+            }
+        }
+        for (int e = 0; e < d; ++e) os[e] /= den;
+    }
+    /* ---- linear branch: phi(q)^T H_I / (phi(q) . Z_I) ---- */
+    double *pq = work + nk;
+    for (int c = 0; c < d; ++c) pq[c] = phi_f(bf(q[(size_t)i * d + c]), phi);
+    double den = 0.0;
+    for (int c = 0; c < d; ++c) den += pq[c] * ZI[c];
+    for (int e = 0; e < d; ++e) {
+        double num = 0.0;
+        for (int c = 0; c < d; ++c) num += pq[c] * HI[(size_t)c * d + e];
+        ol[e] = den != 0.0 ? num / den : 0.0;
+    }
+}
+
+static int cmp_i64(const void *a, const void *b)
+{
+    int64_t x = *(const int64_t *)a, y = *(const int64_t *)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * Forward for a list of rows.  rows: [nrows][2] pairs (bh, i); when rows is
+ * NULL every row of every head is produced in [BH][N] order (nrows ignored).
+ * idx_in (nullable, [BH][n_qb][k_sel]) replaces the oracle's own selection.
+ * out, out_s, out_l: [nrows][d] (out_s / out_l nullable).  Returns 0, or -1
+ * when memory runs out or a row is out of range.
+ */
+int orc_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int BH, int N, int d,
+                int blk_q, int blk_k, double topk, int phi, int quant, const int32_t *idx_in,
+                const int64_t *rows, int64_t nrows, double *out, double *out_s, double *out_l)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int k_sel = orc_topk_count(n_kb, topk);
+    if (!rows) nrows = (int64_t)BH * N;
+    /* order[] = row numbers sorted by (bh, i); key = bh * N + i */
+    int64_t *key = (int64_t *)malloc(sizeof(int64_t) * 2 * (size_t)(nrows + 1));
+    if (!key) return -1;
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t bh = rows ? rows[2 * r] : r / N, i = rows ? rows[2 * r + 1] : r % N;
+        if (bh < 0 || bh >= BH || i < 0 || i >= N) { free(key); return -1; }
+        key[2 * r] = bh * (int64_t)N + i;
+        key[2 * r + 1] = r;
+    }
+    qsort(key, (size_t)nrows, 2 * sizeof(int64_t), cmp_i64);
+
+    size_t hd = (size_t)N * d;
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * ((size_t)n_qb * k_sel + 1));
+    int8_t *q8 = quant ? (int8_t *)malloc(hd) : NULL;
+    int8_t *k8 = quant ? (int8_t *)malloc(hd) : NULL;
+    float *sq = (float *)malloc(sizeof(float) * (size_t)n_qb);
+    float *sk = (float *)malloc(sizeof(float) * (size_t)n_kb);
+    double *h = (double *)malloc(sizeof(double) * (size_t)n_kb * d * d);
+    double *z = (double *)malloc(sizeof(double) * (size_t)n_kb * d);
+    int64_t *gstart = (int64_t *)malloc(sizeof(int64_t) * (size_t)(nrows + 1));
+    if (!idx || (quant && (!q8 || !k8)) || !sq || !sk || !h || !z || !gstart) return -1;
+
+    int64_t pos = 0;
+    while (pos < nrows) {
+        int bh = (int)(key[2 * pos] / N);
+        int64_t end = pos;
+        while (end < nrows && key[2 * end] / N == bh) ++end;
+        const uint16_t *qh = q + bh * hd, *kh = k + bh * hd, *vh = v + bh * hd;
+        if (idx_in)
+            memcpy(idx, idx_in + (size_t)bh * n_qb * k_sel, sizeof(int32_t) * (size_t)n_qb * k_sel);
+        else
+            mask_head(qh, kh, N, d, blk_q, blk_k, k_sel, idx, NULL, NULL);
+        if (quant) quant_head(qh, kh, N, d, blk_q, blk_k, q8, k8, sq, sk, NULL);
+#pragma omp parallel for schedule(dynamic)
+        for (int J = 0; J < n_kb; ++J) {
+            int t0 = J * blk_k;
+            int len = t0 + blk_k < N ? blk_k : N - t0;
+            states_head(kh + (size_t)t0 * d, vh + (size_t)t0 * d, len, d, blk_k, phi,
+                        h + (size_t)J * d * d, z + (size_t)J * d);
+        }
+        /* groups of rows that share a query block */
+        int64_t ng = 0;
+        for (int64_t r = pos; r < end; ++r)
+            if (r == pos || (key[2 * r] % N) / blk_q != (key[2 * r - 2] % N) / blk_q) gstart[ng++] = r;
+        gstart[ng] = end;
+#pragma omp parallel
+        {
+            size_t wn = (size_t)k_sel * blk_k + (size_t)d + 16;
+            double *work = (double *)malloc(sizeof(double) * wn);
+            double *HI = (double *)malloc(sizeof(double) * (size_t)d * d);
+            double *ZI = (double *)malloc(sizeof(double) * (size_t)d);
+            double *os = (double *)malloc(sizeof(double) * (size_t)d);
+            double *ol = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic)
+            for (int64_t g = 0; g < ng; ++g) {
+                int I = (int)((key[2 * gstart[g]] % N) / blk_q);
+                const int32_t *sel = idx + (size_t)I * k_sel;
+                unselected_state(sel, k_sel, n_kb, d, h, z, HI, ZI);
+                for (int64_t r = gstart[g]; r < gstart[g + 1]; ++r) {
+                    int i = (int)(key[2 * r] % N);
+                    int64_t o = key[2 * r + 1];
+                    row_out(i, qh, kh, vh, N, d, blk_q, blk_k, k_sel, sel, phi, quant, q8, k8, sq,
+                            sk, HI, ZI, os, ol, work);
+                    for (int e = 0; e < d; ++e) {
+                        out[(size_t)o * d + e] = os[e] + ol[e];
+                        if (out_s) out_s[(size_t)o * d + e] = os[e];
+                        if (out_l) out_l[(size_t)o * d + e] = ol[e];
+                    }
+                }
+            }
+            free(work); free(HI); free(ZI); free(os); free(ol);
+        }
+        pos = end;
+    }
+    free(key); free(gstart); free(idx); free(q8); free(k8); free(sq); free(sk); free(h); free(z);
+    return 0;
+}

@@ -1,0 +1,66 @@
+"""Planted-mistake check of the oracle's pins (CPU only).
+
+Each mutant is a copy of ``oracle/sla_oracle.c`` with one plausible mistake
+(a dropped term, a wrong sign or index, a transposed operand, a wrong rounding
+rule).  The copy is compiled into a temporary library and every pin of
+``test_oracle_pins`` is run against it; at least one pin must fail.  The
+mistakes are planted in the oracle only, on the CPU.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from test_oracle_pins import PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "sla_oracle.c")
+
+MUTANTS = {
+    "drop_inv_sqrt_d": ("double inv_sqrt_d = 1.0 / sqrt((double)d);", "double inv_sqrt_d = 1.0;"),
+    "linear_over_selected": ("if (r < k_sel && sel[r] == J) { ++r; continue; }",
+                             "if (!(r < k_sel && sel[r] == J)) continue; ++r;"),
+    "transposed_state": ("num += pq[c] * HI[(size_t)c * d + e];", "num += pq[c] * HI[(size_t)e * d + c];"),
+    "tie_prefers_higher_block": ("return (x->j > y->j) - (x->j < y->j);", "return (x->j < y->j) - (x->j > y->j);"),
+    "ceil_count": ("double x = floor(topk * (double)n_kb + 1e-4);", "double x = ceil(topk * (double)n_kb - 1e-4);"),
+    "pool_divides_by_block": ("mean[(size_t)J * d + c] = s / (double)(t1 - t0);", "mean[(size_t)J * d + c] = s / (double)blk;"),
+    "scale_over_128_q": ("        float s = amax / 127.0f;\n        sq[I] = s;", "        float s = amax / 128.0f;\n        sq[I] = s;"),
+    "no_smoothing": ("mu[c] = (float)(s / (double)N);", "mu[c] = 0.0f;"),
+    "softmax_unnormalised": ("for (int e = 0; e < d; ++e) os[e] /= den;", "(void)den;"),
+    "elu_without_plus_one": ("return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x) - 1.0;"),
+    "combine_minus": ("out[(size_t)o * d + e] = os[e] + ol[e];", "out[(size_t)o * d + e] = os[e] - ol[e];"),
+    "drop_key_scale": ("l = (double)acc * (double)sq[I] * (double)sk[J] * inv_sqrt_d;",
+                       "l = (double)acc * (double)sq[I] * inv_sqrt_d;"),
+    "truncating_round": ("float r = rintf(x / s);", "float r = truncf(x / s);"),
+    "score_key_index_swap": ("s = fma(qm[(size_t)I * d + c], km[(size_t)J * d + c], s);",
+                             "s = fma(qm[(size_t)I * d + c], km[(size_t)((J + 1) % n_kb) * d + c], s);"),
+    "ragged_tail_dropped": ("int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;\n        for (int j = t0; j < t1; ++j) {\n            double l;",
+                            "int t0 = J * blk_k, t1 = t0 + blk_k <= N ? t0 + blk_k : t0;\n        for (int j = t0; j < t1; ++j) {\n            double l;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    search, replace = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(search) == 1, f"mutation site for {name} not unique in the oracle"
+    mutated = src.replace(search, replace)
+    with tempfile.TemporaryDirectory() as tmp:
+        c_path = os.path.join(tmp, "mutant.c")
+        so_path = os.path.join(tmp, "mutant.so")
+        with open(c_path, "w") as f:
+            f.write(mutated)
+        subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", so_path, c_path, "-lm"])
+        lib = oracle.load(so_path)
+        caught = []
+        for pin in PINS:
+            try:
+                pin(lib)
+            except AssertionError:
+                caught.append(pin.__name__)
+            except (ValueError, IndexError, MemoryError, FloatingPointError):
+                caught.append(pin.__name__)
+        assert caught, f"no pin catches the planted mistake {name}"
