@@ -1,0 +1,139 @@
+/*
+ * sla.h -- C ABI of libsla.so: the SageSLA attention forward on B200 (sm_100a).
+ *
+ * SageSLA is Sparse-Linear Attention (SLA) with a SageAttention-style sparse
+ * part, the attention used by TurboDiffusion's video DiT
+ * ("TurboDiffusion技术架构解析：稀疏线性注意力应用实战" §2.1: standard
+ * attention softmax(QK^T/sqrt(d))V, linear attention phi(Q)(phi(K)^T V) with
+ * phi = ReLU or elu+1, and SLA keeping the top-k% most important key-value
+ * pairs; "TurboDiffusion" GitHub summary, 使用方式与安装: SageSLA is the
+ * SageAttention-based fast SLA forward; "清华开源TurboDiffusion加速框架",
+ * SageAttention与稀疏计算: INT8 low-bit attention on the tensor cores, about
+ * 10% of the attention connections kept).
+ *
+ * What one call computes, per (batch b, head h):
+ *   1. block means qbar_I (query blocks of blk_q tokens) and kbar_J (key blocks
+ *      of blk_k tokens) over the valid tokens of each block;
+ *   2. score s_IJ = qbar_I . kbar_J in fp64, accumulated over channels in order
+ *      with one fused multiply-add per channel; per query block I the k_sel key
+ *      blocks first in the order (score descending, block index ascending) are
+ *      selected, k_sel = sla_topk_count(n_kb, topk);
+ *   3. (quant = 1) K smoothed by its per-channel mean over all N tokens; Q and
+ *      the smoothed K quantised to INT8 with one fp32 scale per block
+ *      (scale = amax/127, code = clamp(rint_even(x/scale), +-127), IEEE fp32);
+ *   4. sparse branch: per query row, exact softmax attention over the tokens of
+ *      the selected key blocks; logits (qhat.khat)*s_q*s_k/sqrt(d) with
+ *      quant = 1, (q.k)/sqrt(d) in bf16 x bf16 -> fp32 with quant = 0;
+ *   5. linear branch over the unselected key blocks:
+ *      phi(q)^T H_I / (phi(q) . Z_I), H_I = sum_{J unselected} phi(K_J)^T V_J,
+ *      Z_I = sum_{J unselected} (column sums of phi(K_J)); phi acts on the raw
+ *      Q and K; a zero denominator gives a zero linear output;
+ *   6. out = sparse + linear, rounded to bf16.
+ *
+ * Layout: q, k, v, out are contiguous bf16 [B, H, N, d] (token index t-major).
+ * Only d = 128, blk_k = 64 and blk_q in {64, 128} are supported.
+ *
+ * Memory: every pointer is caller-owned device memory (q, k, v, out, outputs
+ * and the workspace), 16-byte aligned.  The library allocates nothing and
+ * keeps no per-call global state; calls on different workspaces may run
+ * concurrently on different streams.  Calls that share one workspace must be
+ * ordered (same stream or explicit events).
+ *
+ * Errors: arguments are validated before anything is enqueued; a bad argument
+ * returns SLA_ERR_INVALID_ARG (null/misaligned pointer, negative size, topk
+ * outside [0,1], phi/quant out of range), SLA_ERR_UNSUPPORTED (valid but not
+ * implemented: d != 128, blk_k != 64, blk_q not 64/128) or SLA_ERR_WORKSPACE
+ * (ws_bytes below sla_workspace_bytes).  A failed launch returns
+ * SLA_ERR_CUDA.  Kernels never trap: every wait is bounded, and a device-side
+ * failure (a wait that ran out, SLA_ERR_TIMEOUT) is recorded in a status word
+ * inside the workspace, which sla_check reads.  Each call that takes a
+ * workspace first clears that word (stream-ordered), so sla_check reports the
+ * most recent call on that workspace.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void*; NULL is the legacy
+ * default stream.  All work is enqueued asynchronously on it.
+ */
+#ifndef SLA_H
+#define SLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SLA_API __attribute__((visibility("default")))
+#else
+#define SLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SLA_OK = 0,
+    SLA_ERR_INVALID_ARG = 1,
+    SLA_ERR_UNSUPPORTED = 2,
+    SLA_ERR_WORKSPACE = 3,
+    SLA_ERR_CUDA = 4,
+    SLA_ERR_TIMEOUT = 5
+} sla_status;
+
+typedef enum { SLA_PHI_ELU1 = 0, SLA_PHI_RELU = 1 } sla_phi;
+
+/* Library version string (static storage). */
+SLA_API const char *sla_version(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SLA_API const char *sla_status_string(int status);
+
+/* Selected key blocks per query block: floor(topk * n_kb + 1e-4) with topk
+ * promoted to double, clamped to [0, n_kb].  Returns -1 if n_kb < 0 or topk
+ * is not in [0, 1]. */
+SLA_API int sla_topk_count(int n_kb, float topk);
+
+/* Bytes of device workspace that sla_forward needs for this problem
+ * (sla_block_mask and sla_quantize_qk need no more than this).  Returns 0
+ * for arguments sla_forward would reject. */
+SLA_API size_t sla_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant);
+
+/* Steps 1-2 only (pooled block scores and top-k selection).
+ *   idx_out    int32 [B, H, n_qb, k_sel], each row ascending (required unless
+ *              k_sel == 0).
+ *   bitmap_out uint32 [B, H, n_qb, ceil(n_kb/32)] (nullable); bit J%32 of word
+ *              J/32 is set iff key block J is selected.
+ * The selection is bit-exact with the fp64 definition above. */
+SLA_API sla_status sla_block_mask(const void *q_bf16, const void *k_bf16, int B, int H, int N, int d,
+                          int blk_q, int blk_k, float topk, int32_t *idx_out, uint32_t *bitmap_out,
+                          void *ws, size_t ws_bytes, void *stream);
+
+/* Step 3 only (smoothing and INT8 quantisation).
+ *   q_i8, k_i8  int8 [B, H, N, d] codes (k_i8 holds the smoothed K's codes)
+ *   q_scale     fp32 [B, H, n_qb],  k_scale fp32 [B, H, n_kb]
+ *   k_mean      fp32 [B, H, d] (nullable): the smoothing mean. */
+SLA_API sla_status sla_quantize_qk(const void *q_bf16, const void *k_bf16, int B, int H, int N, int d,
+                           int blk_q, int blk_k, int8_t *q_i8, int8_t *k_i8, float *q_scale,
+                           float *k_scale, float *k_mean, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole forward, steps 1-6.  out: bf16 [B, H, N, d]. */
+SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
+                       int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
+                       size_t ws_bytes, void *stream);
+
+/* Synchronises `stream` and returns the device-side status word of `ws`
+ * (SLA_OK, or SLA_ERR_TIMEOUT when a bounded wait ran out), or SLA_ERR_CUDA
+ * if the synchronisation itself failed. */
+SLA_API sla_status sla_check(void *ws, void *stream);
+
+/* Byte offsets of the workspace's internal regions for this problem, for
+ * inspection by tests: fills up to `n` entries of `offsets` in the order
+ * {status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean,
+ *  states, partials, htot, hq} and returns how many regions exist.  A region
+ * that a configuration does not use has offset (size_t)-1. */
+SLA_API int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant,
+                         size_t *offsets, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H */

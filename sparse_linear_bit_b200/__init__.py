@@ -1,0 +1,142 @@
+"""Python binding of libsla.so, the B200 (sm_100a) SageSLA attention forward.
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels
+behind the C ABI declared in ``include/sla.h``; torch supplies device memory
+and streams.  The functions carry the C names:
+
+* ``sla_topk_count(n_kb, topk)``
+* ``sla_workspace_bytes(B, H, N, d, blk_q, blk_k, topk, quant)``
+* ``sla_block_mask(q, k, blk_q, blk_k, topk, idx, bitmap, ws)``
+* ``sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws)``
+* ``sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws)``
+* ``sla_check(ws)``, ``sla_status_string(code)``, ``sla_workspace_layout(...)``
+
+Tensors are CUDA tensors laid out as the header states ([B, H, N, d] bf16 for
+q/k/v/out).  Calls enqueue on torch's current stream (or ``stream=``).  A
+non-OK status raises :class:`SlaError`.  There is no CPU fallback: importing
+this package without the built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
+    "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_forward", "sla_check", "workspace",
+    "LAYOUT_REGIONS", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
+LAYOUT_REGIONS = ("status", "qsum", "ksum", "scores", "idx", "amask", "q8", "k8", "qscale", "kscale", "kmean",
+                  "states", "partials", "htot", "hq")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python sparse_linear_bit_b200/build.py` "
+        "(the SageSLA forward has no CPU fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+_P, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+lib.sla_version.restype = ctypes.c_char_p
+lib.sla_status_string.argtypes = [_I]
+lib.sla_status_string.restype = ctypes.c_char_p
+lib.sla_topk_count.argtypes = [_I, _F]
+lib.sla_topk_count.restype = _I
+lib.sla_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _F, _I]
+lib.sla_workspace_bytes.restype = _SZ
+lib.sla_workspace_layout.argtypes = [_I, _I, _I, _I, _I, _I, _F, _I, ctypes.POINTER(_SZ), _I]
+lib.sla_workspace_layout.restype = _I
+lib.sla_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _SZ, _P]
+lib.sla_block_mask.restype = _I
+lib.sla_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]
+lib.sla_quantize_qk.restype = _I
+lib.sla_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P]
+lib.sla_forward.restype = _I
+lib.sla_check.argtypes = [_P, _P]
+lib.sla_check.restype = _I
+
+
+class SlaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = int(code)
+        super().__init__(f"{what}: {sla_status_string(code)} ({code})")
+
+
+def sla_version() -> str:
+    return lib.sla_version().decode()
+
+
+def sla_status_string(code: int) -> str:
+    return lib.sla_status_string(int(code)).decode()
+
+
+def sla_topk_count(n_kb: int, topk: float) -> int:
+    return int(lib.sla_topk_count(int(n_kb), float(topk)))
+
+
+def sla_workspace_bytes(B, H, N, d, blk_q, blk_k, topk, quant) -> int:
+    return int(lib.sla_workspace_bytes(B, H, N, d, blk_q, blk_k, float(topk), int(quant)))
+
+
+def sla_workspace_layout(B, H, N, d, blk_q, blk_k, topk, quant) -> dict:
+    arr = (_SZ * len(LAYOUT_REGIONS))()
+    n = lib.sla_workspace_layout(B, H, N, d, blk_q, blk_k, float(topk), int(quant), arr, len(arr))
+    none = (1 << (8 * ctypes.sizeof(_SZ))) - 1
+    return {name: (None if arr[i] == none else int(arr[i])) for i, name in enumerate(LAYOUT_REGIONS[:n])}
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def _bhnd(q):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def _ok(code: int, what: str) -> None:
+    if code != 0:
+        raise SlaError(code, what)
+
+
+def workspace(B, H, N, d, blk_q, blk_k, topk, quant, device=None):
+    """Allocate a workspace (uint8 CUDA tensor) large enough for sla_forward."""
+    import torch
+    n = sla_workspace_bytes(B, H, N, d, blk_q, blk_k, topk, quant)
+    if n == 0:
+        raise SlaError(1, "sla_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sla_block_mask(q, k, blk_q, blk_k, topk, idx, bitmap, ws, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_block_mask(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, float(topk), _ptr(idx), _ptr(bitmap),
+                           _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_block_mask")
+
+
+def sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_quantize_qk(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, _ptr(q_i8), _ptr(k_i8), _ptr(q_scale),
+                            _ptr(k_scale), _ptr(k_mean), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream)), "sla_quantize_qk")
+
+
+def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk), int(phi),
+                        int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_forward")
+
+
+def sla_check(ws, stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded a device-side failure."""
+    _ok(lib.sla_check(_ptr(ws), _stream(stream)), "sla_check")

@@ -1,0 +1,275 @@
+// sla_api.cu -- the C ABI of libsla.so (declared in include/sla.h): argument
+// validation, workspace layout and the launch sequence of the SageSLA forward.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sla.h"
+#include "sla_internal.h"
+
+namespace sla {
+
+int topk_count(int n_kb, float topk)
+{
+    if (n_kb < 0 || !(topk >= 0.0f && topk <= 1.0f)) return -1;
+    double x = std::floor((double)topk * (double)n_kb + 1e-4);
+    if (x < 0.0) x = 0.0;
+    if (x > (double)n_kb) x = (double)n_kb;
+    return (int)x;
+}
+
+Geometry make_geometry(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant)
+{
+    Geometry g{};
+    g.B = B; g.H = H; g.N = N; g.d = d; g.blk_q = blk_q; g.blk_k = blk_k; g.quant = quant;
+    g.BH = B * H;
+    g.n_qb = (N + blk_q - 1) / blk_q;
+    g.n_kb = (N + blk_k - 1) / blk_k;
+    g.n_kb_pad = (g.n_kb + 7) / 8 * 8;
+    g.k_sel = topk_count(g.n_kb, topk);
+    g.subtract = 2 * g.k_sel <= g.n_kb;
+    g.n_chunks = (g.n_kb + kStateChunk - 1) / kStateChunk;
+    return g;
+}
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+Layout make_layout(const Geometry &g)
+{
+    Layout L{};
+    const size_t BH = (size_t)g.BH, N = (size_t)g.N;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+    L.status = take(256);
+    L.qsum = take(BH * g.n_qb * kD * sizeof(double));
+    L.ksum = take(BH * g.n_kb * kD * sizeof(double));
+    L.scores = take(BH * g.n_qb * g.n_kb * sizeof(double));
+    L.idx = take(BH * g.n_qb * (size_t)(g.k_sel > 0 ? g.k_sel : 1) * sizeof(int32_t));
+    L.amask = take(BH * g.n_qb * g.n_kb_pad * sizeof(uint16_t));
+    const size_t none = (size_t)-1;
+    L.q8 = g.quant ? take(BH * N * kD) : none;
+    L.k8 = g.quant ? take(BH * N * kD) : none;
+    L.qscale = g.quant ? take(BH * g.n_qb * sizeof(float)) : none;
+    L.kscale = g.quant ? take(BH * g.n_kb * sizeof(float)) : none;
+    L.kmean = take(BH * kD * sizeof(float));
+    L.states = take(BH * g.n_kb * (size_t)kStateCols * sizeof(uint16_t));
+    L.partials = take(BH * g.n_chunks * (size_t)kStateCols * sizeof(float));
+    L.htot = take(BH * (size_t)kStateCols * sizeof(float));
+    L.hq = take(BH * g.n_qb * (size_t)kStateCols * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+static std::once_flag g_encode_once;
+
+bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const uint64_t *dims,
+                 const uint64_t *strides_bytes, const uint32_t *box)
+{
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return false;
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i < rank - 1) st[i] = strides_bytes[i];
+    }
+    CUresult r = g_encode(map, dtype, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace sla
+
+using namespace sla;
+
+namespace {
+
+bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+// shared validation of (B, H, N, d, blk_q, blk_k, topk)
+sla_status check_shape(int B, int H, int N, int d, int blk_q, int blk_k, float topk)
+{
+    if (B < 1 || H < 1 || N < 1 || d < 1 || blk_q < 1 || blk_k < 1) return SLA_ERR_INVALID_ARG;
+    if (!(topk >= 0.0f && topk <= 1.0f)) return SLA_ERR_INVALID_ARG;
+    if ((long long)B * H > (1LL << 24) || (long long)N > (1LL << 24)) return SLA_ERR_UNSUPPORTED;
+    if (d != kD || blk_k != kBlkK || (blk_q != 64 && blk_q != 128)) return SLA_ERR_UNSUPPORTED;
+    // int8 logits are converted exactly through a 2^22 window; the top-k kernel keeps one
+    // row of 64-bit keys in shared memory
+    if ((N + blk_k - 1) / blk_k > 24576) return SLA_ERR_UNSUPPORTED;
+    return SLA_OK;
+}
+
+char *ws_at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
+
+#define SLA_TRY(expr)                                                    \
+    do {                                                                 \
+        cudaError_t _e = (expr);                                         \
+        if (_e != cudaSuccess) return SLA_ERR_CUDA;                      \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *sla_version(void) { return "sla-b200 0.1.0 (sm_100a)"; }
+
+const char *sla_status_string(int status)
+{
+    switch (status) {
+    case SLA_OK: return "SLA_OK";
+    case SLA_ERR_INVALID_ARG: return "SLA_ERR_INVALID_ARG";
+    case SLA_ERR_UNSUPPORTED: return "SLA_ERR_UNSUPPORTED";
+    case SLA_ERR_WORKSPACE: return "SLA_ERR_WORKSPACE";
+    case SLA_ERR_CUDA: return "SLA_ERR_CUDA";
+    case SLA_ERR_TIMEOUT: return "SLA_ERR_TIMEOUT";
+    default: return "SLA_ERR_UNKNOWN";
+    }
+}
+
+int sla_topk_count(int n_kb, float topk) { return topk_count(n_kb, topk); }
+
+size_t sla_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant)
+{
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
+    return make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant)).total;
+}
+
+int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant, size_t *offsets,
+                         int n)
+{
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
+    const Layout L = make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant));
+    const size_t v[15] = {L.status, L.qsum,   L.ksum,   L.scores,   L.idx,  L.amask, L.q8, L.k8,
+                          L.qscale, L.kscale, L.kmean, L.states, L.partials, L.htot, L.hq};
+    for (int i = 0; i < n && i < 15; ++i) offsets[i] = v[i];
+    return 15;
+}
+
+sla_status sla_block_mask(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k, float topk,
+                          int32_t *idx_out, uint32_t *bitmap_out, void *ws, size_t ws_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
+    if (st != SLA_OK) return st;
+    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, topk, 0);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(ws)) return SLA_ERR_INVALID_ARG;
+    if (g.k_sel > 0 && (!idx_out || ((uintptr_t)idx_out & 3u))) return SLA_ERR_INVALID_ARG;
+    if (bitmap_out && ((uintptr_t)bitmap_out & 3u)) return SLA_ERR_INVALID_ARG;
+    const Layout L = make_layout(g);
+    if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
+    double *qsum = reinterpret_cast<double *>(ws_at(ws, L.qsum));
+    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
+    SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
+    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
+    SLA_TRY(launch_scores(qsum, ksum, g, scores, s));
+    int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
+    SLA_TRY(launch_topk(scores, g, idx, bitmap_out, reinterpret_cast<uint16_t *>(ws_at(ws, L.amask)), s));
+    return SLA_OK;
+}
+
+sla_status sla_quantize_qk(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k,
+                           int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale, float *k_mean, void *ws,
+                           size_t ws_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, 0.0f);
+    if (st != SLA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(ws) || !aligned16(q_i8) || !aligned16(k_i8))
+        return SLA_ERR_INVALID_ARG;
+    if (!q_scale || !k_scale || ((uintptr_t)q_scale & 3u) || ((uintptr_t)k_scale & 3u) ||
+        (k_mean && ((uintptr_t)k_mean & 3u)))
+        return SLA_ERR_INVALID_ARG;
+    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, 0.0f, 1);
+    const Layout L = make_layout(g);
+    if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
+    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    float *mean = k_mean ? k_mean : reinterpret_cast<float *>(ws_at(ws, L.kmean));
+    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
+    SLA_TRY(launch_kmean(ksum, g.BH, N, g.n_kb, mean, s));
+    SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, s));
+    SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, s));
+    return SLA_OK;
+}
+
+sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
+                       int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
+    if (st != SLA_OK) return st;
+    if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_RELU) return SLA_ERR_INVALID_ARG;
+    if (quant != 0 && quant != 1) return SLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+        return SLA_ERR_INVALID_ARG;
+    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, topk, quant);
+    const Layout L = make_layout(g);
+    if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int *status = reinterpret_cast<int *>(ws_at(ws, L.status));
+    SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+    double *qsum = reinterpret_cast<double *>(ws_at(ws, L.qsum));
+    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
+    int32_t *idx = reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
+    uint16_t *amask = reinterpret_cast<uint16_t *>(ws_at(ws, L.amask));
+    float *kmean = reinterpret_cast<float *>(ws_at(ws, L.kmean));
+    int8_t *q8 = quant ? reinterpret_cast<int8_t *>(ws_at(ws, L.q8)) : nullptr;
+    int8_t *k8 = quant ? reinterpret_cast<int8_t *>(ws_at(ws, L.k8)) : nullptr;
+    float *qscale = quant ? reinterpret_cast<float *>(ws_at(ws, L.qscale)) : nullptr;
+    float *kscale = quant ? reinterpret_cast<float *>(ws_at(ws, L.kscale)) : nullptr;
+    uint16_t *states = reinterpret_cast<uint16_t *>(ws_at(ws, L.states));
+    float *partials = reinterpret_cast<float *>(ws_at(ws, L.partials));
+    float *htot = reinterpret_cast<float *>(ws_at(ws, L.htot));
+    float *hq = reinterpret_cast<float *>(ws_at(ws, L.hq));
+
+    // (1) pooled block sums, (2) scores + top-k selection
+    SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
+    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
+    SLA_TRY(launch_scores(qsum, ksum, g, scores, s));
+    SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
+    // (3) smoothing + INT8 quantisation
+    if (quant) {
+        SLA_TRY(launch_kmean(ksum, g.BH, N, g.n_kb, kmean, s));
+        SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, s));
+        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, s));
+    }
+    // (4) per-key-block linear states and their global sum, (5) per-query-block state
+    SLA_TRY(launch_states(k, v, g, phi, states, partials, status, s));
+    SLA_TRY(launch_htot(partials, g, htot, s));
+    SLA_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));
+    // (6) block-sparse attention + linear epilogue + combine
+    SLA_TRY(launch_attention(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s));
+    return SLA_OK;
+}
+
+sla_status sla_check(void *ws, void *stream)
+{
+    if (!aligned16(ws)) return SLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SLA_ERR_CUDA;
+    return h == 0 ? SLA_OK : (sla_status)h;
+}
+
+}  // extern "C"

@@ -1,0 +1,56 @@
+// sla_internal.h -- shared declarations of the CUDA translation units of
+// libsla.so: problem geometry, workspace layout and kernel launchers.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sla {
+
+constexpr int kD = 128;                  // head dimension supported
+constexpr int kBlkK = 64;                // key block
+constexpr int kStateCols = kD * kD + kD; // h (d x d, stored [dim][channel]) then z (d)
+constexpr int kStateChunk = 32;          // key blocks per partial sum of the global state
+
+struct Geometry {
+    int B, H, N, d, blk_q, blk_k;
+    int BH, n_qb, n_kb, n_kb_pad, k_sel, quant;
+    bool subtract;  // H_I = H_total - sum(selected); otherwise sum(unselected)
+    int n_chunks;   // partial sums of the global state per head
+};
+
+struct Layout {
+    size_t status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean, states, partials, htot, hq;
+    size_t total;
+};
+
+Geometry make_geometry(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant);
+Layout make_layout(const Geometry &g);
+int topk_count(int n_kb, float topk);
+
+// ---- launchers (all asynchronous on `s`; return cudaGetLastError()) ----
+cudaError_t launch_pool_sums(const void *x, int BH, int N, int blk, int nb, double *out, cudaStream_t s);
+cudaError_t launch_kmean(const double *ksum, int BH, int N, int n_kb, float *kmean, cudaStream_t s);
+cudaError_t launch_scores(const double *qsum, const double *ksum, const Geometry &g, double *scores,
+                          cudaStream_t s);
+cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap,
+                        uint16_t *amask, cudaStream_t s);
+cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out,
+                         float *scale, cudaStream_t s);
+
+// linear branch and fused attention (tcgen05)
+cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states,
+                          float *partials, int *status, cudaStream_t s);
+cudaError_t launch_htot(const float *partials, const Geometry &g, float *htot, cudaStream_t s);
+cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, const float *htot,
+                                const Geometry &g, float *hq, int *status, cudaStream_t s);
+cudaError_t launch_attention(const void *q, const void *k, const void *v, const int8_t *q8, const int8_t *k8,
+                             const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
+                             const Geometry &g, int phi, void *out, int *status, cudaStream_t s);
+
+// TMA descriptor encoding (driver entry point fetched once through the runtime)
+bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const uint64_t *dims,
+                 const uint64_t *strides_bytes /* rank-1 entries */, const uint32_t *box);
+
+}  // namespace sla

@@ -1,0 +1,405 @@
+// sla_linear.cu -- linear branch of the SageSLA forward on tcgen05 tensor cores.
+//
+// Kernelised linear attention phi(Q)(phi(K)^T V) ("TurboDiffusion技术架构解析"
+// §2.1, phi = elu+1 or ReLU) applied, for query block I, to the key blocks I
+// did not select.  Three kernels:
+//
+//  states_kernel  per key block J: hT_J = V_J^T phi(K_J) (128 x 128, bf16 MMA,
+//                 fp32 TMEM accumulator) stored bf16 as [dim][channel], and
+//                 z_J = column sums of phi(K_J); a second accumulator sums the
+//                 fp32 states of a chunk of 32 key blocks for the global state.
+//  htot_kernel    global state per head = fixed-order sum of the chunk sums.
+//  reduce_kernel  per query block I: C_I = sum_J A[I][J] S_J as a dense GEMM
+//                 (M = 128 query blocks, N = 256 state columns, K = key
+//                 blocks) with a 0/1 mask A.  When at most half the key blocks
+//                 are selected A marks the selected blocks and the state is
+//                 H_total - C_I (only the selected ~10% go through bf16); else A
+//                 marks the unselected blocks and the state is C_I (exact zeros
+//                 when everything is selected).  Output fp32, the d x d part
+//                 rounded to tf32 for the epilogue MMA of the attention kernel.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "sla_internal.h"
+#include "sla_ptx.cuh"
+
+namespace sla {
+namespace {
+
+constexpr int kStatesThreads = 128;
+constexpr uint32_t kTileBytes = 64 * 128;  // one [64 rows x 128 B] TMA box
+
+struct StatesSmem {
+    alignas(1024) uint8_t k[2][2][kTileBytes];  // [stage][channel half][64 tokens x 64 ch]
+    alignas(1024) uint8_t v[2][2][kTileBytes];  // [stage][dim half][64 tokens x 64 dims]
+    uint64_t full[2];
+    uint64_t mma_done;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ __forceinline__ float phi_f(float x, int phi)
+{
+    if (phi == 1) return fmaxf(x, 0.0f);
+    return x > 0.0f ? x + 1.0f : expf(x);
+}
+
+__global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                                const __grid_constant__ CUtensorMap tm_v, int N,
+                                                                int n_kb, int n_chunks, int phi,
+                                                                uint16_t *__restrict__ states,
+                                                                float *__restrict__ partials, int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    StatesSmem &sm = *reinterpret_cast<StatesSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int bh = blockIdx.y, chunk = blockIdx.x;
+    const int Jbeg = chunk * kStateChunk, nJ = min(kStateChunk, n_kb - Jbeg);
+    volatile int *abort_flag = &sm.abort_flag;
+    if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
+    __syncthreads();
+    if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
+
+    if (tid == 0) {
+        mbar_init(&sm.full[0], 1);
+        mbar_init(&sm.full[1], 1);
+        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t d_blk = tmem, d_sum = tmem + 128;
+    constexpr uint32_t kIdesc = idesc(1, 1, 1, 1, 1, 128, 128);  // f32 <- bf16 (MN) x bf16 (MN)
+
+    auto issue = [&](int j) {
+        const int s = j & 1, J = Jbeg + j;
+        mbar_expect_tx(&sm.full[s], 4 * kTileBytes);
+        tma_load_3d(sm.k[s][0], &tm_k, &sm.full[s], 0, J * 64, bh);
+        tma_load_3d(sm.k[s][1], &tm_k, &sm.full[s], 64, J * 64, bh);
+        tma_load_3d(sm.v[s][0], &tm_v, &sm.full[s], 0, J * 64, bh);
+        tma_load_3d(sm.v[s][1], &tm_v, &sm.full[s], 64, J * 64, bh);
+    };
+    int issued = 0;
+    if (tid == 0) {
+        for (; issued < min(2, nJ); ++issued) issue(issued);
+    }
+
+    float zsum = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nJ && ok; ++j) {
+        const int s = j & 1, J = Jbeg + j;
+        ok = __syncthreads_and(mbar_wait(&sm.full[s], (j >> 1) & 1, status, abort_flag));
+        if (!ok) break;
+        // phi in place (elementwise, so the swizzle permutation is irrelevant);
+        // tokens past N contribute nothing
+        const int valid = min(64, N - J * 64);
+#pragma unroll 4
+        for (int l = 0; l < 8; ++l) {
+            const int e = tid + kStatesThreads * l;  // 16-byte chunk 0..1023 over both halves
+            const int half = e >> 9, row = (e & 511) >> 3;
+            uint4 *p = reinterpret_cast<uint4 *>(sm.k[s][half] + (e & 511) * 16);
+            uint4 w = *p;
+            uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float a = __uint_as_float(ww[i] << 16), b = __uint_as_float(ww[i] & 0xFFFF0000u);
+                ww[i] = row < valid ? pack_bf16x2(phi_f(a, phi), phi_f(b, phi)) : 0u;
+            }
+            *p = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t ka = smem_u32(sm.k[s][0]), va = smem_u32(sm.v[s][0]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = sdesc_sw128(va + 2048 * k, kTileBytes, 1024);  // A = V^T (dims x tokens)
+                const uint64_t bd = sdesc_sw128(ka + 2048 * k, kTileBytes, 1024);  // B = phi(K) (ch x tokens)
+                mma_bf16(d_blk, ad, bd, kIdesc, k > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t ad = sdesc_sw128(va + 2048 * k, kTileBytes, 1024);
+                const uint64_t bd = sdesc_sw128(ka + 2048 * k, kTileBytes, 1024);
+                mma_bf16(d_sum, ad, bd, kIdesc, (j > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.mma_done);
+        }
+        // z_J[c] = sum over tokens of phi(K)[t][c] (thread = channel), row order
+        {
+            const int c = tid, half = c >> 6, u = (c & 63) >> 3, el = c & 7;
+            const uint8_t *base = sm.k[s][half];
+            float z = 0.0f;
+            for (int r = 0; r < 64; ++r) {
+                const uint16_t b = *reinterpret_cast<const uint16_t *>(base + sw128_off(r, u) + el * 2);
+                z += __uint_as_float((uint32_t)b << 16);
+            }
+            zsum += z;
+            const __nv_bfloat16 zb = __float2bfloat16_rn(z);
+            states[((size_t)bh * n_kb + J) * kStateCols + kD * kD + c] = *reinterpret_cast<const uint16_t *>(&zb);
+        }
+        ok = __syncthreads_and(mbar_wait(&sm.mma_done, j & 1, status, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        // epilogue: thread = dim row d of hT_J (TMEM lane), 128 channel columns
+        {
+            const int d = tid;
+            uint16_t *dst = states + ((size_t)bh * n_kb + J) * kStateCols + (size_t)d * kD;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(d_blk + ((uint32_t)(warp * 32) << 16) + c0, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                uint4 *o = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && issued < nJ) issue(issued++);
+    }
+    // chunk sum of the fp32 states
+    if (ok && nJ > 0) {
+        const int d = tid;
+        float *dst = partials + ((size_t)bh * n_chunks + chunk) * kStateCols;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(d_sum + ((uint32_t)(warp * 32) << 16) + c0, r);
+            tmem_wait_ld();
+            float4 *o = reinterpret_cast<float4 *>(dst + (size_t)d * kD + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                o[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        }
+        dst[kD * kD + tid] = zsum;
+    }
+    if (!ok && tid == 0) {
+        // drain: loads and MMAs still in flight retire before shared memory / TMEM are released
+        for (int s = 0; s < 2; ++s) {
+            const int jl = issued - 1 - ((issued - 1 - s) & 1);  // last load issued on stage s
+            if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl >> 1) & 1);
+        }
+        mma_commit(&sm.drain);
+        mbar_wait_quiet(&sm.drain, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// htot[bh][n] = sum over chunks (in order) of partials[bh][chunk][n]
+__global__ void htot_kernel(const float *__restrict__ partials, int n_chunks, float *__restrict__ htot)
+{
+    const int bh = blockIdx.y, n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= kStateCols) return;
+    const float *p = partials + (size_t)bh * n_chunks * kStateCols + n;
+    float s = 0.0f;
+    for (int c = 0; c < n_chunks; ++c) s += p[(size_t)c * kStateCols];
+    htot[(size_t)bh * kStateCols + n] = s;
+}
+
+// ---------------------------------------------------------------------------
+// per-query-block state: warp 0 = TMA producer, warp 1 = MMA issuer,
+// warps 2..5 = epilogue (TMEM lanes by warp index % 4)
+// ---------------------------------------------------------------------------
+constexpr int kRedStages = 4;
+constexpr int kRedThreads = 192;
+constexpr uint32_t kRedA = 128 * 128;      // 128 query blocks x 64 key blocks (bf16)
+constexpr uint32_t kRedB = 4 * kTileBytes; // 64 key blocks x 256 columns (bf16), four 64-column boxes
+
+struct ReduceSmem {
+    alignas(1024) uint8_t a[kRedStages][kRedA];
+    alignas(1024) uint8_t b[kRedStages][kRedB];
+    uint64_t full[kRedStages];
+    uint64_t empty[kRedStages];
+    uint64_t done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(kRedThreads) reduce_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                             const __grid_constant__ CUtensorMap tm_s, int n_qb,
+                                                             int n_kb, int subtract, const float *__restrict__ htot,
+                                                             float *__restrict__ hq, int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    ReduceSmem &sm = *reinterpret_cast<ReduceSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int m_tile = blockIdx.x, n_tile = blockIdx.y, bh = blockIdx.z;
+    const int I0 = m_tile * 128, n0 = n_tile * 256;
+    const int n_valid = min(256, kStateCols - n0);  // 256 or 128
+    const int n_groups = n_valid / 64;
+    const int nk = (n_kb + 63) / 64;
+    volatile int *abort_flag = &sm.abort_flag;
+    if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
+    __syncthreads();
+    if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
+
+    if (tid == 0) {
+        for (int s = 0; s < kRedStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_s);
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        int issued = 0;
+        bool ok = true;
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % kRedStages, u = kt / kRedStages;
+            if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+            mbar_expect_tx(&sm.full[s], kRedA + (uint32_t)n_groups * kTileBytes);
+            tma_load_3d(sm.a[s], &tm_a, &sm.full[s], kt * 64, I0, bh);
+            for (int g = 0; g < n_groups; ++g)
+                tma_load_3d(sm.b[s] + g * kTileBytes, &tm_s, &sm.full[s], n0 + 64 * g, kt * 64, bh);
+            issued = kt + 1;
+        }
+        if (!ok) {  // let in-flight loads land before the CTA exits
+            for (int s = 0; s < kRedStages; ++s) {
+                int jl = -1;
+                for (int kt = 0; kt < issued; ++kt)
+                    if (kt % kRedStages == s) jl = kt;
+                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedStages) & 1);
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t id = idesc(1, 1, 1, 0, 1, 128, (uint32_t)n_valid);  // A K-major, B MN-major
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % kRedStages, u = kt / kRedStages;
+            if (!mbar_wait(&sm.full[s], u & 1, status, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t aa = smem_u32(sm.a[s]), ba = smem_u32(sm.b[s]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_bf16(tmem, sdesc_sw128(aa + 32 * k, 16, 1024), sdesc_sw128(ba + 2048 * k, kTileBytes, 1024), id,
+                         (kt > 0 || k > 0) ? 1u : 0u);
+            mma_commit(&sm.empty[s]);
+        }
+        mma_commit(&sm.done);
+    } else if (warp >= 2) {
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int I = I0 + q * 32 + lane;
+        if (__all_sync(0xffffffffu, mbar_wait(&sm.done, 0, status, abort_flag))) {
+            tc_fence_after();
+            float *dst = hq + ((size_t)bh * n_qb + I) * kStateCols + n0;
+            const float *ht = htot + (size_t)bh * kStateCols + n0;
+            for (int c0 = 0; c0 < n_valid; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + c0, r);
+                tmem_wait_ld();
+                if (I < n_qb) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float x = __uint_as_float(r[i]);
+                        if (subtract) x = __ldg(ht + c0 + i) - x;
+                        v[i] = (n0 + c0 + i < kD * kD) ? to_tf32(x) : x;
+                    }
+                    float4 *o = reinterpret_cast<float4 *>(dst + c0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                }
+            }
+        }
+    }
+    if (warp == 1 && lane == 0) mbar_wait_quiet(&sm.done, 0);  // MMAs retired before TMEM is freed
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states, float *partials,
+                          int *status, cudaStream_t s)
+{
+    CUtensorMap tk, tv;
+    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
+    const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, strides, box)) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(StatesSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(g.n_chunks, g.BH);
+    states_kernel<<<grid, kStatesThreads, smem, s>>>(tk, tv, g.N, g.n_kb, g.n_chunks, phi, states, partials, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_htot(const float *partials, const Geometry &g, float *htot, cudaStream_t s)
+{
+    dim3 grid((kStateCols + 255) / 256, g.BH);
+    htot_kernel<<<grid, 256, 0, s>>>(partials, g.n_chunks, htot);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, const float *htot, const Geometry &g,
+                                float *hq, int *status, cudaStream_t s)
+{
+    CUtensorMap ta, ts;
+    {
+        const uint64_t dims[3] = {(uint64_t)g.n_kb_pad, (uint64_t)g.n_qb, (uint64_t)g.BH};
+        const uint64_t strides[2] = {(uint64_t)g.n_kb_pad * 2, (uint64_t)g.n_qb * g.n_kb_pad * 2};
+        const uint32_t box[3] = {64, 128, 1};
+        if (!encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, amask, dims, strides, box))
+            return cudaErrorInvalidValue;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)kStateCols, (uint64_t)g.n_kb, (uint64_t)g.BH};
+        const uint64_t strides[2] = {(uint64_t)kStateCols * 2, (uint64_t)g.n_kb * kStateCols * 2};
+        const uint32_t box[3] = {64, 64, 1};
+        if (!encode_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, states, dims, strides, box))
+            return cudaErrorInvalidValue;
+    }
+    const size_t smem = sizeof(ReduceSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((g.n_qb + 127) / 128, (kStateCols + 255) / 256, g.BH);
+    reduce_kernel<<<grid, kRedThreads, smem, s>>>(ta, ts, g.n_qb, g.n_kb, g.subtract ? 1 : 0, htot, hq, status);
+    return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,388 @@
+// sla_mask_quant.cu -- block pooling, fp64 block scores, top-k block
+// selection and the smooth-and-quantise step of the SageSLA forward.
+//
+// * Pooling sums each block's bf16 rows in fp64.  Sums of up to 2^17 bf16
+//   values are exact in fp64 unless one (batch, head, channel) spans more than
+//   ~2^29 in magnitude, so block sums (and the per-channel mean used for
+//   smoothing) do not depend on the summation order.
+// * The score of key block J for query block I is the dot product of their
+//   mean rows in fp64, accumulated in channel order with one fused
+//   multiply-add per channel ("TurboDiffusion技术架构解析" §2.1: SLA keeps the
+//   top-k% most important key-value pairs; the pooled dot product is the
+//   importance criterion here).  Identical blocks therefore get identical
+//   scores, and ties go to the lower block index.
+// * Top-k selection per query block is a radix select on order-preserving
+//   64-bit keys of the scores, followed by an in-order pass that takes the
+//   lowest-index blocks among those equal to the threshold.
+// * Quantisation follows SageAttention's recipe ("清华开源TurboDiffusion加速
+//   框架", SageAttention与稀疏计算: FP16 -> INT8): K minus its per-channel mean,
+//   one fp32 scale per block (amax / 127), round-to-nearest-even codes clamped
+//   to [-127, 127]; each step is one IEEE fp32 operation.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sla_internal.h"
+
+namespace sla {
+namespace {
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8])
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// pooling: out[bh][J][c] = sum over valid rows of block J of x[bh][t][c]
+// grid (ceil(nb/kPoolBlocks), BH), 256 threads; thread = (row lane, 8-channel group)
+// ---------------------------------------------------------------------------
+constexpr int kPoolBlocks = 8;
+
+__global__ void __launch_bounds__(256) pool_sums_kernel(const uint4 *__restrict__ x, int N, int blk, int nb,
+                                                        double *__restrict__ out)
+{
+    __shared__ double red[16][kD];
+    const int bh = blockIdx.y;
+    const int cg = threadIdx.x & 15, rl = threadIdx.x >> 4;
+    const uint4 *xh = x + (size_t)bh * N * (kD / 8);
+    for (int J = blockIdx.x * kPoolBlocks; J < min(nb, (blockIdx.x + 1) * kPoolBlocks); ++J) {
+        const int t0 = J * blk, t1 = min(N, t0 + blk);
+        double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int r = t0 + rl; r < t1; r += 16) {
+            float f[8];
+            bf16x8_to_f32(__ldg(xh + (size_t)r * (kD / 8) + cg), f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += (double)f[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) red[rl][cg * 8 + i] = acc[i];
+        __syncthreads();
+        if (threadIdx.x < kD) {
+            double s = 0.0;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) s += red[r][threadIdx.x];
+            out[((size_t)bh * nb + J) * kD + threadIdx.x] = s;
+        }
+        __syncthreads();
+    }
+}
+
+// kmean[bh][c] = fp32( (sum_J ksum[bh][J][c]) / N )
+__global__ void kmean_kernel(const double *__restrict__ ksum, int N, int n_kb, float *__restrict__ kmean)
+{
+    const int bh = blockIdx.x, c = threadIdx.x;
+    const double *p = ksum + (size_t)bh * n_kb * kD + c;
+    double s = 0.0;
+    for (int J = 0; J < n_kb; ++J) s += p[(size_t)J * kD];
+    kmean[(size_t)bh * kD + c] = (float)(s / (double)N);
+}
+
+// ---------------------------------------------------------------------------
+// scores[bh][I][J] = sum_c fma-chain( qsum[I][c]/nI , ksum[J][c]/nJ )
+// 64 x 64 output tile per CTA, 256 threads x (4 x 4) outputs, channel order kept
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) scores_kernel(const double *__restrict__ qsum, const double *__restrict__ ksum,
+                                                     int N, int blk_q, int blk_k, int n_qb, int n_kb,
+                                                     double *__restrict__ scores)
+{
+    __shared__ double As[16][64 + 1];
+    __shared__ double Bs[16][64 + 1];
+    const int bh = blockIdx.z, I0 = blockIdx.y * 64, J0 = blockIdx.x * 64;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const double *qh = qsum + (size_t)bh * n_qb * kD;
+    const double *kh = ksum + (size_t)bh * n_kb * kD;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int c0 = 0; c0 < kD; c0 += 16) {
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            const int e = threadIdx.x + 256 * l;  // 0..1023 = 64 rows x 16 channels
+            const int r = e >> 4, c = e & 15;
+            const int I = I0 + r, J = J0 + r;
+            double a = 0.0, b = 0.0;
+            if (I < n_qb) a = qh[(size_t)I * kD + c0 + c] / (double)(min(N, (I + 1) * blk_q) - I * blk_q);
+            if (J < n_kb) b = kh[(size_t)J * kD + c0 + c] / (double)(min(N, (J + 1) * blk_k) - J * blk_k);
+            As[c][r] = a;
+            Bs[c][r] = b;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            double a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = As[c][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = Bs[c][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    double *sh = scores + (size_t)bh * n_qb * n_kb;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int I = I0 + ty * 4 + i;
+        if (I >= n_qb) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int J = J0 + tx * 4 + j;
+            if (J < n_kb) sh[(size_t)I * n_kb + J] = acc[i][j] + 0.0;  // -0 -> +0
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// top-k selection: one CTA (128 threads) per (bh, I)
+// ---------------------------------------------------------------------------
+constexpr int kTopkThreads = 128;
+
+__device__ __forceinline__ uint64_t order_key(double s)
+{
+    const uint64_t u = (uint64_t)__double_as_longlong(s);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// exclusive prefix sum over the CTA (128 threads); returns the total in *total
+__device__ int block_exclusive_scan(int v, int *total, int *warp_tmp)
+{
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tmp[w] = x;
+    __syncthreads();
+    int base = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kTopkThreads / 32; ++i) {
+        if (i < w) base += warp_tmp[i];
+        tot += warp_tmp[i];
+    }
+    __syncthreads();
+    *total = tot;
+    return base + x - v;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double *__restrict__ scores, int n_qb, int n_kb,
+                                                            int n_kb_pad, int k_sel, int subtract,
+                                                            int32_t *__restrict__ idx, uint32_t *__restrict__ bitmap,
+                                                            uint16_t *__restrict__ amask)
+{
+    extern __shared__ uint64_t keys[];  // [n_kb]
+    __shared__ int hist[256];
+    __shared__ int warp_tmp[kTopkThreads / 32];
+    __shared__ int s_bin, s_remaining;
+    const int row = blockIdx.x;  // bh * n_qb + I
+    const double *sr = scores + (size_t)row * n_kb;
+    for (int J = threadIdx.x; J < n_kb; J += kTopkThreads) keys[J] = order_key(sr[J]);
+
+    // radix select for the k_sel-th largest key
+    uint64_t prefix = 0, mask = 0;
+    int remaining = k_sel;
+    if (k_sel > 0 && k_sel < n_kb) {
+        for (int shift = 56; shift >= 0; shift -= 8) {
+            for (int b = threadIdx.x; b < 256; b += kTopkThreads) hist[b] = 0;
+            __syncthreads();
+            for (int J = threadIdx.x; J < n_kb; J += kTopkThreads) {
+                const uint64_t k = keys[J];
+                if ((k & mask) == prefix) atomicAdd(&hist[(int)((k >> shift) & 255u)], 1);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                int cum = 0, b = 255;
+                for (; b > 0; --b) {
+                    if (cum + hist[b] >= remaining) break;
+                    cum += hist[b];
+                }
+                s_bin = b;
+                s_remaining = remaining - cum;
+            }
+            __syncthreads();
+            prefix |= (uint64_t)s_bin << shift;
+            mask |= (uint64_t)255u << shift;
+            remaining = s_remaining;
+            __syncthreads();
+        }
+    }
+    // selected: key > T, or key == T and among the first `remaining` such in J order
+    const uint64_t T = prefix;
+    const int chunk = (n_kb + kTopkThreads - 1) / kTopkThreads;
+    const int j0 = min(n_kb, threadIdx.x * chunk), j1 = min(n_kb, j0 + chunk);
+    auto base_sel = [&](int J) -> int {
+        if (k_sel == 0) return 0;
+        if (k_sel >= n_kb) return 1;
+        return keys[J] > T ? 1 : 0;
+    };
+    int n_eq = 0;
+    if (k_sel > 0 && k_sel < n_kb)
+        for (int J = j0; J < j1; ++J) n_eq += (keys[J] == T);
+    int tot;
+    const int eq_before = block_exclusive_scan(n_eq, &tot, warp_tmp);
+    int n_sel = 0, e = eq_before;
+    for (int J = j0; J < j1; ++J) {
+        int s = base_sel(J);
+        if (!s && k_sel > 0 && k_sel < n_kb && keys[J] == T) s = (e++ < remaining);
+        n_sel += s;
+    }
+    const int sel_before = block_exclusive_scan(n_sel, &tot, warp_tmp);
+    // write the ascending index list, the bitmap and the state-reduction mask row
+    int32_t *ir = idx + (size_t)row * k_sel;
+    const int words = (n_kb + 31) / 32;
+    uint32_t *br = bitmap ? bitmap + (size_t)row * words : nullptr;
+    uint16_t *ar = amask + (size_t)row * n_kb_pad;
+    const uint16_t one = 0x3F80u;  // bf16 1.0
+    int o = sel_before;
+    e = eq_before;
+    uint32_t word = 0;
+    int cur_w = j0 >> 5;
+    for (int J = j0; J < j1; ++J) {
+        int s = base_sel(J);
+        if (!s && k_sel > 0 && k_sel < n_kb && keys[J] == T) s = (e++ < remaining);
+        if (s) ir[o++] = J;
+        ar[J] = (s ^ (subtract ? 0 : 1)) ? one : (uint16_t)0;
+        if (br) {
+            if ((J >> 5) != cur_w) {
+                if (word) atomicOr(&br[cur_w], word);
+                word = 0;
+                cur_w = J >> 5;
+            }
+            if (s) word |= 1u << (J & 31);
+        }
+    }
+    if (br && word) atomicOr(&br[cur_w], word);
+    for (int J = n_kb + threadIdx.x; J < n_kb_pad; J += kTopkThreads) ar[J] = 0;
+}
+
+// zero the bitmap rows before the atomicOr pass
+__global__ void zero_u32_kernel(uint32_t *p, size_t n)
+{
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        p[i] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// quantisation: one CTA per block, 256 threads; SMOOTH subtracts mean[c]
+// ---------------------------------------------------------------------------
+template <bool SMOOTH, int BLK>
+__global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
+                                                    const float *__restrict__ mean, uint2 *__restrict__ out,
+                                                    float *__restrict__ scale)
+{
+    constexpr int kVec = BLK * (kD / 8) / 256;  // uint4 loads per thread
+    __shared__ float warp_max[8];
+    const int bh = blockIdx.y, J = blockIdx.x;
+    const int t0 = J * BLK;
+    const int rows = min(BLK, N - t0);
+    const uint4 *xb = x + ((size_t)bh * N + t0) * (kD / 8);
+    float v[kVec][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int l = 0; l < kVec; ++l) {
+        const int e = threadIdx.x + 256 * l;  // uint4 index within block: row = e/16, chunk = e%16
+        const int r = e >> 4, cg = e & 15;
+        if (r < rows) {
+            bf16x8_to_f32(__ldg(xb + e), v[l]);
+            if (SMOOTH) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[l][i] = __fsub_rn(v[l][i], __ldg(mean + (size_t)bh * kD + cg * 8 + i));
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[l][i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
+    const float s = __fdiv_rn(amax, 127.0f);
+    if (threadIdx.x == 0) scale[(size_t)bh * nb + J] = s;
+    uint2 *ob = out + ((size_t)bh * N + t0) * (kD / 8);
+#pragma unroll
+    for (int l = 0; l < kVec; ++l) {
+        const int e = threadIdx.x + 256 * l;
+        if ((e >> 4) < rows) {
+            uint32_t w[2] = {0, 0};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int c = 0;
+                if (s != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(v[l][i], s))));
+                w[i >> 2] |= ((uint32_t)(c & 0xFF)) << (8 * (i & 3));
+            }
+            ob[e] = make_uint2(w[0], w[1]);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pool_sums(const void *x, int BH, int N, int blk, int nb, double *out, cudaStream_t s)
+{
+    dim3 grid((nb + kPoolBlocks - 1) / kPoolBlocks, BH);
+    pool_sums_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(x), N, blk, nb, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kmean(const double *ksum, int BH, int N, int n_kb, float *kmean, cudaStream_t s)
+{
+    kmean_kernel<<<BH, kD, 0, s>>>(ksum, N, n_kb, kmean);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const double *qsum, const double *ksum, const Geometry &g, double *scores, cudaStream_t s)
+{
+    dim3 grid((g.n_kb + 63) / 64, (g.n_qb + 63) / 64, g.BH);
+    scores_kernel<<<grid, 256, 0, s>>>(qsum, ksum, g.N, g.blk_q, g.blk_k, g.n_qb, g.n_kb, scores);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap, uint16_t *amask,
+                        cudaStream_t s)
+{
+    if (bitmap) {
+        const size_t n = (size_t)g.BH * g.n_qb * ((g.n_kb + 31) / 32);
+        zero_u32_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, s>>>(bitmap, n);
+    }
+    const size_t smem = sizeof(uint64_t) * (size_t)g.n_kb;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    topk_kernel<<<g.BH * g.n_qb, kTopkThreads, smem, s>>>(scores, g.n_qb, g.n_kb, g.n_kb_pad, g.k_sel,
+                                                          g.subtract ? 1 : 0, idx, bitmap, amask);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out, float *scale,
+                         cudaStream_t s)
+{
+    dim3 grid(nb, BH);
+    const uint4 *xi = static_cast<const uint4 *>(x);
+    uint2 *o = reinterpret_cast<uint2 *>(out);
+    if (mean) {
+        if (blk != 64) return cudaErrorInvalidValue;
+        quant_kernel<true, 64><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale);
+    } else if (blk == 128) {
+        quant_kernel<false, 128><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale);
+    } else if (blk == 64) {
+        quant_kernel<false, 64><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,118 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching a GPU.
+
+No call here reaches a CUDA API: every call is one the library must refuse
+during validation (null / misaligned pointers, unsupported shapes, small
+workspaces), or a pure host function.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sla.h")
+
+sla = pytest.importorskip("sparse_linear_bit_b200")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SLA_API\s+[\w\s\*]*?\b(sla_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 9
+    lib = ctypes.CDLL(sla.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_links_no_torch():
+    with open(sla.LIB_PATH, "rb") as f:
+        blob = f.read()
+    assert b"libtorch" not in blob and b"libc10" not in blob
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in sla.sla_version()
+    for code, name in enumerate(["SLA_OK", "SLA_ERR_INVALID_ARG", "SLA_ERR_UNSUPPORTED", "SLA_ERR_WORKSPACE",
+                                 "SLA_ERR_CUDA", "SLA_ERR_TIMEOUT"]):
+        assert sla.sla_status_string(code) == name
+    assert sla.sla_status_string(99) == "SLA_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("n_kb", [0, 1, 3, 10, 20, 32, 256, 512, 1182, 4096])
+@pytest.mark.parametrize("topk", [0.0, 0.05, 0.1, 0.15, 0.2, 0.3, 0.5, 0.7, 0.99, 1.0])
+def test_topk_count_matches_oracle_rule(n_kb, topk):
+    assert sla.sla_topk_count(n_kb, topk) == oracle.topk_count(n_kb, float(np.float32(topk)))
+
+
+def test_topk_count_rejects():
+    assert sla.sla_topk_count(-1, 0.1) == -1
+    assert sla.sla_topk_count(10, 1.5) == -1
+    assert sla.sla_topk_count(10, -0.1) == -1
+    assert sla.sla_topk_count(10, float("nan")) == -1
+
+
+def test_workspace_bytes():
+    a = sla.sla_workspace_bytes(1, 40, 75600, 128, 128, 64, 0.1, 1)
+    b = sla.sla_workspace_bytes(1, 40, 75600, 128, 128, 64, 0.1, 0)
+    assert a > b > 0
+    assert sla.sla_workspace_bytes(1, 40, 75600, 64, 128, 64, 0.1, 1) == 0      # d != 128
+    assert sla.sla_workspace_bytes(1, 40, 75600, 128, 96, 64, 0.1, 1) == 0      # blk_q
+    assert sla.sla_workspace_bytes(1, 40, 75600, 128, 128, 32, 0.1, 1) == 0     # blk_k
+    assert sla.sla_workspace_bytes(1, 40, 75600, 128, 128, 64, 1.1, 1) == 0     # topk
+    assert sla.sla_workspace_bytes(0, 40, 75600, 128, 128, 64, 0.1, 1) == 0     # B
+    lay = sla.sla_workspace_layout(1, 2, 2048, 128, 64, 64, 0.1, 1)
+    offs = [v for v in lay.values() if v is not None]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert sla.sla_workspace_layout(1, 2, 2048, 128, 64, 64, 0.1, 0)["q8"] is None
+
+
+FAKE = 1 << 20  # an aligned non-null address; never dereferenced because validation fails first
+L = sla.lib
+
+
+def fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, H=2, N=2048, d=128, blk_q=64, blk_k=64, topk=0.1, phi=0,
+             quant=1, ws=FAKE, ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.sla_forward(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["N"], a["d"], a["blk_q"], a["blk_k"],
+                         a["topk"], a["phi"], a["quant"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_forward_host_validation():
+    assert fwd(q=None) == 1
+    assert fwd(out=FAKE + 8) == 1          # misaligned
+    assert fwd(B=0) == 1 and fwd(N=-5) == 1
+    assert fwd(topk=1.5) == 1 and fwd(topk=float("nan")) == 1
+    assert fwd(phi=2) == 1 and fwd(quant=3) == 1
+    assert fwd(d=64) == 2 and fwd(blk_q=32) == 2 and fwd(blk_k=128) == 2
+    assert fwd(ws_bytes=0) == 3            # workspace too small (everything else valid)
+    need = sla.sla_workspace_bytes(1, 2, 2048, 128, 64, 64, 0.1, 1)
+    assert fwd(ws_bytes=need - 1) == 3
+
+
+def test_block_mask_and_quant_host_validation():
+    assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, 0.1, None, None, FAKE, 1 << 40, None) == 1
+    assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, 0.1, FAKE + 2, None, FAKE, 1 << 40, None) == 1
+    assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, 0.1, FAKE, None, FAKE, 16, None) == 3
+    assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 96, 64, 64, 0.1, FAKE, None, FAKE, 1 << 40, None) == 2
+    assert L.sla_quantize_qk(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, None, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                             None) == 1
+    assert L.sla_quantize_qk(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None) == 3
+    assert L.sla_check(None, None) == 1
+
+
+def test_binding_raises():
+    with pytest.raises(sla.SlaError) as e:
+        sla._ok(2, "x")
+    assert e.value.code == 2 and "UNSUPPORTED" in str(e.value)
