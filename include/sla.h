@@ -23,7 +23,9 @@
  *      (scale = amax/127, code = clamp(rint_even(x/scale), +-127), IEEE fp32);
  *   4. sparse branch: per query row, exact softmax attention over the tokens of
  *      the selected key blocks; logits (qhat.khat)*s_q*s_k/sqrt(d) with
- *      quant = 1, (q.k)/sqrt(d) in bf16 x bf16 -> fp32 with quant = 0;
+ *      quant = 1, (q.k)/sqrt(d) in bf16 x bf16 -> fp32 with quant = 0; P.V
+ *      with P rounded to bf16 (quant = 1) or to fp16 against an fp16 copy of
+ *      V (quant = 0; V entries beyond +-65504 saturate), fp32 accumulation;
  *   5. linear branch over the unselected key blocks:
  *      phi(q)^T H_I / (phi(q) . Z_I), H_I = sum_{J unselected} phi(K_J)^T V_J,
  *      Z_I = sum_{J unselected} (column sums of phi(K_J)); phi acts on the raw
@@ -127,7 +129,7 @@ SLA_API sla_status sla_check(void *ws, void *stream);
 /* Byte offsets of the workspace's internal regions for this problem, for
  * inspection by tests: fills up to `n` entries of `offsets` in the order
  * {status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean,
- *  states, partials, htot, hq} and returns how many regions exist.  A region
+ *  states, partials, htot, hq, v16} and returns how many regions exist.  A region
  * that a configuration does not use has offset (size_t)-1. */
 SLA_API int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant,
                          size_t *offsets, int n);

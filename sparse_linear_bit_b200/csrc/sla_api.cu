@@ -61,6 +61,7 @@ Layout make_layout(const Geometry &g)
     L.partials = take(BH * g.n_chunks * (size_t)kStateCols * sizeof(float));
     L.htot = take(BH * (size_t)kStateCols * sizeof(float));
     L.hq = take(BH * g.n_qb * (size_t)kStateCols * sizeof(float));
+    L.v16 = g.quant ? none : take(BH * N * kD * sizeof(uint16_t));
     L.total = off;
     return L;
 }
@@ -157,10 +158,10 @@ int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float
 {
     if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
     const Layout L = make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant));
-    const size_t v[15] = {L.status, L.qsum,   L.ksum,   L.scores,   L.idx,  L.amask, L.q8, L.k8,
-                          L.qscale, L.kscale, L.kmean, L.states, L.partials, L.htot, L.hq};
-    for (int i = 0; i < n && i < 15; ++i) offsets[i] = v[i];
-    return 15;
+    const size_t v[16] = {L.status, L.qsum,   L.ksum,  L.scores, L.idx,      L.amask, L.q8, L.k8,
+                          L.qscale, L.kscale, L.kmean, L.states, L.partials, L.htot,  L.hq, L.v16};
+    for (int i = 0; i < n && i < 16; ++i) offsets[i] = v[i];
+    return 16;
 }
 
 sla_status sla_block_mask(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k, float topk,
@@ -241,6 +242,7 @@ sla_status sla_forward(const void *q, const void *k, const void *v, void *out, i
     float *partials = reinterpret_cast<float *>(ws_at(ws, L.partials));
     float *htot = reinterpret_cast<float *>(ws_at(ws, L.htot));
     float *hq = reinterpret_cast<float *>(ws_at(ws, L.hq));
+    uint16_t *v16 = quant ? nullptr : reinterpret_cast<uint16_t *>(ws_at(ws, L.v16));
 
     // (1) pooled block sums, (2) scores + top-k selection
     SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
@@ -254,11 +256,11 @@ sla_status sla_forward(const void *q, const void *k, const void *v, void *out, i
         SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, s));
     }
     // (4) per-key-block linear states and their global sum, (5) per-query-block state
-    SLA_TRY(launch_states(k, v, g, phi, states, partials, status, s));
+    SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, s));
     SLA_TRY(launch_htot(partials, g, htot, s));
     SLA_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));
     // (6) block-sparse attention + linear epilogue + combine
-    SLA_TRY(launch_attention(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s));
+    SLA_TRY(launch_attention(q, k, quant ? v : v16, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s));
     return SLA_OK;
 }
 

@@ -21,7 +21,7 @@ struct Geometry {
 };
 
 struct Layout {
-    size_t status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean, states, partials, htot, hq;
+    size_t status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean, states, partials, htot, hq, v16;
     size_t total;
 };
 
@@ -41,10 +41,11 @@ cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const fl
 
 // linear branch and fused attention (tcgen05)
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states,
-                          float *partials, int *status, cudaStream_t s);
+                          float *partials, uint16_t *v16, int *status, cudaStream_t s);
 cudaError_t launch_htot(const float *partials, const Geometry &g, float *htot, cudaStream_t s);
 cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, const float *htot,
                                 const Geometry &g, float *hq, int *status, cudaStream_t s);
+// v: bf16 V with quant = 1, the fp16 copy of V with quant = 0
 cudaError_t launch_attention(const void *q, const void *k, const void *v, const int8_t *q8, const int8_t *k8,
                              const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
                              const Geometry &g, int phi, void *out, int *status, cudaStream_t s);

@@ -4,10 +4,14 @@
 // §2.1, phi = elu+1 or ReLU) applied, for query block I, to the key blocks I
 // did not select.  Three kernels:
 //
-//  states_kernel  per key block J: hT_J = V_J^T phi(K_J) (128 x 128, bf16 MMA,
-//                 fp32 TMEM accumulator) stored bf16 as [dim][channel], and
-//                 z_J = column sums of phi(K_J); a second accumulator sums the
-//                 fp32 states of a chunk of 32 key blocks for the global state.
+//  states_kernel  per key block J: hT_J = V_J^T phi(K_J) (128 x 128, fp16 MMA:
+//                 phi(K) and V converted to fp16 in shared memory, saturating
+//                 at +-65504; fp32 TMEM accumulator) stored bf16 as
+//                 [dim][channel], and z_J = column sums of phi(K_J); a second
+//                 accumulator sums the fp32 states of a chunk of 32 key blocks
+//                 for the global state.  Optionally writes the fp16 copy of V
+//                 that the attention kernel's fp16 P.V uses when quantisation
+//                 is off.
 //  htot_kernel    global state per head = fixed-order sum of the chunk sums.
 //  reduce_kernel  per query block I: C_I = sum_J A[I][J] S_J as a dense GEMM
 //                 (M = 128 query blocks, N = 256 state columns, K = key
@@ -19,6 +23,7 @@
 //                 rounded to tf32 for the epilogue MMA of the attention kernel.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -52,7 +57,8 @@ __global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_con
                                                                 const __grid_constant__ CUtensorMap tm_v, int N,
                                                                 int n_kb, int n_chunks, int phi,
                                                                 uint16_t *__restrict__ states,
-                                                                float *__restrict__ partials, int *status)
+                                                                float *__restrict__ partials,
+                                                                uint16_t *__restrict__ v16, int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     StatesSmem &sm = *reinterpret_cast<StatesSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t d_blk = tmem, d_sum = tmem + 128;
-    constexpr uint32_t kIdesc = idesc(1, 1, 1, 1, 1, 128, 128);  // f32 <- bf16 (MN) x bf16 (MN)
+    constexpr uint32_t kIdesc = idesc(1, 0, 0, 1, 1, 128, 128);  // f32 <- f16 (MN) x f16 (MN)
 
     auto issue = [&](int j) {
         const int s = j & 1, J = Jbeg + j;
@@ -104,22 +110,34 @@ __global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_con
         const int s = j & 1, J = Jbeg + j;
         ok = __syncthreads_and(mbar_wait(&sm.full[s], (j >> 1) & 1, status, abort_flag));
         if (!ok) break;
-        // phi in place (elementwise, so the swizzle permutation is irrelevant);
-        // tokens past N contribute nothing
+        // phi(K) and V to fp16 in place (elementwise, so the swizzle permutation
+        // is irrelevant); tokens past N contribute nothing
         const int valid = min(64, N - J * 64);
-#pragma unroll 4
-        for (int l = 0; l < 8; ++l) {
-            const int e = tid + kStatesThreads * l;  // 16-byte chunk 0..1023 over both halves
-            const int half = e >> 9, row = (e & 511) >> 3;
-            uint4 *p = reinterpret_cast<uint4 *>(sm.k[s][half] + (e & 511) * 16);
+#pragma unroll 2
+        for (int l = 0; l < 16; ++l) {
+            const int e = tid + kStatesThreads * l;  // 16-byte chunk 0..2047: K halves, then V halves
+            const bool is_v = e >= 1024;
+            const int e2 = e & 1023, half = e2 >> 9, row = (e2 & 511) >> 3;
+            uint8_t *tile = is_v ? sm.v[s][half] : sm.k[s][half];
+            uint4 *p = reinterpret_cast<uint4 *>(tile + (e2 & 511) * 16);
             uint4 w = *p;
             uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float a = __uint_as_float(ww[i] << 16), b = __uint_as_float(ww[i] & 0xFFFF0000u);
-                ww[i] = row < valid ? pack_bf16x2(phi_f(a, phi), phi_f(b, phi)) : 0u;
+                float a = __uint_as_float(ww[i] << 16), b = __uint_as_float(ww[i] & 0xFFFF0000u);
+                if (!is_v) {
+                    a = phi_f(a, phi);
+                    b = phi_f(b, phi);
+                }
+                ww[i] = row < valid ? pack_f16x2_sat(a, b) : 0u;
             }
             *p = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+            if (is_v && v16 != nullptr && row < valid) {
+                // un-swizzled fp16 copy of V: chunk (e2 & 7) of this row holds logical chunk ^ (row & 7)
+                const int u = (e2 & 7) ^ (row & 7);
+                *reinterpret_cast<uint4 *>(v16 + (((size_t)bh * N + J * 64 + row) * kD + half * 64 + u * 8)) =
+                    make_uint4(ww[0], ww[1], ww[2], ww[3]);
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -147,8 +165,8 @@ __global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_con
             const uint8_t *base = sm.k[s][half];
             float z = 0.0f;
             for (int r = 0; r < 64; ++r) {
-                const uint16_t b = *reinterpret_cast<const uint16_t *>(base + sw128_off(r, u) + el * 2);
-                z += __uint_as_float((uint32_t)b << 16);
+                const __half b = *reinterpret_cast<const __half *>(base + sw128_off(r, u) + el * 2);
+                z += __half2float(b);
             }
             zsum += z;
             const __nv_bfloat16 zb = __float2bfloat16_rn(z);
@@ -353,7 +371,7 @@ __global__ void __launch_bounds__(kRedThreads) reduce_kernel(const __grid_consta
 }  // namespace
 
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states, float *partials,
-                          int *status, cudaStream_t s)
+                          uint16_t *v16, int *status, cudaStream_t s)
 {
     CUtensorMap tk, tv;
     const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
@@ -361,11 +379,13 @@ cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int p
     const uint32_t box[3] = {64, 64, 1};
     if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box)) return cudaErrorInvalidValue;
     if (!encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, strides, box)) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(StatesSmem) + 1024;
+    // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
+    const size_t smem = sizeof(StatesSmem) + 1024 > 100 * 1024 ? sizeof(StatesSmem) + 1024 : 100 * 1024;
     cudaError_t e = cudaFuncSetAttribute(states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(g.n_chunks, g.BH);
-    states_kernel<<<grid, kStatesThreads, smem, s>>>(tk, tv, g.N, g.n_kb, g.n_chunks, phi, states, partials, status);
+    states_kernel<<<grid, kStatesThreads, smem, s>>>(tk, tv, g.N, g.n_kb, g.n_chunks, phi, states, partials, v16,
+                                                     status);
     return cudaGetLastError();
 }
 
