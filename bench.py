@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the SageSLA attention forward (libsla.so, sm_100a).
+
+One step = one sla_forward call over the whole workload (pooling, top-k block
+selection, smoothing + INT8 quantisation, linear states, per-query-block state,
+fused block-sparse attention + linear epilogue).  Default workload: the
+14B-720P attention shape (B=1, H=40, N=75600 tokens on a 21x45x80 grid,
+d=128, blk_q=128, blk_k=64, topk=0.1, phi=elu+1, INT8 on), synthetic seeded
+inputs.  The inputs (2.3 GB of Q/K/V) exceed the 126 MB L2, so no flush is
+needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--topk T] [--quant 0|1]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+Multi-GPU (launched with torch.distributed.run, one rank per GPU): every rank
+runs the full workload on its own GPU (weak scaling, no data-path collective;
+heads are independent).  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SLA fwd ms & dense-equiv TOPS at N=75600,H=40,d=128; % of tensor peak"
+ATTN_SRC = os.path.join(ROOT, "sparse_linear_bit_b200", "csrc", "sla_attention.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = {1: 11, 0: 8}  # our launches per sla_forward call (quant on / off)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan14b-720p")
+    ap.add_argument("--topk", type=float, default=0.10)
+    ap.add_argument("--quant", type=int, default=1)
+    ap.add_argument("--phi", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dense_equiv_ops(B, H, N, d):
+    """4 B H N^2 d: the multiply-adds of dense softmax attention (QK^T and PV), x2."""
+    return 4.0 * B * H * float(N) * float(N) * d
+
+
+def workload_config(w, a):
+    nbytes = w.B * w.H * w.N * w.d * 2
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid_thw": list(w.grid),
+            "blk_q": w.blk_q, "blk_k": w.blk_k, "topk": a.topk, "phi": ["elu+1", "relu"][a.phi],
+            "quant": "int8 Q/K, bf16 P.V" if a.quant else "bf16 Q.K^T, fp16 P.V",
+            "l2": ("inputs (3 x %.2f GB) exceed the 126 MB L2; no flush between steps" if 3 * nbytes > 126e6 else
+                   "inputs (3 x %.3f GB) fit in L2: steps run warm") % (nbytes / 1e9)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle leg (reference arm and cpu_baseline)
+# --------------------------------------------------------------------------
+
+def oracle_sample(q, k, v, w, a, n_qblocks, head=0):
+    """Time the fp64 oracle on one head's first n_qblocks query blocks."""
+    import oracle
+    oracle.build()
+    rows_i = np.arange(min(w.N, n_qblocks * w.blk_q), dtype=np.int64)
+    rows = np.stack([np.full_like(rows_i, head), rows_i], axis=1)
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, w.blk_q, w.blk_k, float(np.float32(a.topk)), phi=a.phi, quant=a.quant, rows=rows)
+    dt = time.perf_counter() - t0
+    ops = 4.0 * len(rows_i) * float(w.N) * w.d  # dense-equivalent ops of the sampled rows
+    return ops, dt, len(rows_i), oracle.num_threads()
+
+
+def run_reference(a, w, rank, world):
+    if rank != 0:
+        return 0
+    import synth
+    q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
+    n_qb = 16
+    for _ in range(a.warmup):
+        oracle_sample(q, k, v, w, a, n_qb)
+    times, ops_total = [], 0.0
+    for _ in range(a.steps):
+        ops, dt, nrows, cores = oracle_sample(q, k, v, w, a, n_qb)
+        times.append(dt)
+        ops_total += ops
+    tot = sum(times)
+    value = ops_total / tot / 1e12
+    sample = (f"one head, first {nrows} query rows ({n_qb} query blocks) of the {w.name} workload per step, "
+              f"with that head's mask, quantisation and states; dense-equivalent ops of those rows")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * tot / a.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, a),
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# helpers
+# --------------------------------------------------------------------------
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def attn_source_sha():
+    h = hashlib.sha256()
+    for name in ("sla_attention.cu", "sla_ptx.cuh"):
+        with open(os.path.join(ROOT, "sparse_linear_bit_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, topk, quant):
+    """DRAM bytes per attention launch from a committed ncu capture, or None when
+    the capture does not match the current kernel source or this workload."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("kernel_source_sha") != attn_source_sha():
+        return None
+    key = f"{workload}|topk={topk:g}|quant={quant}"
+    return t.get("bytes_per_launch", {}).get(key)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.f.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def selected_work(idx, w, k_sel):
+    """Exact multiply-adds of the sparse branch: rows x valid selected keys x d, per launch."""
+    n_qb = -(-w.N // w.blk_q)
+    rows = np.minimum(w.blk_q, w.N - np.arange(n_qb) * w.blk_q).astype(np.float64)
+    keys_per_block = np.minimum(64, w.N - np.arange(-(-w.N // 64)) * 64).astype(np.float64)
+    keys = keys_per_block[idx].sum(axis=-1)  # [BH, n_qb]
+    return float((keys * rows[None, :]).sum()) * w.d
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+
+def main():
+    a = parse()
+    import synth
+
+    w0 = synth.WORKLOADS[a.workload]
+    w = synth.Workload(w0.name, w0.B, w0.H, w0.grid, blk_q=w0.blk_q, blk_k=w0.blk_k, topk=a.topk, phi=a.phi,
+                       quant=a.quant, seed=w0.seed)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        return run_reference(a, w, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    import sparse_linear_bit_b200 as sla
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    # ---- inputs: generated once (rank 0) and shared through /dev/shm
+    shm = f"/dev/shm/sla_bench_{w.name}_{w.seed}_{os.getuid()}"
+    if world == 1:
+        q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
+    else:
+        if rank == 0:
+            q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
+            for nm, x in (("q", q), ("k", k), ("v", v)):
+                np.save(shm + f"_{nm}.npy", x)
+        dist.barrier()
+        if rank != 0:
+            q, k, v = (np.load(shm + f"_{nm}.npy") for nm in ("q", "k", "v"))
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    out = torch.empty_like(qd)
+    ws = sla.workspace(w.B, w.H, w.N, w.d, w.blk_q, w.blk_k, a.topk, a.quant, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd = lambda: sla.sla_forward(qd, kd, vd, out, w.blk_q, w.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
+
+    for _ in range(max(3, a.warmup)):
+        fwd()
+    sla.sla_check(ws, stream=stream)
+
+    # ---- per-stage device times (CUDA events between the stages, same stream)
+    stage = {n: [] for n in sla.PROFILE_STAGES}
+    for _ in range(min(5, max(1, a.steps))):
+        r = sla.sla_forward_profile(qd, kd, vd, out, w.blk_q, w.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
+        for n_, t_ in r.items():
+            stage[n_].append(t_)
+    stage_ms = {n_: float(np.median(t_)) for n_, t_ in stage.items()}
+
+    # ---- timed region: K steps, inputs resident in HBM
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(vis.split(",")[local].strip() if vis else local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler start
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(a.steps):
+        fwd()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    sla.sla_check(ws, stream=stream)
+    ms = e0.elapsed_time(e1) / a.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ops = dense_equiv_ops(w.B, w.H, w.N, w.d)
+    value = world * ops / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the same call: pinned host Q/K/V in, bf16 out back to pinned host
+    e2e = None
+    if not a.no_e2e:
+        hq_, hk_, hv_ = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
+        hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+        steps_e2e = max(2, min(a.steps, 5))
+
+        def e2e_step():
+            qd.copy_(hq_, non_blocking=True)
+            kd.copy_(hk_, non_blocking=True)
+            vd.copy_(hv_, non_blocking=True)
+            fwd()
+            hout.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(steps_e2e):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = f0.elapsed_time(f1) / steps_e2e
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        nbytes = qd.numel() * 2
+        e2e = {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
+               "note": "host->device copy of Q, K, V from pinned memory, sla_forward, output copied back"}
+
+    # ---- roofline of the dominant kernel (attention), against the measured peaks
+    peaks, peak_kind = load_peaks()
+    n_kb = -(-w.N // w.blk_k)
+    k_sel = sla.sla_topk_count(n_kb, a.topk)
+    lay = sla.sla_workspace_layout(w.B, w.H, w.N, w.d, w.blk_q, w.blk_k, a.topk, a.quant)
+    n_qb = -(-w.N // w.blk_q)
+    idx = ws[lay["idx"]:lay["idx"] + w.B * w.H * n_qb * max(k_sel, 1) * 4].cpu().numpy().view(np.int32)
+    idx = idx.reshape(w.B * w.H, n_qb, max(k_sel, 1))[..., :k_sel]
+    macs = selected_work(idx, w, k_sel) if k_sel > 0 else 0.0
+    ops_qk, ops_pv = 2.0 * macs, 2.0 * macs
+    ops_lin = 2.0 * w.B * w.H * n_qb * 128.0 * w.d * w.d  # phi(Q_I) H_I, tf32
+    p_bf16 = float(peaks["bf16_tflops"]) * 1e12
+    p_qk = 2.0 * p_bf16 if a.quant else p_bf16  # int8 = 2x bf16 (nominal ratio)
+    p_tf32 = 0.5 * p_bf16
+    t_attn = stage_ms["attention"] * 1e-3
+    ideal = ops_qk / p_qk + ops_pv / p_bf16 + ops_lin / p_tf32
+    tot_ops = ops_qk + ops_pv + ops_lin
+    achieved = tot_ops / t_attn / 1e12
+    peak = tot_ops / ideal / 1e12
+    traffic = recorded_traffic(w.name, a.topk, a.quant)
+    roofline = {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s (burst); int8 = 2x, tf32 = 0.5x",
+                "ops_per_launch": {"qk_int8" if a.quant else "qk_bf16": ops_qk, "pv_bf16": ops_pv,
+                                   "linear_tf32": ops_lin},
+                "launch_ms": stage_ms["attention"]}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, single GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        n_qb_s = -(-w.N // w.blk_q)  # one whole head (about 10 s on 16 cores)
+        ops_s, dt, nrows, cores = oracle_sample(q, k, v, w, a, n_qb_s)
+        cpu = {"value": ops_s / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+               "sample": f"one of {w.B * w.H} heads of {w.name} ({nrows} query rows, {n_qb_s} query blocks), including "
+                         f"that head's mask, quantisation and states; {dt:.1f} s; dense-equivalent ops of those rows"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
+                "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "i8+bf16" if a.quant else "bf16+fp16", "data": "synthetic",
+                "config": workload_config(w, a), "stages_ms": stage_ms, "roofline": roofline,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "gpu_launches": KERNELS_PER_STEP[a.quant] * a.steps,
+                "dense_equiv_ops_per_step_per_gpu": ops}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+        if rank == 0:
+            for nm in ("q", "k", "v"):
+                try:
+                    os.unlink(shm + f"_{nm}.npy")
+                except OSError:
+                    pass
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

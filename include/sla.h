@@ -121,6 +121,15 @@ SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void
                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                        size_t ws_bytes, void *stream);
 
+/* sla_forward with per-stage device timing: enqueues the same launches with a
+ * CUDA event between stages, waits for them, and writes 7 floats to the host
+ * array stage_ms: milliseconds of {pooling, scores + top-k, quantisation,
+ * linear states, per-query-block state, attention, whole call}.  Blocks the
+ * calling host thread until the call has finished on `stream`. */
+SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
+                                       int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
+                                       size_t ws_bytes, void *stream, float *stage_ms);
+
 /* Synchronises `stream` and returns the device-side status word of `ws`
  * (SLA_OK, or SLA_ERR_TIMEOUT when a bounded wait ran out), or SLA_ERR_CUDA
  * if the synchronisation itself failed. */

@@ -9,7 +9,8 @@ and streams.  The functions carry the C names:
 * ``sla_block_mask(q, k, blk_q, blk_k, topk, idx, bitmap, ws)``
 * ``sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws)``
 * ``sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws)``
-* ``sla_check(ws)``, ``sla_status_string(code)``, ``sla_workspace_layout(...)``
+* ``sla_forward_profile(...)`` (per-stage device times), ``sla_check(ws)``,
+  ``sla_status_string(code)``, ``sla_workspace_layout(...)``
 
 Tensors are CUDA tensors laid out as the header states ([B, H, N, d] bf16 for
 q/k/v/out).  Calls enqueue on torch's current stream (or ``stream=``).  A
@@ -25,7 +26,7 @@ from typing import Optional
 __all__ = [
     "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_forward", "sla_check", "workspace",
-    "LAYOUT_REGIONS", "LIB_PATH",
+    "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -54,6 +55,9 @@ lib.sla_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, 
 lib.sla_quantize_qk.restype = _I
 lib.sla_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P]
 lib.sla_forward.restype = _I
+lib.sla_forward_profile.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P,
+                                    ctypes.POINTER(ctypes.c_float)]
+lib.sla_forward_profile.restype = _I
 lib.sla_check.argtypes = [_P, _P]
 lib.sla_check.restype = _I
 
@@ -135,6 +139,19 @@ def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -
     B, H, N, d = _bhnd(q)
     _ok(lib.sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk), int(phi),
                         int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_forward")
+
+
+PROFILE_STAGES = ("pool", "scores_topk", "quantize", "states", "state_reduce", "attention", "total")
+
+
+def sla_forward_profile(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -> dict:
+    """sla_forward with per-stage device times (ms) from CUDA events between stages."""
+    B, H, N, d = _bhnd(q)
+    arr = (ctypes.c_float * len(PROFILE_STAGES))()
+    _ok(lib.sla_forward_profile(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk),
+                                int(phi), int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream),
+                                arr), "sla_forward_profile")
+    return {name: float(arr[i]) for i, name in enumerate(PROFILE_STAGES)}
 
 
 def sla_check(ws, stream=None) -> None:

@@ -213,8 +213,16 @@ sla_status sla_quantize_qk(const void *q, const void *k, int B, int H, int N, in
     return SLA_OK;
 }
 
-sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
-                       int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The forward's launch sequence.  When `ev` is non-null, an event is recorded
+// before the first stage and after each of the kStages stages (on `s`).
+constexpr int kProfStages = 7;  // pool, scores+top-k, quantise, states, state reduce, attention, total
+sla_status run_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
+                       int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, cudaStream_t s,
+                       cudaEvent_t *ev)
 {
     sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
     if (st != SLA_OK) return st;
@@ -225,9 +233,7 @@ sla_status sla_forward(const void *q, const void *k, const void *v, void *out, i
     const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, topk, quant);
     const Layout L = make_layout(g);
     if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     int *status = reinterpret_cast<int *>(ws_at(ws, L.status));
-    SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
     double *qsum = reinterpret_cast<double *>(ws_at(ws, L.qsum));
     double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
     double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
@@ -243,25 +249,71 @@ sla_status sla_forward(const void *q, const void *k, const void *v, void *out, i
     float *htot = reinterpret_cast<float *>(ws_at(ws, L.htot));
     float *hq = reinterpret_cast<float *>(ws_at(ws, L.hq));
     uint16_t *v16 = quant ? nullptr : reinterpret_cast<uint16_t *>(ws_at(ws, L.v16));
+    int e = 0;
+    auto mark = [&]() { if (ev) cudaEventRecord(ev[e++], s); };
 
-    // (1) pooled block sums, (2) scores + top-k selection
+    SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+    mark();
+    // (1) pooled block sums
     SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
     SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
+    mark();
+    // (2) scores + top-k selection
     SLA_TRY(launch_scores(qsum, ksum, g, scores, s));
     SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
+    mark();
     // (3) smoothing + INT8 quantisation
     if (quant) {
         SLA_TRY(launch_kmean(ksum, g.BH, N, g.n_kb, kmean, s));
         SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, s));
         SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, s));
     }
-    // (4) per-key-block linear states and their global sum, (5) per-query-block state
+    mark();
+    // (4) per-key-block linear states and their global sum
     SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, s));
     SLA_TRY(launch_htot(partials, g, htot, s));
+    mark();
+    // (5) per-query-block state
     SLA_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));
+    mark();
     // (6) block-sparse attention + linear epilogue + combine
     SLA_TRY(launch_attention(q, k, quant ? v : v16, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s));
+    mark();
     return SLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
+                       int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, void *stream)
+{
+    return run_forward(q, k, v, out, B, H, N, d, blk_q, blk_k, topk, phi, quant, ws, ws_bytes,
+                       static_cast<cudaStream_t>(stream), nullptr);
+}
+
+sla_status sla_forward_profile(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
+                               int blk_q, int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes,
+                               void *stream, float *stage_ms)
+{
+    if (!stage_ms) return SLA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev[kProfStages];
+    int made = 0;
+    for (; made < kProfStages; ++made)
+        if (cudaEventCreate(&ev[made]) != cudaSuccess) break;
+    sla_status st = made == kProfStages ? SLA_OK : SLA_ERR_CUDA;
+    if (st == SLA_OK) st = run_forward(q, k, v, out, B, H, N, d, blk_q, blk_k, topk, phi, quant, ws, ws_bytes, s, ev);
+    if (st == SLA_OK && cudaEventSynchronize(ev[kProfStages - 1]) != cudaSuccess) st = SLA_ERR_CUDA;
+    if (st == SLA_OK) {
+        for (int i = 0; i + 1 < kProfStages; ++i)
+            if (cudaEventElapsedTime(&stage_ms[i], ev[i], ev[i + 1]) != cudaSuccess) st = SLA_ERR_CUDA;
+        if (cudaEventElapsedTime(&stage_ms[kProfStages - 1], ev[0], ev[kProfStages - 1]) != cudaSuccess)
+            st = SLA_ERR_CUDA;
+    }
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+    return st;
 }
 
 sla_status sla_check(void *ws, void *stream)
