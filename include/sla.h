@@ -121,6 +121,33 @@ SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void
                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                        size_t ws_bytes, void *stream);
 
+/* sla_block_mask for callers that cannot allocate device memory (for example
+ * code inside a framework that owns the whole device-memory budget and hands
+ * out no scratch buffers, or a latency-critical path where cudaMalloc's
+ * implicit synchronisation is not acceptable).  The pages have no counterpart:
+ * this is a deployment variant of the block-mask entry point.
+ *
+ * Same arguments, results and checks as sla_block_mask, without the
+ * workspace: the scratch (block sums, scores, mask rows) lives in one
+ * file-scope device array of sla_block_mask_noalloc_limit() bytes (16 MiB),
+ * which every GPU that loads the library holds until the process exits.
+ * Problems whose scratch would exceed it return SLA_ERR_WORKSPACE before any
+ * launch (about B*H*n_qb*(8*n_kb + 2*n_kb_pad) + 1 KiB*B*H*(n_qb + n_kb)
+ * bytes are needed).  It allocates nothing.
+ *
+ * The first call on a device resolves the array's device address for that
+ * device (cudaGetSymbolAddress, device current); make that first call before
+ * any stream capture.  All calls share the one array: calls whose work
+ * overlaps on the GPU (different streams, or different host threads without
+ * ordering) race on it and must be serialised by the caller.  Nothing in the
+ * array needs to start at zero: every value a call reads it wrote first. */
+SLA_API sla_status sla_block_mask_noalloc(const void *q_bf16, const void *k_bf16, int B, int H, int N, int d,
+                                          int blk_q, int blk_k, float topk, int32_t *idx_out,
+                                          uint32_t *bitmap_out, void *stream);
+
+/* Size in bytes of the static scratch array sla_block_mask_noalloc uses. */
+SLA_API size_t sla_block_mask_noalloc_limit(void);
+
 /* sla_forward with per-stage device timing: enqueues the same launches with a
  * CUDA event between stages, waits for them, and writes 7 floats to the host
  * array stage_ms: milliseconds of {pooling, scores + top-k, quantisation,

@@ -26,7 +26,8 @@ from typing import Optional
 __all__ = [
     "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_forward", "sla_check", "workspace",
-    "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES",
+    "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
+    "sla_block_mask_noalloc_limit",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -58,6 +59,9 @@ lib.sla_forward.restype = _I
 lib.sla_forward_profile.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P,
                                     ctypes.POINTER(ctypes.c_float)]
 lib.sla_forward_profile.restype = _I
+lib.sla_block_mask_noalloc.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]
+lib.sla_block_mask_noalloc.restype = _I
+lib.sla_block_mask_noalloc_limit.restype = _SZ
 lib.sla_check.argtypes = [_P, _P]
 lib.sla_check.restype = _I
 
@@ -126,6 +130,17 @@ def sla_block_mask(q, k, blk_q, blk_k, topk, idx, bitmap, ws, stream=None) -> No
     B, H, N, d = _bhnd(q)
     _ok(lib.sla_block_mask(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, float(topk), _ptr(idx), _ptr(bitmap),
                            _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_block_mask")
+
+
+def sla_block_mask_noalloc(q, k, blk_q, blk_k, topk, idx, bitmap, stream=None) -> None:
+    """sla_block_mask without a workspace (scratch in a fixed static device array)."""
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_block_mask_noalloc(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, float(topk), _ptr(idx),
+                                   _ptr(bitmap), _stream(stream)), "sla_block_mask_noalloc")
+
+
+def sla_block_mask_noalloc_limit() -> int:
+    return int(lib.sla_block_mask_noalloc_limit())
 
 
 def sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws, stream=None) -> None:

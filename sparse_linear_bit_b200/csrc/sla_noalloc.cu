@@ -1,0 +1,85 @@
+// sla_noalloc.cu -- sla_block_mask_noalloc: the block-mask entry point for
+// callers that cannot allocate device memory.
+//
+// sla_block_mask needs scratch memory (block sums, fp64 scores, a status word
+// and the state-reduction mask rows) that its callers pass as a workspace.
+// Some callers cannot provide one: code that runs where no allocation may
+// happen (inside a framework that owns the whole device-memory budget and
+// hands out no raw buffers, or on a latency-critical path where cudaMalloc's
+// implicit device synchronisation is not acceptable).  This variant keeps its
+// scratch in one file-scope device array of fixed size instead, resident on
+// every GPU that loads the library until the process exits.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/sla.h"
+#include "sla_internal.h"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;  // 16 MiB per device
+
+__device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
+
+// Device address of g_scratch per device.  In host code `g_scratch` names a
+// host-side stand-in, so the address must come from cudaGetSymbolAddress with
+// that device current.
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+void *scratch_for_current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess) return nullptr;
+        g_scratch_addr[dev] = p;
+    }
+    return g_scratch_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sla_block_mask_noalloc_limit(void) { return kStaticScratchBytes; }
+
+sla_status sla_block_mask_noalloc(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k,
+                                  float topk, int32_t *idx_out, uint32_t *bitmap_out, void *stream)
+{
+    // same arguments and checks as sla_block_mask, minus the workspace
+    if (B < 1 || H < 1 || N < 1 || d < 1 || blk_q < 1 || blk_k < 1) return SLA_ERR_INVALID_ARG;
+    if (!(topk >= 0.0f && topk <= 1.0f)) return SLA_ERR_INVALID_ARG;
+    if (d != sla::kD || blk_k != sla::kBlkK || (blk_q != 64 && blk_q != 128)) return SLA_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1LL << 24) || (long long)N > (1LL << 24)) return SLA_ERR_UNSUPPORTED;
+    // the scratch the mask path uses is the prefix of the forward's workspace layout, up to the mask rows
+    const sla::Geometry g = sla::make_geometry(B, H, N, d, blk_q, blk_k, topk, 0);
+    const sla::Layout L = sla::make_layout(g);
+    const size_t need = L.amask + (size_t)g.BH * g.n_qb * g.n_kb_pad * sizeof(uint16_t);
+    if (need > kStaticScratchBytes) return SLA_ERR_WORKSPACE;  // problem too large for the static scratch
+    auto misaligned = [](const void *p, uintptr_t a) { return p == nullptr || ((uintptr_t)p & (a - 1)) != 0; };
+    if (misaligned(q, 16) || misaligned(k, 16)) return SLA_ERR_INVALID_ARG;
+    if (g.k_sel > 0 && misaligned(idx_out, 4)) return SLA_ERR_INVALID_ARG;
+    if (bitmap_out && ((uintptr_t)bitmap_out & 3u)) return SLA_ERR_INVALID_ARG;
+    char *scratch = static_cast<char *>(scratch_for_current_device());
+    if (!scratch) return SLA_ERR_CUDA;
+    // the mask stages of the forward, with their scratch in the static array
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    double *qsum = reinterpret_cast<double *>(scratch + L.qsum);
+    double *ksum = reinterpret_cast<double *>(scratch + L.ksum);
+    double *scores = reinterpret_cast<double *>(scratch + L.scores);
+    int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(scratch + L.idx);
+    uint16_t *amask = reinterpret_cast<uint16_t *>(scratch + L.amask);
+    if (sla::launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_scores(qsum, ksum, g, scores, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_topk(scores, g, idx, bitmap_out, amask, s) != cudaSuccess) return SLA_ERR_CUDA;
+    return SLA_OK;
+}
+
+}  // extern "C"
