@@ -164,8 +164,10 @@ SLA_API sla_status sla_check(void *ws, void *stream);
 
 /* Byte offsets of the workspace's internal regions for this problem, for
  * inspection by tests: fills up to `n` entries of `offsets` in the order
- * {status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean,
- *  states, partials, htot, hq, v16} and returns how many regions exist.  A region
+ * {status, qbar, kbar, scores, idx, amask, q8, k8, qscale, kscale, kmean,
+ *  states, partials, htot, hq, v16, kpart} and returns how many regions exist
+ *  (qbar/kbar: fp64 pooled block means; kpart: fp64 partial sums of K for its
+ *  per-channel mean).  A region
  * that a configuration does not use has offset (size_t)-1. */
 SLA_API int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant,
                          size_t *offsets, int n);

@@ -31,8 +31,8 @@ __all__ = [
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
-LAYOUT_REGIONS = ("status", "qsum", "ksum", "scores", "idx", "amask", "q8", "k8", "qscale", "kscale", "kmean",
-                  "states", "partials", "htot", "hq", "v16")
+LAYOUT_REGIONS = ("status", "qbar", "kbar", "scores", "idx", "amask", "q8", "k8", "qscale", "kscale", "kmean",
+                  "states", "partials", "htot", "hq", "v16", "kpart")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(

@@ -46,8 +46,9 @@ Layout make_layout(const Geometry &g)
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
     L.status = take(256);
-    L.qsum = take(BH * g.n_qb * kD * sizeof(double));
-    L.ksum = take(BH * g.n_kb * kD * sizeof(double));
+    L.qbar = take(BH * g.n_qb * kD * sizeof(double));
+    L.kbar = take(BH * g.n_kb * kD * sizeof(double));
+    L.kpart = take(BH * (size_t)pool_parts(g.n_kb) * kD * sizeof(double));
     L.scores = take(BH * g.n_qb * g.n_kb * sizeof(double));
     L.idx = take(BH * g.n_qb * (size_t)(g.k_sel > 0 ? g.k_sel : 1) * sizeof(int32_t));
     L.amask = take(BH * g.n_qb * g.n_kb_pad * sizeof(uint16_t));
@@ -158,10 +159,10 @@ int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float
 {
     if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
     const Layout L = make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant));
-    const size_t v[16] = {L.status, L.qsum,   L.ksum,  L.scores, L.idx,      L.amask, L.q8, L.k8,
-                          L.qscale, L.kscale, L.kmean, L.states, L.partials, L.htot,  L.hq, L.v16};
-    for (int i = 0; i < n && i < 16; ++i) offsets[i] = v[i];
-    return 16;
+    const size_t v[17] = {L.status, L.qbar,  L.kbar,   L.scores,   L.idx,  L.amask, L.q8,  L.k8,   L.qscale,
+                          L.kscale, L.kmean, L.states, L.partials, L.htot, L.hq,    L.v16, L.kpart};
+    for (int i = 0; i < n && i < 17; ++i) offsets[i] = v[i];
+    return 17;
 }
 
 sla_status sla_block_mask(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k, float topk,
@@ -177,12 +178,12 @@ sla_status sla_block_mask(const void *q, const void *k, int B, int H, int N, int
     if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
-    double *qsum = reinterpret_cast<double *>(ws_at(ws, L.qsum));
-    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    double *qbar = reinterpret_cast<double *>(ws_at(ws, L.qbar));
+    double *kbar = reinterpret_cast<double *>(ws_at(ws, L.kbar));
     double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
-    SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
-    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
-    SLA_TRY(launch_scores(qsum, ksum, g, scores, s));
+    SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
+    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, nullptr, s));
+    SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
     int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
     SLA_TRY(launch_topk(scores, g, idx, bitmap_out, reinterpret_cast<uint16_t *>(ws_at(ws, L.amask)), s));
     return SLA_OK;
@@ -204,10 +205,11 @@ sla_status sla_quantize_qk(const void *q, const void *k, int B, int H, int N, in
     if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
-    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    double *kbar = reinterpret_cast<double *>(ws_at(ws, L.kbar));
+    double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
     float *mean = k_mean ? k_mean : reinterpret_cast<float *>(ws_at(ws, L.kmean));
-    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
-    SLA_TRY(launch_kmean(ksum, g.BH, N, g.n_kb, mean, s));
+    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, kpart, s));
+    SLA_TRY(launch_kmean(kpart, g.BH, N, g.n_kb, mean, s));
     SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, s));
     SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, s));
     return SLA_OK;
@@ -234,8 +236,9 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     const Layout L = make_layout(g);
     if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
     int *status = reinterpret_cast<int *>(ws_at(ws, L.status));
-    double *qsum = reinterpret_cast<double *>(ws_at(ws, L.qsum));
-    double *ksum = reinterpret_cast<double *>(ws_at(ws, L.ksum));
+    double *qbar = reinterpret_cast<double *>(ws_at(ws, L.qbar));
+    double *kbar = reinterpret_cast<double *>(ws_at(ws, L.kbar));
+    double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
     double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
     int32_t *idx = reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
     uint16_t *amask = reinterpret_cast<uint16_t *>(ws_at(ws, L.amask));
@@ -254,17 +257,17 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
 
     SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
     mark();
-    // (1) pooled block sums
-    SLA_TRY(launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s));
-    SLA_TRY(launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s));
+    // (1) pooled block means (and the partial sums of K for its per-channel mean)
+    SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
+    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, quant ? kpart : nullptr, s));
     mark();
     // (2) scores + top-k selection
-    SLA_TRY(launch_scores(qsum, ksum, g, scores, s));
+    SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
     SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
     mark();
     // (3) smoothing + INT8 quantisation
     if (quant) {
-        SLA_TRY(launch_kmean(ksum, g.BH, N, g.n_kb, kmean, s));
+        SLA_TRY(launch_kmean(kpart, g.BH, N, g.n_kb, kmean, s));
         SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, s));
         SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, s));
     }

@@ -21,7 +21,7 @@ struct Geometry {
 };
 
 struct Layout {
-    size_t status, qsum, ksum, scores, idx, amask, q8, k8, qscale, kscale, kmean, states, partials, htot, hq, v16;
+    size_t status, qbar, kbar, kpart, scores, idx, amask, q8, k8, qscale, kscale, kmean, states, partials, htot, hq, v16;
     size_t total;
 };
 
@@ -30,9 +30,11 @@ Layout make_layout(const Geometry &g);
 int topk_count(int n_kb, float topk);
 
 // ---- launchers (all asynchronous on `s`; return cudaGetLastError()) ----
-cudaError_t launch_pool_sums(const void *x, int BH, int N, int blk, int nb, double *out, cudaStream_t s);
-cudaError_t launch_kmean(const double *ksum, int BH, int N, int n_kb, float *kmean, cudaStream_t s);
-cudaError_t launch_scores(const double *qsum, const double *ksum, const Geometry &g, double *scores,
+// block means (and, when part != nullptr, per-CTA partial sums for launch_kmean)
+int pool_parts(int nb);
+cudaError_t launch_pool(const void *x, int BH, int N, int blk, int nb, double *mean, double *part, cudaStream_t s);
+cudaError_t launch_kmean(const double *part, int BH, int N, int n_kb, float *kmean, cudaStream_t s);
+cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry &g, double *scores,
                           cudaStream_t s);
 cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap,
                         uint16_t *amask, cudaStream_t s);

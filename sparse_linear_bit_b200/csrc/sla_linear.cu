@@ -243,8 +243,11 @@ __global__ void htot_kernel(const float *__restrict__ partials, int n_chunks, fl
 }
 
 // ---------------------------------------------------------------------------
-// per-query-block state: warp 0 = TMA producer, warp 1 = MMA issuer,
-// warps 2..5 = epilogue (TMEM lanes by warp index % 4)
+// per-query-block state: persistent GEMM over tiles (bh, 256 state columns,
+// 128 query blocks), m fastest so the 5 query-block tiles of one column tile
+// run together and share the state columns through L2.  Warp 0 = TMA producer,
+// warp 1 = MMA issuer, warps 2..5 = epilogue (TMEM lanes by warp index % 4).
+// Two TMEM accumulators: the epilogue of one tile overlaps the next tile's MMAs.
 // ---------------------------------------------------------------------------
 constexpr int kRedStages = 4;
 constexpr int kRedThreads = 192;
@@ -254,25 +257,27 @@ constexpr uint32_t kRedB = 4 * kTileBytes; // 64 key blocks x 256 columns (bf16)
 struct ReduceSmem {
     alignas(1024) uint8_t a[kRedStages][kRedA];
     alignas(1024) uint8_t b[kRedStages][kRedB];
+    float ht[4][256];  // global-state columns of the tile in the epilogue, one copy per epilogue warp
     uint64_t full[kRedStages];
     uint64_t empty[kRedStages];
-    uint64_t done;
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
 };
 
-__global__ void __launch_bounds__(kRedThreads) reduce_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                             const __grid_constant__ CUtensorMap tm_s, int n_qb,
-                                                             int n_kb, int subtract, const float *__restrict__ htot,
-                                                             float *__restrict__ hq, int *status)
+__device__ __forceinline__ uint64_t dadd16(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
+__global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_constant__ CUtensorMap tm_a,
+                                                                const __grid_constant__ CUtensorMap tm_s, int n_qb,
+                                                                int n_kb, int n_tiles, int subtract,
+                                                                const float *__restrict__ htot,
+                                                                float *__restrict__ hq, int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     ReduceSmem &sm = *reinterpret_cast<ReduceSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m_tile = blockIdx.x, n_tile = blockIdx.y, bh = blockIdx.z;
-    const int I0 = m_tile * 128, n0 = n_tile * 256;
-    const int n_valid = min(256, kStateCols - n0);  // 256 or 128
-    const int n_groups = n_valid / 64;
+    const int n_mt = (n_qb + 127) / 128, n_nt = (kStateCols + 255) / 256;
     const int nk = (n_kb + 63) / 64;
     volatile int *abort_flag = &sm.abort_flag;
     if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
@@ -284,71 +289,117 @@ __global__ void __launch_bounds__(kRedThreads) reduce_kernel(const __grid_consta
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.done, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 128);
+        }
+        mbar_init(&sm.drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_s);
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, 256);
+        tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    auto tile_coords = [&](int t, int &bh, int &I0, int &n0) {
+        const int m = t % n_mt, rest = t / n_mt;
+        bh = rest / n_nt;
+        n0 = (rest % n_nt) * 256;
+        I0 = m * 128;
+    };
 
     if (warp == 0 && lane == 0) {
-        int issued = 0;
+        // ------------------------------------------------------------ producer
+        int kc = 0;  // k-steps issued over all tiles of this CTA
         bool ok = true;
-        for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kRedStages, u = kt / kRedStages;
-            if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
-            mbar_expect_tx(&sm.full[s], kRedA + (uint32_t)n_groups * kTileBytes);
-            tma_load_3d(sm.a[s], &tm_a, &sm.full[s], kt * 64, I0, bh);
-            for (int g = 0; g < n_groups; ++g)
-                tma_load_3d(sm.b[s] + g * kTileBytes, &tm_s, &sm.full[s], n0 + 64 * g, kt * 64, bh);
-            issued = kt + 1;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+            int bh, I0, n0;
+            tile_coords(t, bh, I0, n0);
+            const int n_groups = min(256, kStateCols - n0) / 64;
+            for (int kt = 0; kt < nk; ++kt, ++kc) {
+                const int s = kc % kRedStages, u = kc / kRedStages;
+                if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+                mbar_expect_tx(&sm.full[s], kRedA + (uint32_t)n_groups * kTileBytes);
+                tma_load_3d(sm.a[s], &tm_a, &sm.full[s], kt * 64, I0, bh);
+                for (int g = 0; g < n_groups; ++g)
+                    tma_load_3d(sm.b[s] + g * kTileBytes, &tm_s, &sm.full[s], n0 + 64 * g, kt * 64, bh);
+            }
         }
         if (!ok) {  // let in-flight loads land before the CTA exits
             for (int s = 0; s < kRedStages; ++s) {
                 int jl = -1;
-                for (int kt = 0; kt < issued; ++kt)
-                    if (kt % kRedStages == s) jl = kt;
+                for (int j = s; j < kc; j += kRedStages) jl = j;
                 if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedStages) & 1);
             }
         }
     } else if (warp == 1 && lane == 0) {
-        const uint32_t id = idesc(1, 1, 1, 0, 1, 128, (uint32_t)n_valid);  // A K-major, B MN-major
-        for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % kRedStages, u = kt / kRedStages;
-            if (!mbar_wait(&sm.full[s], u & 1, status, abort_flag)) break;
+        // ------------------------------------------------------------ MMA issuer
+        const uint64_t ad0 = sdesc_sw128(smem_u32(sm.a[0]), 16, 1024);
+        const uint64_t bd0 = sdesc_sw128(smem_u32(sm.b[0]), kTileBytes, 1024);
+        int kc = 0, lt = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
+            int bh, I0, n0;
+            tile_coords(t, bh, I0, n0);
+            const uint32_t id = idesc(1, 1, 1, 0, 1, 128, (uint32_t)min(256, kStateCols - n0));  // A K-, B MN-major
+            const int buf = lt & 1;
+            const uint32_t acc = tmem + 256 * buf;
+            if (lt >= 2 && !(ok = mbar_wait(&sm.acc_empty[buf], ((lt >> 1) - 1) & 1, status, abort_flag))) break;
             tc_fence_after();
-            const uint32_t aa = smem_u32(sm.a[s]), ba = smem_u32(sm.b[s]);
+            for (int kt = 0; kt < nk; ++kt, ++kc) {
+                const int s = kc % kRedStages, u = kc / kRedStages;
+                if (!(ok = mbar_wait(&sm.full[s], u & 1, status, abort_flag))) break;
+                tc_fence_after();
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_bf16(tmem, sdesc_sw128(aa + 32 * k, 16, 1024), sdesc_sw128(ba + 2048 * k, kTileBytes, 1024), id,
-                         (kt > 0 || k > 0) ? 1u : 0u);
-            mma_commit(&sm.empty[s]);
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(acc, dadd16(ad0, s * kRedA + 32 * k), dadd16(bd0, s * kRedB + 2048 * k), id,
+                             (kt > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.empty[s]);
+            }
+            if (!ok) break;
+            mma_commit(&sm.acc_full[buf]);
         }
-        mma_commit(&sm.done);
+        mma_commit(&sm.drain);
+        mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
     } else if (warp >= 2) {
+        // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int I = I0 + q * 32 + lane;
-        if (__all_sync(0xffffffffu, mbar_wait(&sm.done, 0, status, abort_flag))) {
+        int lt = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
+            int bh, I0, n0;
+            tile_coords(t, bh, I0, n0);
+            const int n_valid = min(256, kStateCols - n0);
+            const int buf = lt & 1;
+            // global-state columns of this tile (subtract mode), staged per warp so that only
+            // warp-local synchronisation is needed
+            float *ht = sm.ht[q];
+            if (subtract) {
+                __syncwarp();
+                for (int c = lane; c < n_valid; c += 32) ht[c] = __ldg(htot + (size_t)bh * kStateCols + n0 + c);
+                __syncwarp();
+            }
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[buf], (lt >> 1) & 1, status, abort_flag))))
+                break;
             tc_fence_after();
+            const int I = I0 + q * 32 + lane;
             float *dst = hq + ((size_t)bh * n_qb + I) * kStateCols + n0;
-            const float *ht = htot + (size_t)bh * kStateCols + n0;
+            const uint32_t acc = tmem + 256 * buf + ((uint32_t)(q * 32) << 16);
             for (int c0 = 0; c0 < n_valid; c0 += 32) {
                 uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + c0, r);
+                tmem_ld32(acc + c0, r);
                 tmem_wait_ld();
                 if (I < n_qb) {
                     float v[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         float x = __uint_as_float(r[i]);
-                        if (subtract) x = __ldg(ht + c0 + i) - x;
+                        if (subtract) x = ht[c0 + i] - x;
                         v[i] = (n0 + c0 + i < kD * kD) ? to_tf32(x) : x;
                     }
                     float4 *o = reinterpret_cast<float4 *>(dst + c0);
@@ -356,15 +407,16 @@ __global__ void __launch_bounds__(kRedThreads) reduce_kernel(const __grid_consta
                     for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[buf]);
         }
     }
-    if (warp == 1 && lane == 0) mbar_wait_quiet(&sm.done, 0);  // MMAs retired before TMEM is freed
     tc_fence_before();
     __syncthreads();
     __syncwarp();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -417,8 +469,12 @@ cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, c
     const size_t smem = sizeof(ReduceSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((g.n_qb + 127) / 128, (kStateCols + 255) / 256, g.BH);
-    reduce_kernel<<<grid, kRedThreads, smem, s>>>(ta, ts, g.n_qb, g.n_kb, g.subtract ? 1 : 0, htot, hq, status);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_tiles = g.BH * ((g.n_qb + 127) / 128) * ((kStateCols + 255) / 256);
+    reduce_kernel<<<n_tiles < sms ? n_tiles : sms, kRedThreads, smem, s>>>(ta, ts, g.n_qb, g.n_kb, n_tiles,
+                                                                         g.subtract ? 1 : 0, htot, hq, status);
     return cudaGetLastError();
 }
 

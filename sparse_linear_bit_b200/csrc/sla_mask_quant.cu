@@ -1,10 +1,11 @@
 // sla_mask_quant.cu -- block pooling, fp64 block scores, top-k block
 // selection and the smooth-and-quantise step of the SageSLA forward.
 //
-// * Pooling sums each block's bf16 rows in fp64.  Sums of up to 2^17 bf16
-//   values are exact in fp64 unless one (batch, head, channel) spans more than
-//   ~2^29 in magnitude, so block sums (and the per-channel mean used for
-//   smoothing) do not depend on the summation order.
+// * Pooling sums each block's bf16 rows in fp64 and divides by the block's
+//   token count once.  Sums of up to 2^17 bf16 values are exact in fp64 unless
+//   one (batch, head, channel) spans more than ~2^29 in magnitude, so block
+//   sums (and the per-channel mean used for smoothing, summed from per-CTA
+//   partial sums) do not depend on the summation order.
 // * The score of key block J for query block I is the dot product of their
 //   mean rows in fp64, accumulated in channel order with one fused
 //   multiply-add per channel ("TurboDiffusion技术架构解析" §2.1: SLA keeps the
@@ -37,21 +38,25 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8])
 }
 
 // ---------------------------------------------------------------------------
-// pooling: out[bh][J][c] = sum over valid rows of block J of x[bh][t][c]
+// pooling: mean[bh][J][c] = (sum over the valid rows of block J of x[bh][t][c]) / count,
+// and optionally part[bh][chunk][c] = the sum of the block sums of the kPoolBlocks
+// blocks this CTA pools (for the per-channel mean over all tokens).
 // grid (ceil(nb/kPoolBlocks), BH), 256 threads; thread = (row lane, 8-channel group)
 // ---------------------------------------------------------------------------
 constexpr int kPoolBlocks = 8;
 
-__global__ void __launch_bounds__(256) pool_sums_kernel(const uint4 *__restrict__ x, int N, int blk, int nb,
-                                                        double *__restrict__ out)
+__global__ void __launch_bounds__(256) pool_kernel(const uint4 *__restrict__ x, int N, int blk, int nb,
+                                                   double *__restrict__ mean, double *__restrict__ part)
 {
     __shared__ double red[16][kD];
     const int bh = blockIdx.y;
     const int cg = threadIdx.x & 15, rl = threadIdx.x >> 4;
     const uint4 *xh = x + (size_t)bh * N * (kD / 8);
+    double total = 0.0;  // thread c < kD: sum of this CTA's block sums of channel c
     for (int J = blockIdx.x * kPoolBlocks; J < min(nb, (blockIdx.x + 1) * kPoolBlocks); ++J) {
         const int t0 = J * blk, t1 = min(N, t0 + blk);
         double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
         for (int r = t0 + rl; r < t1; r += 16) {
             float f[8];
             bf16x8_to_f32(__ldg(xh + (size_t)r * (kD / 8) + cg), f);
@@ -62,79 +67,95 @@ __global__ void __launch_bounds__(256) pool_sums_kernel(const uint4 *__restrict_
         for (int i = 0; i < 8; ++i) red[rl][cg * 8 + i] = acc[i];
         __syncthreads();
         if (threadIdx.x < kD) {
-            double s = 0.0;
+            double sum = 0.0;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) s += red[r][threadIdx.x];
-            out[((size_t)bh * nb + J) * kD + threadIdx.x] = s;
+            for (int r = 0; r < 16; ++r) sum += red[r][threadIdx.x];
+            mean[((size_t)bh * nb + J) * kD + threadIdx.x] = sum / (double)(t1 - t0);
+            total += sum;
         }
         __syncthreads();
     }
+    if (part && threadIdx.x < kD) part[((size_t)bh * gridDim.x + blockIdx.x) * kD + threadIdx.x] = total;
 }
 
-// kmean[bh][c] = fp32( (sum_J ksum[bh][J][c]) / N )
-__global__ void kmean_kernel(const double *__restrict__ ksum, int N, int n_kb, float *__restrict__ kmean)
+// kmean[bh][c] = fp32( (sum of the pooling partial sums of channel c) / N )
+__global__ void kmean_kernel(const double *__restrict__ part, int n_parts, int N, float *__restrict__ kmean)
 {
     const int bh = blockIdx.x, c = threadIdx.x;
-    const double *p = ksum + (size_t)bh * n_kb * kD + c;
+    const double *p = part + (size_t)bh * n_parts * kD + c;
     double s = 0.0;
-    for (int J = 0; J < n_kb; ++J) s += p[(size_t)J * kD];
+#pragma unroll 8
+    for (int i = 0; i < n_parts; ++i) s += p[(size_t)i * kD];
     kmean[(size_t)bh * kD + c] = (float)(s / (double)N);
 }
 
 // ---------------------------------------------------------------------------
-// scores[bh][I][J] = sum_c fma-chain( qsum[I][c]/nI , ksum[J][c]/nJ )
-// 64 x 64 output tile per CTA, 256 threads x (4 x 4) outputs, channel order kept
+// scores[bh][I][J] = fma chain over channels c = 0..127 of qbar[I][c] * kbar[J][c]
+// 128 x 128 output tile per CTA; 256 threads as 16 x 16, each 8 x 8 outputs at
+// rows 2*ty + {0,1} + 32m and columns 2*tx + {0,1} + 32m (m = 0..3), so each
+// operand read is one 16-byte shared load serving two outputs.  Channels are
+// staged 16 at a time, transposed to [channel][row] in shared memory.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) scores_kernel(const double *__restrict__ qsum, const double *__restrict__ ksum,
-                                                     int N, int blk_q, int blk_k, int n_qb, int n_kb,
-                                                     double *__restrict__ scores)
+constexpr int kScTile = 128;
+constexpr int kScChan = 16;
+
+__global__ void __launch_bounds__(256, 1) scores_kernel(const double *__restrict__ qbar,
+                                                        const double *__restrict__ kbar, int n_qb, int n_kb,
+                                                        double *__restrict__ scores)
 {
-    __shared__ double As[16][64 + 1];
-    __shared__ double Bs[16][64 + 1];
-    const int bh = blockIdx.z, I0 = blockIdx.y * 64, J0 = blockIdx.x * 64;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const double *qh = qsum + (size_t)bh * n_qb * kD;
-    const double *kh = ksum + (size_t)bh * n_kb * kD;
-    double acc[4][4];
+    __shared__ __align__(16) double As[kScChan][kScTile];
+    __shared__ __align__(16) double Bs[kScChan][kScTile];
+    const int bh = blockIdx.z, I0 = blockIdx.y * kScTile, J0 = blockIdx.x * kScTile;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const double *qh = qbar + (size_t)bh * n_qb * kD;
+    const double *kh = kbar + (size_t)bh * n_kb * kD;
+    double acc[8][8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
-    for (int c0 = 0; c0 < kD; c0 += 16) {
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    for (int c0 = 0; c0 < kD; c0 += kScChan) {
+        // 128 rows x 8 channel pairs per operand: thread -> (row = e & 127, pair = e >> 7),
+        // so consecutive threads store consecutive rows of one channel (no bank conflicts)
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
-            const int e = threadIdx.x + 256 * l;  // 0..1023 = 64 rows x 16 channels
-            const int r = e >> 4, c = e & 15;
-            const int I = I0 + r, J = J0 + r;
-            double a = 0.0, b = 0.0;
-            if (I < n_qb) a = qh[(size_t)I * kD + c0 + c] / (double)(min(N, (I + 1) * blk_q) - I * blk_q);
-            if (J < n_kb) b = kh[(size_t)J * kD + c0 + c] / (double)(min(N, (J + 1) * blk_k) - J * blk_k);
-            As[c][r] = a;
-            Bs[c][r] = b;
+            const int e = tid + 256 * l, r = e & 127, c = 2 * (e >> 7);
+            double2 a = make_double2(0.0, 0.0), b = make_double2(0.0, 0.0);
+            if (I0 + r < n_qb) a = __ldg(reinterpret_cast<const double2 *>(qh + (size_t)(I0 + r) * kD + c0 + c));
+            if (J0 + r < n_kb) b = __ldg(reinterpret_cast<const double2 *>(kh + (size_t)(J0 + r) * kD + c0 + c));
+            As[c][r] = a.x;
+            As[c + 1][r] = a.y;
+            Bs[c][r] = b.x;
+            Bs[c + 1][r] = b.y;
         }
         __syncthreads();
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            double a[4], b[4];
+        for (int c = 0; c < kScChan; ++c) {
+            double a[8], b[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = As[c][ty * 4 + i];
+            for (int m = 0; m < 4; ++m) {
+                const double2 av = *reinterpret_cast<const double2 *>(&As[c][2 * ty + 32 * m]);
+                const double2 bv = *reinterpret_cast<const double2 *>(&Bs[c][2 * tx + 32 * m]);
+                a[2 * m] = av.x;
+                a[2 * m + 1] = av.y;
+                b[2 * m] = bv.x;
+                b[2 * m + 1] = bv.y;
+            }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = Bs[c][tx * 4 + j];
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
         }
         __syncthreads();
     }
     double *sh = scores + (size_t)bh * n_qb * n_kb;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int I = I0 + ty * 4 + i;
+    for (int i = 0; i < 8; ++i) {
+        const int I = I0 + 2 * ty + (i & 1) + 32 * (i >> 1);
         if (I >= n_qb) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int J = J0 + tx * 4 + j;
+        for (int j = 0; j < 8; ++j) {
+            const int J = J0 + 2 * tx + (j & 1) + 32 * (j >> 1);
             if (J < n_kb) sh[(size_t)I * n_kb + J] = acc[i][j] + 0.0;  // -0 -> +0
         }
     }
@@ -329,23 +350,25 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
 
 }  // namespace
 
-cudaError_t launch_pool_sums(const void *x, int BH, int N, int blk, int nb, double *out, cudaStream_t s)
+int pool_parts(int nb) { return (nb + kPoolBlocks - 1) / kPoolBlocks; }
+
+cudaError_t launch_pool(const void *x, int BH, int N, int blk, int nb, double *mean, double *part, cudaStream_t s)
 {
-    dim3 grid((nb + kPoolBlocks - 1) / kPoolBlocks, BH);
-    pool_sums_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(x), N, blk, nb, out);
+    dim3 grid(pool_parts(nb), BH);
+    pool_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(x), N, blk, nb, mean, part);
     return cudaGetLastError();
 }
 
-cudaError_t launch_kmean(const double *ksum, int BH, int N, int n_kb, float *kmean, cudaStream_t s)
+cudaError_t launch_kmean(const double *part, int BH, int N, int n_kb, float *kmean, cudaStream_t s)
 {
-    kmean_kernel<<<BH, kD, 0, s>>>(ksum, N, n_kb, kmean);
+    kmean_kernel<<<BH, kD, 0, s>>>(part, pool_parts(n_kb), N, kmean);
     return cudaGetLastError();
 }
 
-cudaError_t launch_scores(const double *qsum, const double *ksum, const Geometry &g, double *scores, cudaStream_t s)
+cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry &g, double *scores, cudaStream_t s)
 {
-    dim3 grid((g.n_kb + 63) / 64, (g.n_qb + 63) / 64, g.BH);
-    scores_kernel<<<grid, 256, 0, s>>>(qsum, ksum, g.N, g.blk_q, g.blk_k, g.n_qb, g.n_kb, scores);
+    dim3 grid((g.n_kb + kScTile - 1) / kScTile, (g.n_qb + kScTile - 1) / kScTile, g.BH);
+    scores_kernel<<<grid, 256, 0, s>>>(qbar, kbar, g.n_qb, g.n_kb, scores);
     return cudaGetLastError();
 }
 

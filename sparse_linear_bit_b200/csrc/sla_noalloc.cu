@@ -70,14 +70,14 @@ sla_status sla_block_mask_noalloc(const void *q, const void *k, int B, int H, in
     if (!scratch) return SLA_ERR_CUDA;
     // the mask stages of the forward, with their scratch in the static array
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    double *qsum = reinterpret_cast<double *>(scratch + L.qsum);
-    double *ksum = reinterpret_cast<double *>(scratch + L.ksum);
+    double *qbar = reinterpret_cast<double *>(scratch + L.qbar);
+    double *kbar = reinterpret_cast<double *>(scratch + L.kbar);
     double *scores = reinterpret_cast<double *>(scratch + L.scores);
     int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(scratch + L.idx);
     uint16_t *amask = reinterpret_cast<uint16_t *>(scratch + L.amask);
-    if (sla::launch_pool_sums(q, g.BH, N, blk_q, g.n_qb, qsum, s) != cudaSuccess) return SLA_ERR_CUDA;
-    if (sla::launch_pool_sums(k, g.BH, N, blk_k, g.n_kb, ksum, s) != cudaSuccess) return SLA_ERR_CUDA;
-    if (sla::launch_scores(qsum, ksum, g, scores, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (sla::launch_scores(qbar, kbar, g, scores, s) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla::launch_topk(scores, g, idx, bitmap_out, amask, s) != cudaSuccess) return SLA_ERR_CUDA;
     return SLA_OK;
 }

@@ -73,7 +73,8 @@ def test_workspace_bytes():
     assert sla.sla_workspace_bytes(0, 40, 75600, 128, 128, 64, 0.1, 1) == 0     # B
     lay = sla.sla_workspace_layout(1, 2, 2048, 128, 64, 64, 0.1, 1)
     offs = [v for v in lay.values() if v is not None]
-    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert len(set(offs)) == len(offs) and all(o % 256 == 0 for o in offs)
+    assert set(lay) == set(sla.LAYOUT_REGIONS)
     assert sla.sla_workspace_layout(1, 2, 2048, 128, 64, 64, 0.1, 0)["q8"] is None
 
 
