@@ -14,20 +14,22 @@
 // accumulator, normalised by phi(q) . Z_I on the CUDA cores; output =
 // sparse + linear, rounded to bf16.
 //
-// Tiling.  Key blocks are processed in selection order, two per S tile: one
-// Q.K^T chain (M=128, N=128, INT8) fills both blocks' logits.  Two softmax
-// warpgroups take one block each (warpgroup g: blocks 2t+g) with their own P,
-// O accumulator and running (max, sum), merged in the epilogue.  The two
+// Tiling.  Key blocks are processed in selection order, loaded two per ring
+// stage.  Two softmax warpgroups take one block each (warpgroup g: blocks
+// 2t+g) with their own S (one M=128, N=64 Q.K^T chain per block), P, O
+// accumulator and running (max, sum), merged in the epilogue; the groups share
+// nothing but Q, the ring and the exponential token, so one group's Q.K^T is
+// issued while the other group is still reading its logits.  The two
 // warps that share an SM sub-partition (same query rows, one per group) pass a
 // token so that their exponential phases alternate: the MUFU unit is the
 // scarcest resource, and one group's exponentials overlap the other group's
 // TMEM loads, row maxima and stores.
 //
 // Issue.  tcgen05 and mbarrier operations cost tens of cycles each on the
-// issuing thread, so issue is spread over three threads: one issues Q.K^T
-// (per tile), one per softmax group issues that group's P.V.  Dependencies go
-// through mbarriers only: S is rewritten once both groups have read it; P of a
-// group is rewritten once that group's previous P.V has completed.
+// issuing thread, so each softmax group has its own issuing thread for its
+// Q.K^T and P.V.  Dependencies go through mbarriers only: S of a group is
+// rewritten once that group has read it; P of a group is rewritten once that
+// group's previous P.V has completed.
 //
 // Shared-memory bandwidth (128 B/clk, shared by TMA writes and tensor-core
 // operand reads): both A operands live in tensor memory -- Q (written once per
@@ -36,10 +38,10 @@
 // pair-stages.  The linear branch runs at the end, reusing the ring for its
 // operands and the S columns for its accumulator.
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 Q.K^T / linear issuer and
+// Roles (384 threads): warp 0 TMA producer, warp 1 linear-branch issuer and
 // TMEM owner, warps 2-5 / 6-9 softmax groups 0 / 1 (one query row per thread,
-// one TMEM lane quarter per warp), warps 10 / 11 P.V issuers of groups 0 / 1.
-// TMEM columns: S [0,128) (group g reads 64g..64g+63; L at the end), P of
+// one TMEM lane quarter per warp), warps 10 / 11 Q.K^T + P.V issuers of groups
+// 0 / 1.  TMEM columns: S of group g at 64g (L over both at the end), P of
 // group g at 128 + 32g, Q at 192, O of group g at 256 + 128g.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -78,7 +80,7 @@ struct AttnSmem {
     float fin[2][3][128];   // epilogue exchange: [group][max, sum, den]
     uint64_t bar_q, bar_h, bar_phiq, bar_lin, drain[3];
     uint64_t full[AttnCfg<QUANT>::kStages], empty[AttnCfg<QUANT>::kStages];
-    uint64_t bar_s, bar_sfree, bar_p[2], bar_pv[2];
+    uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_pv[2];
     uint64_t tok[2][4];     // exponential-phase token per group and lane quarter
     uint32_t tmem_base;
     int abort_flag;
@@ -202,9 +204,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 2);  // one commit from each P.V issuer per tile
         }
-        mbar_init(&sm.bar_s, 1);
-        mbar_init(&sm.bar_sfree, 256);
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_s[b], 1);
+            mbar_init(&sm.bar_sfree[b], 128);
             mbar_init(&sm.bar_p[b], 128);
             mbar_init(&sm.bar_pv[b], 1);
             for (int q = 0; q < 4; ++q) mbar_init(&sm.tok[b][q], 1);
@@ -270,30 +272,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ Q.K^T issuer, then the linear MMA
+        // ------------------------------------------------------------ linear-branch MMA
         if (lane == 0) {
-            constexpr uint32_t id_qk2 = QUANT ? idesc(2, 1, 1, 0, 0, 128, 128) : idesc(1, 1, 1, 0, 0, 128, 128);
-            constexpr uint32_t id_qk1 = QUANT ? idesc(2, 1, 1, 0, 0, 128, 64) : idesc(1, 1, 1, 0, 0, 128, 64);
-            const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
             bool ok = true;
-            if (k_sel > 0) ok = mbar_wait(&sm.bar_q, 0, status, abort_flag);
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                if (!(ok = mbar_wait(&sm.full[t % NS], (t / NS) & 1, status, abort_flag))) break;
-                if (t > 0 && !(ok = mbar_wait(&sm.bar_sfree, (t - 1) & 1, status, abort_flag))) break;
-                tc_fence_after();
-                const uint32_t so = (t % NS) * Cfg::kStageBytes;
-                const uint32_t id = (2 * t + 1 < k_sel) ? id_qk2 : id_qk1;
-                if (QUANT) {  // K-step of 32 int8 = 8 TMEM columns of Q
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(t_s, t_q + 8 * k, dadd(kd0, so + 32 * k), id, k > 0 ? 1u : 0u);
-                } else {  // K-step of 16 bf16 = 8 TMEM columns of Q
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_f16_tmem_a(t_s, t_q + 8 * k, dadd(kd0, so + (k >> 2) * 2 * kBox + 32 * (k & 3)), id,
-                                       k > 0 ? 1u : 0u);
-                }
-                mma_commit(&sm.bar_s);
-            }
             // linear branch: L = phi(Q_I) H_I (tf32) into the S columns, after the softmax groups are done
             if (ok) ok = mbar_wait(&sm.bar_h, 0, status, abort_flag) && mbar_wait(&sm.bar_phiq, 0, status, abort_flag);
             if (ok) {
@@ -311,14 +292,43 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             mbar_wait_quiet(&sm.drain[0], 0);  // this thread's MMAs retired before TMEM is released
         }
     } else if (warp >= 10) {
-        // ------------------------------------------------------------ P.V issuer of group g
+        // ------------------------------------------------------------ Q.K^T + P.V issuer of group g
         const int g = warp - 10;
         if (lane == 0) {
+            constexpr uint32_t id_qk = QUANT ? idesc(2, 1, 1, 0, 0, 128, 64) : idesc(1, 1, 1, 0, 0, 128, 64);
             constexpr uint32_t id_pv = QUANT ? idesc(1, 1, 1, 0, 1, 128, 128) : idesc(1, 0, 0, 0, 1, 128, 128);
+            const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
             const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), 2 * kBox, 1024);
+            const uint32_t s_g = t_s + 64 * g;
+            const int nb = n_blk(g);
             bool ok = true;
+            // S_g = Q K_j^T for this group's block of tile t (K rows of block g of the pair)
+            auto issue_qk = [&](int t) {
+                if (!(ok = mbar_wait(&sm.full[t % NS], (t / NS) & 1, status, abort_flag))) return;
+                if (t > 0 && !(ok = mbar_wait(&sm.bar_sfree[g], (t - 1) & 1, status, abort_flag))) return;
+                tc_fence_after();
+                const uint32_t so = (t % NS) * Cfg::kStageBytes + g * kBox;
+                if (QUANT) {  // K-step of 32 int8 = 8 TMEM columns of Q
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(s_g, t_q + 8 * k, dadd(kd0, so + 32 * k), id_qk, k > 0 ? 1u : 0u);
+                } else {  // K-step of 16 bf16 = 8 TMEM columns of Q
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_f16_tmem_a(s_g, t_q + 8 * k, dadd(kd0, so + (k >> 2) * 2 * kBox + 32 * (k & 3)), id_qk,
+                                       k > 0 ? 1u : 0u);
+                }
+                mma_commit(&sm.bar_s[g]);
+            };
+            if (nb > 0) {
+                ok = mbar_wait(&sm.bar_q, 0, status, abort_flag);
+                if (ok) issue_qk(0);
+            }
             for (int t = 0; ok && t < n_tiles; ++t) {
-                if (t < n_blk(g)) {
+                if (t < nb) {
+                    if (t + 1 < nb) {  // next logits as soon as this group has read S
+                        issue_qk(t + 1);
+                        if (!ok) break;
+                    }
                     if (!(ok = mbar_wait(&sm.bar_p[g], t & 1, status, abort_flag))) break;
                     tc_fence_after();
                     const uint32_t vo = (t % NS) * Cfg::kStageBytes + g * kBox;  // this block's rows of the pair
@@ -328,7 +338,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                                        (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&sm.bar_pv[g]);
                 }
-                mma_commit(&sm.empty[t % NS]);  // stage t free once both groups' P.V have retired
+                mma_commit(&sm.empty[t % NS]);  // stage t free once both groups' MMAs on it have retired
             }
             mma_commit(&sm.drain[1 + g]);
             mbar_wait_quiet(&sm.drain[1 + g], 0);
@@ -392,25 +402,23 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         float ks_a = (QUANT && J_a >= 0) ? __ldg(kscale + (size_t)bh * n_kb + J_a) : 0.0f;
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
-        for (int t = 0; ok && t < n_tiles; ++t) {
+        const int nb = n_blk(g);
+        for (int t = 0; ok && t < nb; ++t) {
             const int J = J_a;
             const float c = QUANT ? sq * ks_a * kscale_log2 : kscale_log2;
-            if (t + 1 < n_tiles) {
+            if (t + 1 < nb) {
                 J_a = J_b;
-                if (QUANT && J_b >= 0) ks_a = __ldg(kscale + (size_t)bh * n_kb + J_b);
+                if (QUANT) ks_a = __ldg(kscale + (size_t)bh * n_kb + J_b);
             }
-            if (t + 2 < n_tiles) J_b = blk_of(t + 2);
-            if (!(ok = wait_all(&sm.bar_s, t & 1))) break;
+            if (t + 2 < nb) J_b = blk_of(t + 2);
+            if (!(ok = wait_all(&sm.bar_s[g], t & 1))) break;
             tc_fence_after();
             uint32_t sv[64];
-            if (J >= 0) {
-                tmem_ld32(s_own, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-                tmem_ld32(s_own + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-                tmem_wait_ld();
-            }
+            tmem_ld32(s_own, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(s_own + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&sm.bar_sfree);  // S may be rewritten once both groups have read it
-            if (J < 0) break;            // last tile of an odd selection: nothing for group 1
+            mbar_arrive(&sm.bar_sfree[g]);  // S_g may be rewritten now
             const int valid = min(64, N - J * 64);
             // the two paths are separate instantiations so the full-tile path carries no masking
             const float tmax = valid == 64 ? tile_max<QUANT, false>(sv, 64, c) : tile_max<QUANT, true>(sv, valid, c);

@@ -34,14 +34,26 @@
 namespace sla {
 namespace {
 
-constexpr int kStatesThreads = 128;
 constexpr uint32_t kTileBytes = 64 * 128;  // one [64 rows x 128 B] TMA box
 
+// ---------------------------------------------------------------------------
+// per-key-block states: persistent, one CTA per SM over (bh, chunk of 32 key
+// blocks) items.  Warp 0 = TMA producer (4 stages of K and V), warp 1 = MMA
+// issuer, warps 2..5 = epilogue (TMEM lane quarter = warp index % 4), warps
+// 6..13 = converters (phi(K) and V to fp16 in place, z_J by warp shuffles).
+// TMEM: two per-block accumulators and two chunk-sum accumulators, so the
+// epilogue of block J overlaps the MMAs of block J+1 and the chunk sum of one
+// item is read while the next item accumulates.  The epilogue writes h_J^T
+// through a swizzled shared stage and TMA tensor stores (one per warp slice).
+// ---------------------------------------------------------------------------
+constexpr int kStatesThreads = 448;
+constexpr int kStStages = 4;
+
 struct StatesSmem {
-    alignas(1024) uint8_t k[2][2][kTileBytes];  // [stage][channel half][64 tokens x 64 ch]
-    alignas(1024) uint8_t v[2][2][kTileBytes];  // [stage][dim half][64 tokens x 64 dims]
-    uint64_t full[2];
-    uint64_t mma_done;
+    alignas(1024) uint8_t kv[kStStages][4][kTileBytes];  // per stage: K channels 0-63, 64-127; V dims 0-63, 64-127
+    alignas(1024) uint8_t out[2][2][2 * kTileBytes];     // [buffer][channel half]: 128 dims x 128 B, SW128
+    uint64_t full[kStStages], conv[kStStages], empty[kStStages];
+    uint64_t acc_full[2], acc_empty[2], sum_full[2], sum_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -50,184 +62,258 @@ struct StatesSmem {
 __device__ __forceinline__ float phi_f(float x, int phi)
 {
     if (phi == 1) return fmaxf(x, 0.0f);
-    return x > 0.0f ? x + 1.0f : expf(x);
+    return x > 0.0f ? x + 1.0f : __expf(x);  // the result is rounded to fp16 next
 }
 
-__global__ void __launch_bounds__(kStatesThreads) states_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                                                const __grid_constant__ CUtensorMap tm_v, int N,
-                                                                int n_kb, int n_chunks, int phi,
-                                                                uint16_t *__restrict__ states,
-                                                                float *__restrict__ partials,
-                                                                uint16_t *__restrict__ v16, int *status)
+__global__ void __launch_bounds__(kStatesThreads, 1) states_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                                   const __grid_constant__ CUtensorMap tm_v,
+                                                                   const __grid_constant__ CUtensorMap tm_out, int N,
+                                                                   int n_kb, int n_chunks, int n_items, int phi,
+                                                                   uint16_t *__restrict__ states,
+                                                                   float *__restrict__ partials,
+                                                                   uint16_t *__restrict__ v16, int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     StatesSmem &sm = *reinterpret_cast<StatesSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int bh = blockIdx.y, chunk = blockIdx.x;
-    const int Jbeg = chunk * kStateChunk, nJ = min(kStateChunk, n_kb - Jbeg);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     volatile int *abort_flag = &sm.abort_flag;
     if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
     __syncthreads();
     if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
 
     if (tid == 0) {
-        mbar_init(&sm.full[0], 1);
-        mbar_init(&sm.full[1], 1);
-        mbar_init(&sm.mma_done, 1);
+        for (int s = 0; s < kStStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.conv[s], 256);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 128);
+            mbar_init(&sm.sum_full[b], 1);
+            mbar_init(&sm.sum_empty[b], 128);
+        }
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_out);
     }
     __syncwarp();
-    if (warp == 0) {
-        tmem_alloc(&sm.tmem_base, 256);
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sm.tmem_base;
-    const uint32_t d_blk = tmem, d_sum = tmem + 128;
-    constexpr uint32_t kIdesc = idesc(1, 0, 0, 1, 1, 128, 128);  // f32 <- f16 (MN) x f16 (MN)
+    const uint32_t tmem = sm.tmem_base;  // [0,256): block accumulators, [256,512): chunk sums
 
-    auto issue = [&](int j) {
-        const int s = j & 1, J = Jbeg + j;
-        mbar_expect_tx(&sm.full[s], 4 * kTileBytes);
-        tma_load_3d(sm.k[s][0], &tm_k, &sm.full[s], 0, J * 64, bh);
-        tma_load_3d(sm.k[s][1], &tm_k, &sm.full[s], 64, J * 64, bh);
-        tma_load_3d(sm.v[s][0], &tm_v, &sm.full[s], 0, J * 64, bh);
-        tma_load_3d(sm.v[s][1], &tm_v, &sm.full[s], 64, J * 64, bh);
-    };
-    int issued = 0;
-    if (tid == 0) {
-        for (; issued < min(2, nJ); ++issued) issue(issued);
-    }
-
-    float zsum = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < nJ && ok; ++j) {
-        const int s = j & 1, J = Jbeg + j;
-        ok = __syncthreads_and(mbar_wait(&sm.full[s], (j >> 1) & 1, status, abort_flag));
-        if (!ok) break;
-        // phi(K) and V to fp16 in place (elementwise, so the swizzle permutation
-        // is irrelevant); tokens past N contribute nothing
-        const int valid = min(64, N - J * 64);
-#pragma unroll 2
-        for (int l = 0; l < 16; ++l) {
-            const int e = tid + kStatesThreads * l;  // 16-byte chunk 0..2047: K halves, then V halves
-            const bool is_v = e >= 1024;
-            const int e2 = e & 1023, half = e2 >> 9, row = (e2 & 511) >> 3;
-            uint8_t *tile = is_v ? sm.v[s][half] : sm.k[s][half];
-            uint4 *p = reinterpret_cast<uint4 *>(tile + (e2 & 511) * 16);
-            uint4 w = *p;
-            uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float a = __uint_as_float(ww[i] << 16), b = __uint_as_float(ww[i] & 0xFFFF0000u);
-                if (!is_v) {
-                    a = phi_f(a, phi);
-                    b = phi_f(b, phi);
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int j = 0;  // blocks issued by this CTA
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+                const int bh = it / n_chunks, Jbeg = (it % n_chunks) * kStateChunk;
+                const int nJ = min(kStateChunk, n_kb - Jbeg);
+                for (int jj = 0; jj < nJ; ++jj, ++j) {
+                    const int s = j % kStStages, u = j / kStStages, row = (Jbeg + jj) * 64;
+                    if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+                    mbar_expect_tx(&sm.full[s], 4 * kTileBytes);
+                    tma_load_3d(sm.kv[s][0], &tm_k, &sm.full[s], 0, row, bh);
+                    tma_load_3d(sm.kv[s][1], &tm_k, &sm.full[s], 64, row, bh);
+                    tma_load_3d(sm.kv[s][2], &tm_v, &sm.full[s], 0, row, bh);
+                    tma_load_3d(sm.kv[s][3], &tm_v, &sm.full[s], 64, row, bh);
                 }
-                ww[i] = row < valid ? pack_f16x2_sat(a, b) : 0u;
             }
-            *p = make_uint4(ww[0], ww[1], ww[2], ww[3]);
-            if (is_v && v16 != nullptr && row < valid) {
-                // un-swizzled fp16 copy of V: chunk (e2 & 7) of this row holds logical chunk ^ (row & 7)
-                const int u = (e2 & 7) ^ (row & 7);
-                *reinterpret_cast<uint4 *>(v16 + (((size_t)bh * N + J * 64 + row) * kD + half * 64 + u * 8)) =
-                    make_uint4(ww[0], ww[1], ww[2], ww[3]);
+            if (!ok) {  // loads in flight land before the CTA exits
+                for (int s = 0; s < kStStages; ++s) {
+                    int jl = -1;
+                    for (int x = s; x < j; x += kStStages) jl = x;
+                    if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kStStages) & 1);
+                }
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdesc = idesc(1, 0, 0, 1, 1, 128, 128);  // f32 <- f16 (MN) x f16 (MN)
+            const uint64_t vd0 = sdesc_sw128(smem_u32(sm.kv[0][2]), kTileBytes, 1024);  // A = V^T (dims x tokens)
+            const uint64_t kd0 = sdesc_sw128(smem_u32(sm.kv[0][0]), kTileBytes, 1024);  // B = phi(K) (ch x tokens)
+            constexpr uint32_t kStage16 = 4 * kTileBytes >> 4;
+            int j = 0, li = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+                const int Jbeg = (it % n_chunks) * kStateChunk, nJ = min(kStateChunk, n_kb - Jbeg);
+                const int cb = li & 1;
+                const uint32_t d_sum = tmem + 256 + 128 * cb;
+                if (li >= 2 && !(ok = mbar_wait(&sm.sum_empty[cb], ((li >> 1) - 1) & 1, status, abort_flag))) break;
+                for (int jj = 0; jj < nJ; ++jj, ++j) {
+                    const int s = j % kStStages, b = j & 1;
+                    const uint32_t d_blk = tmem + 128 * b;
+                    if (j >= 2 && !(ok = mbar_wait(&sm.acc_empty[b], ((j >> 1) - 1) & 1, status, abort_flag))) break;
+                    if (!(ok = mbar_wait(&sm.conv[s], (j / kStStages) & 1, status, abort_flag))) break;
+                    tc_fence_after();
+                    const uint64_t vd = vd0 + (uint64_t)(s * kStage16), kd = kd0 + (uint64_t)(s * kStage16);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_bf16(d_blk, vd + 128 * k, kd + 128 * k, kIdesc, k > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(d_sum, vd + 128 * k, kd + 128 * k, kIdesc, (jj > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(&sm.empty[s]);
+                    mma_commit(&sm.acc_full[b]);
+                    if (jj == nJ - 1) mma_commit(&sm.sum_full[cb]);
+                }
+            }
+            mma_commit(&sm.drain);
+            mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3, d = 32 * q + lane;  // TMEM lane = dim row of h_J^T
+        int j = 0, li = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+            const int bh = it / n_chunks, chunk = it % n_chunks, Jbeg = chunk * kStateChunk;
+            const int nJ = min(kStateChunk, n_kb - Jbeg), cb = li & 1;
+            for (int jj = 0; jj < nJ; ++jj, ++j) {
+                const int b = j & 1;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], (j >> 1) & 1, status, abort_flag))))
+                    break;
+                tc_fence_after();
+                if (lane == 0) bulk_wait_read<1>();  // the store issued from this buffer two blocks ago has read it
+                __syncwarp();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {  // channel half: two 32-column loads, one wait
+                    uint32_t r[64];
+                    const uint32_t ta = tmem + 128 * b + ((uint32_t)(32 * q) << 16) + 64 * hh;
+                    tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                    tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                    tmem_wait_ld();
+                    uint8_t *row = sm.out[b][hh] + d * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        *reinterpret_cast<uint4 *>(row + ((u ^ (d & 7)) << 4)) =
+                            make_uint4(pack_bf16x2(__uint_as_float(r[8 * u]), __uint_as_float(r[8 * u + 1])),
+                                       pack_bf16x2(__uint_as_float(r[8 * u + 2]), __uint_as_float(r[8 * u + 3])),
+                                       pack_bf16x2(__uint_as_float(r[8 * u + 4]), __uint_as_float(r[8 * u + 5])),
+                                       pack_bf16x2(__uint_as_float(r[8 * u + 6]), __uint_as_float(r[8 * u + 7])));
+                }
+                tc_fence_before();
+                mbar_arrive(&sm.acc_empty[b]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int blk = bh * n_kb + Jbeg + jj;
+                    tma_store_3d(&tm_out, sm.out[b][0] + 32 * q * 128, 0, 32 * q, blk);
+                    tma_store_3d(&tm_out, sm.out[b][1] + 32 * q * 128, 64, 32 * q, blk);
+                    bulk_commit();
+                }
+            }
+            if (!ok) break;
+            // chunk sum of the fp32 states
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.sum_full[cb], (li >> 1) & 1, status, abort_flag))))
+                break;
             tc_fence_after();
-            const uint32_t ka = smem_u32(sm.k[s][0]), va = smem_u32(sm.v[s][0]);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = sdesc_sw128(va + 2048 * k, kTileBytes, 1024);  // A = V^T (dims x tokens)
-                const uint64_t bd = sdesc_sw128(ka + 2048 * k, kTileBytes, 1024);  // B = phi(K) (ch x tokens)
-                mma_bf16(d_blk, ad, bd, kIdesc, k > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t ad = sdesc_sw128(va + 2048 * k, kTileBytes, 1024);
-                const uint64_t bd = sdesc_sw128(ka + 2048 * k, kTileBytes, 1024);
-                mma_bf16(d_sum, ad, bd, kIdesc, (j > 0 || k > 0) ? 1u : 0u);
-            }
-            mma_commit(&sm.mma_done);
-        }
-        // z_J[c] = sum over tokens of phi(K)[t][c] (thread = channel), row order
-        {
-            const int c = tid, half = c >> 6, u = (c & 63) >> 3, el = c & 7;
-            const uint8_t *base = sm.k[s][half];
-            float z = 0.0f;
-            for (int r = 0; r < 64; ++r) {
-                const __half b = *reinterpret_cast<const __half *>(base + sw128_off(r, u) + el * 2);
-                z += __half2float(b);
-            }
-            zsum += z;
-            const __nv_bfloat16 zb = __float2bfloat16_rn(z);
-            states[((size_t)bh * n_kb + J) * kStateCols + kD * kD + c] = *reinterpret_cast<const uint16_t *>(&zb);
-        }
-        ok = __syncthreads_and(mbar_wait(&sm.mma_done, j & 1, status, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        // epilogue: thread = dim row d of hT_J (TMEM lane), 128 channel columns
-        {
-            const int d = tid;
-            uint16_t *dst = states + ((size_t)bh * n_kb + J) * kStateCols + (size_t)d * kD;
+            float *dst = partials + ((size_t)bh * n_chunks + chunk) * kStateCols + (size_t)d * kD;
 #pragma unroll 1
             for (int c0 = 0; c0 < kD; c0 += 32) {
                 uint32_t r[32];
-                tmem_ld32(d_blk + ((uint32_t)(warp * 32) << 16) + c0, r);
+                tmem_ld32(tmem + 256 + 128 * cb + ((uint32_t)(32 * q) << 16) + c0, r);
                 tmem_wait_ld();
-                uint32_t pk[16];
+                float4 *o = reinterpret_cast<float4 *>(dst + c0);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                uint4 *o = reinterpret_cast<uint4 *>(dst + c0);
+                for (int i = 0; i < 8; ++i)
+                    o[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.sum_empty[cb]);
+        }
+        if (lane == 0) bulk_wait<0>();  // stores complete before shared memory is released
+    } else {
+        // ------------------------------------------------------------ converters
+        // thread -> (channel half, 16-byte unit u, row group rg): rows rg + 16i of unit u,
+        // whose swizzled position is u ^ (rg & 7); lanes rg = 0..15 reduce z by shuffles
+        const int ct = tid - 192, cw = ct >> 5, rg = lane & 15;
+        const int half = cw >> 2, u = (cw & 3) * 2 + (lane >> 4);
+        const int ch0 = half * 64 + u * 8;  // first of this thread's 8 channels
+        const uint32_t off0 = rg * 128 + ((u ^ (rg & 7)) << 4);
+        int j = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            const int bh = it / n_chunks, chunk = it % n_chunks, Jbeg = chunk * kStateChunk;
+            const int nJ = min(kStateChunk, n_kb - Jbeg);
+            float zc[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // chunk sums of z (lanes rg == 0)
+            for (int jj = 0; jj < nJ; ++jj, ++j) {
+                const int s = j % kStStages, J = Jbeg + jj;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[s], (j / kStStages) & 1, status, abort_flag))))
+                    break;
+                const int valid = min(64, N - J * 64);  // tokens past N contribute nothing
+                float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                uint4 wk[4], wv[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) o[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    wk[i] = *reinterpret_cast<const uint4 *>(sm.kv[s][half] + off0 + i * 2048);
+                    wv[i] = *reinterpret_cast<const uint4 *>(sm.kv[s][2 + half] + off0 + i * 2048);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int r = rg + 16 * i;
+                    const uint32_t kk[4] = {wk[i].x, wk[i].y, wk[i].z, wk[i].w};
+                    const uint32_t vv[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+                    uint32_t ok4[4], ov4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a = phi_f(__uint_as_float(kk[e] << 16), phi);
+                        const float c = phi_f(__uint_as_float(kk[e] & 0xFFFF0000u), phi);
+                        ok4[e] = r < valid ? pack_f16x2_sat(a, c) : 0u;
+                        ov4[e] = r < valid ? pack_f16x2_sat(__uint_as_float(vv[e] << 16),
+                                                            __uint_as_float(vv[e] & 0xFFFF0000u))
+                                           : 0u;
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ok4[e]));
+                        z[2 * e] += f.x;
+                        z[2 * e + 1] += f.y;
+                    }
+                    *reinterpret_cast<uint4 *>(sm.kv[s][half] + off0 + i * 2048) =
+                        make_uint4(ok4[0], ok4[1], ok4[2], ok4[3]);
+                    *reinterpret_cast<uint4 *>(sm.kv[s][2 + half] + off0 + i * 2048) =
+                        make_uint4(ov4[0], ov4[1], ov4[2], ov4[3]);
+                    if (v16 != nullptr && r < valid)  // fp16 copy of V for the attention kernel's fp16 P.V
+                        *reinterpret_cast<uint4 *>(v16 + ((size_t)bh * N + J * 64 + r) * kD + ch0) =
+                            make_uint4(ov4[0], ov4[1], ov4[2], ov4[3]);
+                }
+                fence_async_smem();
+                mbar_arrive(&sm.conv[s]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+#pragma unroll
+                    for (int o = 1; o < 16; o <<= 1) z[e] += __shfl_xor_sync(0xffffffffu, z[e], o);
+                }
+                if (rg == 0) {
+                    *reinterpret_cast<uint4 *>(states + ((size_t)bh * n_kb + J) * kStateCols + kD * kD + ch0) =
+                        make_uint4(pack_bf16x2(z[0], z[1]), pack_bf16x2(z[2], z[3]), pack_bf16x2(z[4], z[5]),
+                                   pack_bf16x2(z[6], z[7]));
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) zc[e] += z[e];
+                }
+            }
+            if (!ok) break;
+            if (rg == 0) {
+                float4 *o = reinterpret_cast<float4 *>(partials + ((size_t)bh * n_chunks + chunk) * kStateCols +
+                                                       kD * kD + ch0);
+                o[0] = make_float4(zc[0], zc[1], zc[2], zc[3]);
+                o[1] = make_float4(zc[4], zc[5], zc[6], zc[7]);
             }
         }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0 && issued < nJ) issue(issued++);
-    }
-    // chunk sum of the fp32 states
-    if (ok && nJ > 0) {
-        const int d = tid;
-        float *dst = partials + ((size_t)bh * n_chunks + chunk) * kStateCols;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kD; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(d_sum + ((uint32_t)(warp * 32) << 16) + c0, r);
-            tmem_wait_ld();
-            float4 *o = reinterpret_cast<float4 *>(dst + (size_t)d * kD + c0);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                o[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-        }
-        dst[kD * kD + tid] = zsum;
-    }
-    if (!ok && tid == 0) {
-        // drain: loads and MMAs still in flight retire before shared memory / TMEM are released
-        for (int s = 0; s < 2; ++s) {
-            const int jl = issued - 1 - ((issued - 1 - s) & 1);  // last load issued on stage s
-            if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl >> 1) & 1);
-        }
-        mma_commit(&sm.drain);
-        mbar_wait_quiet(&sm.drain, 0);
     }
     tc_fence_before();
     __syncthreads();
     __syncwarp();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -425,19 +511,29 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_con
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states, float *partials,
                           uint16_t *v16, int *status, cudaStream_t s)
 {
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, to;
     const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
     const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
     const uint32_t box[3] = {64, 64, 1};
     if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box)) return cudaErrorInvalidValue;
     if (!encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, strides, box)) return cudaErrorInvalidValue;
-    // at most two CTAs per SM: each holds 256 of the SM's 512 TMEM columns
-    const size_t smem = sizeof(StatesSmem) + 1024 > 100 * 1024 ? sizeof(StatesSmem) + 1024 : 100 * 1024;
+    {
+        // h_J^T of every key block: [BH * n_kb][128 dims][128 channels] inside rows of kStateCols
+        const uint64_t od[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)g.BH * g.n_kb};
+        const uint64_t os[2] = {(uint64_t)kD * 2, (uint64_t)kStateCols * 2};
+        const uint32_t ob[3] = {64, 32, 1};
+        if (!encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, states, od, os, ob)) return cudaErrorInvalidValue;
+    }
+    const size_t smem = sizeof(StatesSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(g.n_chunks, g.BH);
-    states_kernel<<<grid, kStatesThreads, smem, s>>>(tk, tv, g.N, g.n_kb, g.n_chunks, phi, states, partials, v16,
-                                                     status);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int n_items = g.BH * g.n_chunks;
+    states_kernel<<<n_items < sms ? n_items : sms, kStatesThreads, smem, s>>>(tk, tv, to, g.N, g.n_kb, g.n_chunks,
+                                                                             n_items, phi, states, partials, v16,
+                                                                             status);
     return cudaGetLastError();
 }
 

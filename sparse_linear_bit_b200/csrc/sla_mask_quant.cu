@@ -293,33 +293,54 @@ __global__ void zero_u32_kernel(uint32_t *p, size_t n)
 }
 
 // ---------------------------------------------------------------------------
-// quantisation: one CTA per block, 256 threads; SMOOTH subtracts mean[c]
+// quantisation: one CTA per block, 256 threads; SMOOTH subtracts mean[c].
+// The block stays in registers as packed bf16 (the values are re-expanded for
+// the second pass), which keeps the kernel at full occupancy.
+//
+// Codes: c = clamp(rint(fl(x / s)), -127, 127) with fl the IEEE fp32 quotient.
+// Instead of a division per element, t = fl(x * r) with r = fl(1 / s) is
+// used: |t - x/s| <= |x/s| (2^-24 + 2^-24 + 2^-48) and |fl(x/s) - x/s| <=
+// |x/s| 2^-24, so for |x/s| <= 128 (|x| <= amax = 127 s, up to rounding)
+// |t - fl(x/s)| < 2.3e-5.  Unless t lies within 2^-14 of a half-integer, no
+// rounding boundary of rint separates t from fl(x/s) and rint(t) is the
+// code; otherwise (about 1 element in 8000) the IEEE quotient is taken.
 // ---------------------------------------------------------------------------
 template <bool SMOOTH, int BLK>
 __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
                                                     const float *__restrict__ mean, uint2 *__restrict__ out,
                                                     float *__restrict__ scale)
 {
-    constexpr int kVec = BLK * (kD / 8) / 256;  // uint4 loads per thread
+    constexpr int kVec = BLK * (kD / 8) / 256;  // uint4 per thread
     __shared__ float warp_max[8];
     const int bh = blockIdx.y, J = blockIdx.x;
     const int t0 = J * BLK;
     const int rows = min(BLK, N - t0);
+    const int cg = threadIdx.x & 15;  // the thread's 8-channel group (same for every l)
     const uint4 *xb = x + ((size_t)bh * N + t0) * (kD / 8);
-    float v[kVec][8];
-    float amax = 0.0f;
+    float mu[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mu[i] = SMOOTH ? __ldg(mean + (size_t)bh * kD + cg * 8 + i) : 0.0f;
+    uint4 raw[kVec];
 #pragma unroll
     for (int l = 0; l < kVec; ++l) {
         const int e = threadIdx.x + 256 * l;  // uint4 index within block: row = e/16, chunk = e%16
-        const int r = e >> 4, cg = e & 15;
-        if (r < rows) {
-            bf16x8_to_f32(__ldg(xb + e), v[l]);
-            if (SMOOTH) {
+        raw[l] = (e >> 4) < rows ? __ldg(xb + e) : make_uint4(0, 0, 0, 0);
+    }
+    auto expand = [&](const uint4 &u, float (&f)[8]) {
+        bf16x8_to_f32(u, f);
+        if (SMOOTH) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[l][i] = __fsub_rn(v[l][i], __ldg(mean + (size_t)bh * kD + cg * 8 + i));
-            }
+            for (int i = 0; i < 8; ++i) f[i] = __fsub_rn(f[i], mu[i]);
+        }
+    };
+    float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[l][i]));
+    for (int l = 0; l < kVec; ++l) {
+        if (((threadIdx.x + 256 * l) >> 4) < rows) {
+            float f[8];
+            expand(raw[l], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
         }
     }
 #pragma unroll
@@ -331,16 +352,26 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
     const float s = __fdiv_rn(amax, 127.0f);
     if (threadIdx.x == 0) scale[(size_t)bh * nb + J] = s;
+    const float r = s != 0.0f ? __fdiv_rn(1.0f, s) : 0.0f;
+    const bool fast = s != 0.0f && isfinite(r);
     uint2 *ob = out + ((size_t)bh * N + t0) * (kD / 8);
 #pragma unroll
     for (int l = 0; l < kVec; ++l) {
         const int e = threadIdx.x + 256 * l;
         if ((e >> 4) < rows) {
+            float f[8];
+            expand(raw[l], f);
             uint32_t w[2] = {0, 0};
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 int c = 0;
-                if (s != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(v[l][i], s))));
+                if (s != 0.0f) {
+                    const float t = f[i] * r;
+                    const float rt = rintf(t);
+                    float q = rt;
+                    if (!fast || fabsf(t - rt) > 0.5f - 6.103515625e-05f) q = rintf(__fdiv_rn(f[i], s));
+                    c = max(-127, min(127, __float2int_rn(q)));
+                }
                 w[i >> 2] |= ((uint32_t)(c & 0xFF)) << (8 * (i & 3));
             }
             ob[e] = make_uint2(w[0], w[1]);

@@ -106,6 +106,40 @@ def test_quantize_bit_exact(blk_q, grid, H, adv):
     assert np.array_equal(k8.cpu().numpy(), k8o)
 
 
+@pytest.mark.parametrize("N", [2048, 1000])
+def test_quantize_half_integer_quotients(N):
+    """Every quotient x/s an exact half-integer (s = 1): codes must round half to even, like
+    the IEEE fp32 quotient followed by rint in the oracle.  K is built from +-pairs per channel
+    so that its smoothing mean is exactly 0 and K - mean keeps the half-integers."""
+    rng = np.random.default_rng(11)
+    B, H, d = 1, 2, 128
+    qv = rng.integers(-254, 255, size=(B, H, N, d)) / 2.0
+    qv[:, :, ::64, 0] = 127.0  # every block of 64 or 128 rows reaches amax = 127, so s = 1
+    half = rng.integers(-254, 255, size=(B, H, N // 2, d)) / 2.0
+    half[:, :, ::32, 1] = 127.0
+    kv = np.empty((B, H, N, d))
+    kv[:, :, 0::2] = half
+    kv[:, :, 1::2] = -half
+    q = synth.f64_to_bf16_bits(qv)
+    k = synth.f64_to_bf16_bits(kv)
+    for blk_q in (64, 128):
+        n_qb, n_kb = -(-N // blk_q), -(-N // 64)
+        q8o, k8o, sqo, sko, kmo = oracle.quantize(q, k, blk_q, 64)
+        assert np.all(kmo == 0.0) and np.all(sqo == 1.0) and np.all(sko == 1.0)
+        qd, kd = to_dev(q, torch), to_dev(k, torch)
+        q8 = torch.empty(q.shape, dtype=torch.int8, device="cuda")
+        k8 = torch.empty(q.shape, dtype=torch.int8, device="cuda")
+        sq = torch.empty((B, H, n_qb), dtype=torch.float32, device="cuda")
+        sk = torch.empty((B, H, n_kb), dtype=torch.float32, device="cuda")
+        ws = sla.workspace(B, H, N, d, blk_q, 64, 0.0, 1)
+        sla.sla_quantize_qk(qd, kd, blk_q, 64, q8, k8, sq, sk, None, ws)
+        sla.sla_check(ws)
+        assert np.array_equal(q8.cpu().numpy(), q8o)
+        assert np.array_equal(k8.cpu().numpy(), k8o)
+        # the half-integers really were rounded half to even
+        assert np.array_equal(q8o.astype(np.float64), np.clip(np.round(qv), -127, 127))
+
+
 FWD_CASES = {
     # name: ((B, H, grid), blk_q, topk, phi, quant)
     "tiny_quant_elu": ((1, 2, (8, 16, 16)), 64, 0.1, 0, 1),
