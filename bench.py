@@ -12,9 +12,14 @@ needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--topk T] [--quant 0|1]
     python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
 
-Multi-GPU (launched with torch.distributed.run, one rank per GPU): every rank
-runs the full workload on its own GPU (weak scaling, no data-path collective;
-heads are independent).  Rank 0 prints one JSON line.
+Multi-GPU (launched with torch.distributed.run, one rank per GPU), no data-path
+collective since every (batch, head) is independent:
+  --scaling weak   (default) every rank runs the whole workload as its own batch
+                   element; the job grows with the number of GPUs.
+  --scaling strong the workload's B*H heads are split into contiguous ranges, one
+                   per rank (sparse_linear_bit_b200.head_shard).
+Times are taken on the device and the max over ranks is reported.  Rank 0
+prints one JSON line.
 """
 from __future__ import annotations
 
@@ -55,7 +60,19 @@ def parse():
     ap.add_argument("--phi", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"])
     return ap.parse_args()
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """Max of a per-rank scalar (a device-timed duration) over all ranks."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def dense_equiv_ops(B, H, N, d):
@@ -250,12 +267,20 @@ def main():
         dist.barrier()
         if rank != 0:
             q, k, v = (np.load(shm + f"_{nm}.npy") for nm in ("q", "k", "v"))
+    # ---- this rank's share: the whole workload (weak) or a contiguous head range (strong)
+    ops_job = dense_equiv_ops(w.B, w.H, w.N, w.d) * (world if a.scaling == "weak" else 1)
+    wl = w
+    if a.scaling == "strong" and world > 1:
+        first, count = sla.head_shard(w.B, w.H, world, rank)
+        q, k, v = (np.ascontiguousarray(sla.shard_heads(x, world, rank)) for x in (q, k, v))
+        wl = synth.Workload(w.name, 1, count, w.grid, d=w.d, blk_q=w.blk_q, blk_k=w.blk_k, topk=a.topk, phi=a.phi,
+                            quant=a.quant, seed=w.seed)
     to_dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     out = torch.empty_like(qd)
-    ws = sla.workspace(w.B, w.H, w.N, w.d, w.blk_q, w.blk_k, a.topk, a.quant, device=dev)
+    ws = sla.workspace(wl.B, wl.H, wl.N, wl.d, wl.blk_q, wl.blk_k, a.topk, a.quant, device=dev)
     stream = torch.cuda.current_stream(dev)
-    fwd = lambda: sla.sla_forward(qd, kd, vd, out, w.blk_q, w.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
+    fwd = lambda: sla.sla_forward(qd, kd, vd, out, wl.blk_q, wl.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
 
     for _ in range(max(3, a.warmup)):
         fwd()
@@ -264,7 +289,7 @@ def main():
     # ---- per-stage device times (CUDA events between the stages, same stream)
     stage = {n: [] for n in sla.PROFILE_STAGES}
     for _ in range(min(5, max(1, a.steps))):
-        r = sla.sla_forward_profile(qd, kd, vd, out, w.blk_q, w.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
+        r = sla.sla_forward_profile(qd, kd, vd, out, wl.blk_q, wl.blk_k, a.topk, a.phi, a.quant, ws, stream=stream)
         for n_, t_ in r.items():
             stage[n_].append(t_)
     stage_ms = {n_: float(np.median(t_)) for n_, t_ in stage.items()}
@@ -287,13 +312,9 @@ def main():
     if world > 1:
         dist.barrier()
     sla.sla_check(ws, stream=stream)
-    ms = e0.elapsed_time(e1) / a.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    ops = dense_equiv_ops(w.B, w.H, w.N, w.d)
-    value = world * ops / (ms * 1e-3) / 1e12
+    ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dev, world)
+    ops = dense_equiv_ops(wl.B, wl.H, wl.N, wl.d)  # this rank's share
+    value = ops_job / (ms * 1e-3) / 1e12
 
     # ---- end to end through the same call: pinned host Q/K/V in, bf16 out back to pinned host
     e2e = None
@@ -319,13 +340,9 @@ def main():
             e2e_step()
         f1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = f0.elapsed_time(f1) / steps_e2e
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1) / steps_e2e, dev, world)
         nbytes = qd.numel() * 2
-        e2e = {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
+        e2e = {"value": ops_job / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
                "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes,
                "note": "host->device copy of Q, K, V from pinned memory, sla_forward, output copied back"}
 
@@ -333,13 +350,13 @@ def main():
     peaks, peak_kind = load_peaks()
     n_kb = -(-w.N // w.blk_k)
     k_sel = sla.sla_topk_count(n_kb, a.topk)
-    lay = sla.sla_workspace_layout(w.B, w.H, w.N, w.d, w.blk_q, w.blk_k, a.topk, a.quant)
+    lay = sla.sla_workspace_layout(wl.B, wl.H, wl.N, wl.d, wl.blk_q, wl.blk_k, a.topk, a.quant)
     n_qb = -(-w.N // w.blk_q)
-    idx = ws[lay["idx"]:lay["idx"] + w.B * w.H * n_qb * max(k_sel, 1) * 4].cpu().numpy().view(np.int32)
-    idx = idx.reshape(w.B * w.H, n_qb, max(k_sel, 1))[..., :k_sel]
+    idx = ws[lay["idx"]:lay["idx"] + wl.B * wl.H * n_qb * max(k_sel, 1) * 4].cpu().numpy().view(np.int32)
+    idx = idx.reshape(wl.B * wl.H, n_qb, max(k_sel, 1))[..., :k_sel]
     macs = selected_work(idx, w, k_sel) if k_sel > 0 else 0.0
     ops_qk, ops_pv = 2.0 * macs, 2.0 * macs
-    ops_lin = 2.0 * w.B * w.H * n_qb * 128.0 * w.d * w.d  # phi(Q_I) H_I, tf32
+    ops_lin = 2.0 * wl.B * wl.H * n_qb * 128.0 * w.d * w.d  # phi(Q_I) H_I, tf32
     p_bf16 = float(peaks["bf16_tflops"]) * 1e12
     p_qk = 2.0 * p_bf16 if a.quant else p_bf16  # int8 = 2x bf16 (nominal ratio)
     p_tf32 = 0.5 * p_bf16
@@ -367,9 +384,12 @@ def main():
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
-                "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": a.scaling,
                 "vs_baseline": None, "dtype": "i8+bf16" if a.quant else "bf16+fp16", "data": "synthetic",
-                "config": workload_config(w, a), "stages_ms": stage_ms, "roofline": roofline,
+                "config": dict(workload_config(w, a), parallelism=(
+                    f"{world} rank(s), one per GPU; " + ("each runs the whole workload" if a.scaling == "weak"
+                                                         else "B*H heads split in contiguous ranges"))),
+                "stages_ms": stage_ms, "roofline": roofline,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
                 "gpu_launches": KERNELS_PER_STEP[a.quant] * a.steps,
                 "dense_equiv_ops_per_step_per_gpu": ops}

@@ -27,7 +27,7 @@ __all__ = [
     "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_forward", "sla_check", "workspace",
     "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
-    "sla_block_mask_noalloc_limit",
+    "sla_block_mask_noalloc_limit", "head_shard", "shard_heads",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -70,6 +70,29 @@ class SlaError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = int(code)
         super().__init__(f"{what}: {sla_status_string(code)} ({code})")
+
+
+def head_shard(B: int, H: int, world: int, rank: int) -> tuple:
+    """(first, count): the contiguous range of the B*H (batch, head) pairs that rank
+    ``rank`` of ``world`` owns.  Every stage of the forward (mask, smoothing mean,
+    scales, states, per-query-block states, output) depends only on its own
+    (batch, head), so sharded ranks exchange nothing.  The first B*H % world ranks
+    take one pair more; a rank may own none when world > B*H."""
+    if world < 1 or not 0 <= rank < world or B < 1 or H < 1:
+        raise ValueError("need B, H, world >= 1 and 0 <= rank < world")
+    bh = B * H
+    base, extra = divmod(bh, world)
+    first = rank * base + min(rank, extra)
+    return first, base + (1 if rank < extra else 0)
+
+
+def shard_heads(x, world: int, rank: int):
+    """This rank's (batch, head) pairs of a [B, H, N, d] tensor (torch or numpy) as a
+    [1, count, N, d] view: the pairs are consecutive rows of [B*H, N, d], so the view
+    is contiguous and can go straight to sla_forward."""
+    B, H, N, d = x.shape
+    first, count = head_shard(B, H, world, rank)
+    return x.reshape(B * H, N, d)[first:first + count].reshape(1, count, N, d)
 
 
 def sla_version() -> str:
