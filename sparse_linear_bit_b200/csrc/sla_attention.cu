@@ -69,7 +69,7 @@ struct AttnCfg {
     static constexpr uint32_t kVBytes = 4 * kBox;                           // V of a pair of key blocks
     static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
     static constexpr int kStages = QUANT ? 4 : 3;
-    static constexpr uint32_t kLinBytes = 8 * kQRowsBox;                    // H_I 64 KB + phi(Q) 64 KB
+    static constexpr uint32_t kLinBytes = 10 * kQRowsBox;  // H_I 64 KB + phi(Q) 64 KB + raw Q 32 KB
     static constexpr uint32_t kRegion = (kStages * kStageBytes > kLinBytes) ? kStages * kStageBytes : kLinBytes;
 };
 
@@ -78,7 +78,7 @@ struct AttnSmem {
     alignas(1024) uint8_t region[AttnCfg<QUANT>::kRegion];  // K/V ring, then the linear operands
     float z[kD];
     float fin[2][3][128];   // epilogue exchange: [group][max, sum, den]
-    uint64_t bar_q, bar_h, bar_phiq, bar_lin, drain[3];
+    uint64_t bar_q, bar_h, bar_qr, bar_phiq, bar_lin, drain[3];
     uint64_t full[AttnCfg<QUANT>::kStages], empty[AttnCfg<QUANT>::kStages];
     uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_pv[2];
     uint64_t tok[2][4];     // exponential-phase token per group and lane quarter
@@ -96,7 +96,7 @@ SLA_DEV float ex2(float x)
 SLA_DEV float phi_f(float x, int phi)
 {
     if (phi == 1) return fmaxf(x, 0.0f);
-    return x > 0.0f ? x + 1.0f : expf(x);
+    return x > 0.0f ? x + 1.0f : __expf(x);  // rounded to tf32 next
 }
 
 SLA_DEV void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -174,7 +174,8 @@ SLA_DEV uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(
 template <bool QUANT>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-            const __grid_constant__ CUtensorMap tm_h, const uint16_t *__restrict__ qraw,
+            const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_qr,
+            const uint16_t *__restrict__ qraw,
             const int8_t *__restrict__ q8, const float *__restrict__ qscale, const float *__restrict__ kscale,
             const int32_t *__restrict__ idx, const float *__restrict__ hq, int N, int blk_q, int n_qb, int n_kb,
             int k_sel, int phi, uint16_t *__restrict__ out, int *status)
@@ -197,6 +198,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     if (tid == 0) {
         mbar_init(&sm.bar_q, 256);
         mbar_init(&sm.bar_h, 1);
+        mbar_init(&sm.bar_qr, 1);
         mbar_init(&sm.bar_phiq, 256);
         mbar_init(&sm.bar_lin, 1);
         for (int d = 0; d < 3; ++d) mbar_init(&sm.drain[d], 1);
@@ -224,23 +226,31 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     const uint32_t t_s = tmem, t_p = tmem + 128, t_q = tmem + 192, t_o = tmem + 256, t_l = tmem;
     uint8_t *h_s = sm.region;                       // end: 4 x [128 dims x 32 fp32]
     uint8_t *phiq_s = sm.region + 4 * kQRowsBox;    // end: 4 x [128 rows x 32 fp32]
+    uint8_t *qraw_s = sm.region + 8 * kQRowsBox;    // end: 2 x [128 rows x 64 bf16] (raw Q for phi)
 
+    // Issuing warps (producer, linear branch, Q.K^T + P.V of each group) run their
+    // loops with all 32 lanes, so that stage offsets and descriptors are
+    // warp-uniform, and elect one lane for each TMA / tcgen05 instruction.
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        if (elect_one()) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_h);
-            int issued = 0;
-            bool ok = true;
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                const int s = t % NS, u = t / NS;
-                if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
-                const int nb = min(2, k_sel - 2 * t);
-                uint8_t *st = sm.region + s * Cfg::kStageBytes;
+            tma_prefetch_desc(&tm_qr);
+        }
+        int issued = 0;
+        bool ok = true;
+        for (int t = 0; ok && t < n_tiles; ++t) {
+            const int s = t % NS, u = t / NS;
+            if (u > 0 && !(ok = mbar_wait_warp(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+            const int nb = min(2, k_sel - 2 * t);
+            uint8_t *st = sm.region + s * Cfg::kStageBytes;
+            const int J0 = __ldg(sel + 2 * t), J1 = nb > 1 ? __ldg(sel + 2 * t + 1) : 0;
+            if (elect_one()) {
                 mbar_expect_tx(&sm.full[s], (uint32_t)nb * Cfg::kStageBytes / 2);
                 for (int x = 0; x < nb; ++x) {
-                    const int J = __ldg(sel + 2 * t + x);
+                    const int J = x ? J1 : J0;
                     // K: rows 64x..64x+63 of the pair (one 128-channel int8 box, or two 64-channel bf16 boxes)
                     tma_load_3d(st + x * kBox, &tm_k, &sm.full[s], 0, J * 64, bh);
                     if (!QUANT) tma_load_3d(st + 2 * kBox + x * kBox, &tm_k, &sm.full[s], 64, J * 64, bh);
@@ -248,39 +258,44 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                     tma_load_3d(st + Cfg::kKBytes + x * kBox, &tm_v, &sm.full[s], 0, J * 64, bh);
                     tma_load_3d(st + Cfg::kKBytes + 2 * kBox + x * kBox, &tm_v, &sm.full[s], 64, J * 64, bh);
                 }
-                issued = t + 1;
             }
-            // H_I into the first 64 KB of the region once the stages there are retired
-            for (int s = 0; ok && s < NS && s * Cfg::kStageBytes < 4 * kQRowsBox; ++s) {
+            __syncwarp();
+            issued = t + 1;
+        }
+        // H_I and the raw Q rows into the region once every stage is retired
+        for (int s = 0; ok && s < NS; ++s) {
+            int tl = -1;
+            for (int t = s; t < n_tiles; t += NS) tl = t;
+            if (tl >= 0) ok = mbar_wait_warp(&sm.empty[s], (tl / NS) & 1, status, abort_flag);
+        }
+        if (ok && elect_one()) {
+            mbar_expect_tx(&sm.bar_h, 4 * kQRowsBox);
+            for (int c = 0; c < 4; ++c) tma_load_3d(h_s + c * kQRowsBox, &tm_h, &sm.bar_h, 32 * c, 0, bh * n_qb + I);
+            mbar_expect_tx(&sm.bar_qr, 2 * kQRowsBox);
+            for (int c = 0; c < 2; ++c)
+                tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_qr, 64 * c, I * blk_q, bh);
+        }
+        __syncwarp();
+        if (!ok) {  // failure: let loads in flight land before shared memory is released
+            for (int s = 0; s < NS; ++s) {
                 int tl = -1;
-                for (int t = s; t < n_tiles; t += NS) tl = t;
-                if (tl >= 0) ok = mbar_wait(&sm.empty[s], (tl / NS) & 1, status, abort_flag);
+                for (int t = s; t < issued; t += NS) tl = t;
+                if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / NS) & 1);
             }
-            if (ok) {
-                mbar_expect_tx(&sm.bar_h, 4 * kQRowsBox);
-                for (int c = 0; c < 4; ++c)
-                    tma_load_3d(h_s + c * kQRowsBox, &tm_h, &sm.bar_h, 32 * c, 0, bh * n_qb + I);
-            }
-            if (!ok) {  // failure: let loads in flight land before shared memory is released
-                for (int s = 0; s < NS; ++s) {
-                    int tl = -1;
-                    for (int t = s; t < issued; t += NS) tl = t;
-                    if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / NS) & 1);
-                }
-            } else {
-                mbar_wait_quiet(&sm.bar_h, 0);
-            }
+        } else {
+            mbar_wait_quiet(&sm.bar_h, 0);
+            mbar_wait_quiet(&sm.bar_qr, 0);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ linear-branch MMA
-        if (lane == 0) {
-            bool ok = true;
-            // linear branch: L = phi(Q_I) H_I (tf32) into the S columns, after the softmax groups are done
-            if (ok) ok = mbar_wait(&sm.bar_h, 0, status, abort_flag) && mbar_wait(&sm.bar_phiq, 0, status, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                constexpr uint32_t id_lin = idesc(1, 2, 2, 0, 0, 128, 128);  // f32 <- tf32 x tf32, K-major
-                const uint64_t pd = sdesc_sw128(smem_u32(phiq_s), 16, 1024), hd = sdesc_sw128(smem_u32(h_s), 16, 1024);
+        // L = phi(Q_I) H_I (tf32) into the S columns, after the softmax groups are done
+        bool ok = mbar_wait_warp(&sm.bar_h, 0, status, abort_flag);
+        if (ok) ok = mbar_wait_warp(&sm.bar_phiq, 0, status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            constexpr uint32_t id_lin = idesc(1, 2, 2, 0, 0, 128, 128);  // f32 <- tf32 x tf32, K-major
+            const uint64_t pd = sdesc_sw128(smem_u32(phiq_s), 16, 1024), hd = sdesc_sw128(smem_u32(h_s), 16, 1024);
+            if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const uint32_t off = (k >> 2) * kQRowsBox + (k & 3) * 32;
@@ -288,61 +303,72 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 }
                 mma_commit(&sm.bar_lin);
             }
+            __syncwarp();
+        }
+        if (elect_one()) {
             mma_commit(&sm.drain[0]);
             mbar_wait_quiet(&sm.drain[0], 0);  // this thread's MMAs retired before TMEM is released
         }
+        __syncwarp();
     } else if (warp >= 10) {
         // ------------------------------------------------------------ Q.K^T + P.V issuer of group g
         const int g = warp - 10;
-        if (lane == 0) {
-            constexpr uint32_t id_qk = QUANT ? idesc(2, 1, 1, 0, 0, 128, 64) : idesc(1, 1, 1, 0, 0, 128, 64);
-            constexpr uint32_t id_pv = QUANT ? idesc(1, 1, 1, 0, 1, 128, 128) : idesc(1, 0, 0, 0, 1, 128, 128);
-            const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
-            const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), 2 * kBox, 1024);
-            const uint32_t s_g = t_s + 64 * g;
-            const int nb = n_blk(g);
-            bool ok = true;
-            // S_g = Q K_j^T for this group's block of tile t (K rows of block g of the pair)
-            auto issue_qk = [&](int t) {
-                if (!(ok = mbar_wait(&sm.full[t % NS], (t / NS) & 1, status, abort_flag))) return;
-                if (t > 0 && !(ok = mbar_wait(&sm.bar_sfree[g], (t - 1) & 1, status, abort_flag))) return;
-                tc_fence_after();
-                const uint32_t so = (t % NS) * Cfg::kStageBytes + g * kBox;
+        constexpr uint32_t id_qk = QUANT ? idesc(2, 1, 1, 0, 0, 128, 64) : idesc(1, 1, 1, 0, 0, 128, 64);
+        constexpr uint32_t id_pv = QUANT ? idesc(1, 1, 1, 0, 1, 128, 128) : idesc(1, 0, 0, 0, 1, 128, 128);
+        const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
+        const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), 2 * kBox, 1024);
+        const uint32_t s_g = t_s + 64 * g, o_g = t_o + 128 * g, p_g = t_p + 32 * g;
+        const int nb = n_blk(g);
+        bool ok = true;
+        // S_g = Q K_j^T for this group's block of tile t (K rows of block g of the pair)
+        auto issue_qk = [&](int t) {
+            if (!(ok = mbar_wait_warp(&sm.full[t % NS], (t / NS) & 1, status, abort_flag))) return;
+            if (t > 0 && !(ok = mbar_wait_warp(&sm.bar_sfree[g], (t - 1) & 1, status, abort_flag))) return;
+            tc_fence_after();
+            const uint64_t kd = dadd(kd0, (t % NS) * Cfg::kStageBytes + g * kBox);
+            if (elect_one()) {
                 if (QUANT) {  // K-step of 32 int8 = 8 TMEM columns of Q
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(s_g, t_q + 8 * k, dadd(kd0, so + 32 * k), id_qk, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(s_g, t_q + 8 * k, kd + 2 * k, id_qk, k > 0 ? 1u : 0u);
                 } else {  // K-step of 16 bf16 = 8 TMEM columns of Q
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_f16_tmem_a(s_g, t_q + 8 * k, dadd(kd0, so + (k >> 2) * 2 * kBox + 32 * (k & 3)), id_qk,
+                        mma_f16_tmem_a(s_g, t_q + 8 * k, kd + (k >> 2) * (2 * kBox >> 4) + 2 * (k & 3), id_qk,
                                        k > 0 ? 1u : 0u);
                 }
                 mma_commit(&sm.bar_s[g]);
-            };
-            if (nb > 0) {
-                ok = mbar_wait(&sm.bar_q, 0, status, abort_flag);
-                if (ok) issue_qk(0);
             }
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                if (t < nb) {
-                    if (t + 1 < nb) {  // next logits as soon as this group has read S
-                        issue_qk(t + 1);
-                        if (!ok) break;
-                    }
-                    if (!(ok = mbar_wait(&sm.bar_p[g], t & 1, status, abort_flag))) break;
-                    tc_fence_after();
-                    const uint32_t vo = (t % NS) * Cfg::kStageBytes + g * kBox;  // this block's rows of the pair
+            __syncwarp();
+        };
+        if (nb > 0) {
+            ok = mbar_wait_warp(&sm.bar_q, 0, status, abort_flag);
+            if (ok) issue_qk(0);
+        }
+        for (int t = 0; ok && t < n_tiles; ++t) {
+            if (t < nb) {
+                if (t + 1 < nb) {  // next logits as soon as this group has read S
+                    issue_qk(t + 1);
+                    if (!ok) break;
+                }
+                if (!(ok = mbar_wait_warp(&sm.bar_p[g], t & 1, status, abort_flag))) break;
+                tc_fence_after();
+                const uint64_t vd = dadd(vd0, (t % NS) * Cfg::kStageBytes + g * kBox);  // this block's rows
+                if (elect_one()) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_f16_tmem_a(t_o + 128 * g, t_p + 32 * g + 8 * k, dadd(vd0, vo + 2048 * k), id_pv,
-                                       (t > 0 || k > 0) ? 1u : 0u);
+                        mma_f16_tmem_a(o_g, p_g + 8 * k, vd + 128 * k, id_pv, (t > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&sm.bar_pv[g]);
                 }
-                mma_commit(&sm.empty[t % NS]);  // stage t free once both groups' MMAs on it have retired
+                __syncwarp();
             }
+            if (elect_one()) mma_commit(&sm.empty[t % NS]);  // stage t free once both groups' MMAs retired
+            __syncwarp();
+        }
+        if (elect_one()) {
             mma_commit(&sm.drain[1 + g]);
             mbar_wait_quiet(&sm.drain[1 + g], 0);
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax / epilogue
         const int g = (warp - 2) >> 2;                  // group: key blocks 2t + g
@@ -403,6 +429,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         const int nb = n_blk(g);
+        // Phase tests are issued ahead of use (see mbar_test); a negative answer
+        // falls back to the bounded wait.
+        bool s_ready = false;
         for (int t = 0; ok && t < nb; ++t) {
             const int J = J_a;
             const float c = QUANT ? sq * ks_a * kscale_log2 : kscale_log2;
@@ -411,7 +440,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 if (QUANT) ks_a = __ldg(kscale + (size_t)bh * n_kb + J_b);
             }
             if (t + 2 < nb) J_b = blk_of(t + 2);
-            if (!(ok = wait_all(&sm.bar_s[g], t & 1))) break;
+            if (!__all_sync(0xffffffffu, s_ready) && !(ok = wait_all(&sm.bar_s[g], t & 1))) break;
             tc_fence_after();
             uint32_t sv[64];
             tmem_ld32(s_own, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -419,6 +448,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_sfree[g]);  // S_g may be rewritten now
+            const bool tok_ready = mbar_test(&sm.tok[g][quarter], t & 1);
             const int valid = min(64, N - J * 64);
             // the two paths are separate instantiations so the full-tile path carries no masking
             const float tmax = valid == 64 ? tile_max<QUANT, false>(sv, 64, c) : tile_max<QUANT, true>(sv, valid, c);
@@ -431,7 +461,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 l *= alpha;
             }
             // exponential phase, alternating with the other group's warp on this sub-partition
-            if (!(ok = wait_all(&sm.tok[g][quarter], t & 1))) break;
+            if (!__all_sync(0xffffffffu, tok_ready) && !(ok = wait_all(&sm.tok[g][quarter], t & 1))) break;
+            const bool pv_ready = t == 0 || mbar_test(&sm.bar_pv[g], (t - 1) & 1);
             uint32_t pk[32];
             const float off = QUANT ? -fmaf(kBias, c, m_used) : -m_used;
             if (valid == 64) l += tile_exp<QUANT, false>(sv, 64, c, off, pk);
@@ -439,7 +470,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.tok[g ^ 1][quarter]);
             // P and O of this group are free/stable once its previous P.V has retired
-            if (t > 0 && !(ok = wait_all(&sm.bar_pv[g], (t - 1) & 1))) break;
+            if (!__all_sync(0xffffffffu, pv_ready) && !(ok = wait_all(&sm.bar_pv[g], (t - 1) & 1))) break;
             if (t > 0 && __any_sync(0xffffffffu, need)) {  // rescale O of this group
                 tc_fence_after();
                 uint32_t o[32];
@@ -456,18 +487,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&sm.bar_p[g]);
+            if (t + 1 < nb) s_ready = mbar_test(&sm.bar_s[g], (t + 1) & 1);
         }
         // ---- linear branch operands: wait for every P.V (the ring is then free), then phi(Q) + den
         if (ok && n_blk(0) > 0) ok = wait_all(&sm.bar_pv[0], (n_blk(0) - 1) & 1);
         if (ok && n_blk(1) > 0) ok = wait_all(&sm.bar_pv[1], (n_blk(1) - 1) & 1);
         named_bar_sync(5, 256);  // every group past its P.V waits (z is also visible now)
         float den = 0.0f;
+        if (ok) ok = wait_all(&sm.bar_qr, 0);  // raw Q rows of this tile (rows past N read as 0)
         if (ok) {
-            const uint4 *qr = reinterpret_cast<const uint4 *>(qraw + ((size_t)bh * N + (row_valid ? i : 0)) * kD);
-#pragma unroll 4
+#pragma unroll 2
             for (int uu = 0; uu < 8; ++uu) {  // group g: channels 64g..64g+63, 8 per iteration
                 const int u = 8 * g + uu;
-                uint4 w = row_valid ? __ldg(qr + u) : make_uint4(0, 0, 0, 0);
+                const uint4 w = *reinterpret_cast<const uint4 *>(qraw_s + g * kQRowsBox + sw128_off(r, uu));
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                 float f[8];
 #pragma unroll
@@ -547,7 +579,7 @@ cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int
                           const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
                           const Geometry &g, int phi, void *out, int *status, cudaStream_t s)
 {
-    CUtensorMap tk, tv, th;
+    CUtensorMap tk, tv, th, tq;
     const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
     if (QUANT) {
         const uint64_t st[2] = {(uint64_t)kD, (uint64_t)g.N * kD};
@@ -570,11 +602,17 @@ cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int
         const uint32_t bh[3] = {32, 128, 1};
         if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, hd, st, bh)) return cudaErrorInvalidValue;
     }
+    {
+        // raw Q rows of a query block for phi(Q): [BH, N, 128] bf16, boxes of 64 channels x 128 rows
+        const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
+        const uint32_t bq[3] = {64, 128, 1};
+        if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, st, bq)) return cudaErrorInvalidValue;
+    }
     const size_t smem = sizeof(AttnSmem<QUANT>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(g.n_qb, g.BH);
-    attn_kernel<QUANT><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, static_cast<const uint16_t *>(q), q8, qscale,
+    attn_kernel<QUANT><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, tq, static_cast<const uint16_t *>(q), q8, qscale,
                                                         kscale, idx, hq, g.N, g.blk_q, g.n_qb, g.n_kb, g.k_sel, phi,
                                                         static_cast<uint16_t *>(out), status);
     return cudaGetLastError();

@@ -86,6 +86,44 @@ SLA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, int *status, volatile int
     }
 }
 
+// Non-blocking test of a phase (returns at once).  Issued ahead of the point
+// where the phase is needed, its latency (over a hundred cycles even for a
+// phase that has long completed) overlaps independent work; the caller falls
+// back to the bounded wait only if the test came back negative.
+SLA_DEV bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
+// every lane saw the phase complete (a timeout on any lane fails the warp).
+SLA_DEV bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, abort_flag));
+}
+
+// One lane of a fully active warp (always the lowest, lane 0), for instructions
+// that a single thread issues (tcgen05.mma / commit, TMA, expect_tx) while the
+// warp computes their operands together, so that they stay warp-uniform.
+SLA_DEV bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Bounded wait used only on failure paths, to let copies or MMAs already in
 // flight retire before a CTA releases its shared memory / TMEM.  Ignores the
 // abort flags; gives up after ~50 ms.
