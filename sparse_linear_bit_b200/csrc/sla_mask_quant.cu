@@ -91,60 +91,70 @@ __global__ void kmean_kernel(const double *__restrict__ part, int n_parts, int N
 
 // ---------------------------------------------------------------------------
 // scores[bh][I][J] = fma chain over channels c = 0..127 of qbar[I][c] * kbar[J][c]
-// 128 x 128 output tile per CTA; 256 threads as 16 x 16, each 8 x 8 outputs at
-// rows 2*ty + {0,1} + 32m and columns 2*tx + {0,1} + 32m (m = 0..3), so each
-// operand read is one 16-byte shared load serving two outputs.  Channels are
-// staged 16 at a time, transposed to [channel][row] in shared memory.
+// 128 (I) x 64 (J) output tile per CTA; 256 threads as 16 x 16, each 8 x 4
+// outputs at rows 2*ty + {0,1} + 32m (m < 4) and columns 2*tx + {0,1} + 32n
+// (n < 2), so each operand read is one 16-byte shared load serving two outputs.
+// At most 128 registers, so two CTAs share an SM and one's loads overlap the
+// other's FMAs.  Channels are staged 16 at a time, transposed to [channel][row].
 // ---------------------------------------------------------------------------
-constexpr int kScTile = 128;
+constexpr int kScI = 128;
+constexpr int kScJ = 64;
 constexpr int kScChan = 16;
 
-__global__ void __launch_bounds__(256, 1) scores_kernel(const double *__restrict__ qbar,
+__global__ void __launch_bounds__(256, 2) scores_kernel(const double *__restrict__ qbar,
                                                         const double *__restrict__ kbar, int n_qb, int n_kb,
                                                         double *__restrict__ scores)
 {
-    __shared__ __align__(16) double As[kScChan][kScTile];
-    __shared__ __align__(16) double Bs[kScChan][kScTile];
-    const int bh = blockIdx.z, I0 = blockIdx.y * kScTile, J0 = blockIdx.x * kScTile;
+    __shared__ __align__(16) double As[kScChan][kScI];
+    __shared__ __align__(16) double Bs[kScChan][kScJ];
+    const int bh = blockIdx.z, I0 = blockIdx.y * kScI, J0 = blockIdx.x * kScJ;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     const double *qh = qbar + (size_t)bh * n_qb * kD;
     const double *kh = kbar + (size_t)bh * n_kb * kD;
-    double acc[8][8];
+    double acc[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
     for (int c0 = 0; c0 < kD; c0 += kScChan) {
-        // 128 rows x 8 channel pairs per operand: thread -> (row = e & 127, pair = e >> 7),
-        // so consecutive threads store consecutive rows of one channel (no bank conflicts)
+        // thread -> (row = e & 127, channel pair = e >> 7): consecutive threads store consecutive
+        // rows of one channel (no bank conflicts); B covers 64 rows with the same mapping
 #pragma unroll
         for (int l = 0; l < 4; ++l) {
             const int e = tid + 256 * l, r = e & 127, c = 2 * (e >> 7);
-            double2 a = make_double2(0.0, 0.0), b = make_double2(0.0, 0.0);
+            double2 a = make_double2(0.0, 0.0);
             if (I0 + r < n_qb) a = __ldg(reinterpret_cast<const double2 *>(qh + (size_t)(I0 + r) * kD + c0 + c));
-            if (J0 + r < n_kb) b = __ldg(reinterpret_cast<const double2 *>(kh + (size_t)(J0 + r) * kD + c0 + c));
             As[c][r] = a.x;
             As[c + 1][r] = a.y;
+        }
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+            const int e = tid + 256 * l, r = e & 63, c = 2 * (e >> 6);
+            double2 b = make_double2(0.0, 0.0);
+            if (J0 + r < n_kb) b = __ldg(reinterpret_cast<const double2 *>(kh + (size_t)(J0 + r) * kD + c0 + c));
             Bs[c][r] = b.x;
             Bs[c + 1][r] = b.y;
         }
         __syncthreads();
 #pragma unroll
         for (int c = 0; c < kScChan; ++c) {
-            double a[8], b[8];
+            double a[8], b[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 const double2 av = *reinterpret_cast<const double2 *>(&As[c][2 * ty + 32 * m]);
-                const double2 bv = *reinterpret_cast<const double2 *>(&Bs[c][2 * tx + 32 * m]);
                 a[2 * m] = av.x;
                 a[2 * m + 1] = av.y;
-                b[2 * m] = bv.x;
-                b[2 * m + 1] = bv.y;
+            }
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                const double2 bv = *reinterpret_cast<const double2 *>(&Bs[c][2 * tx + 32 * n]);
+                b[2 * n] = bv.x;
+                b[2 * n + 1] = bv.y;
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
         }
         __syncthreads();
     }
@@ -154,7 +164,7 @@ __global__ void __launch_bounds__(256, 1) scores_kernel(const double *__restrict
         const int I = I0 + 2 * ty + (i & 1) + 32 * (i >> 1);
         if (I >= n_qb) continue;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
             const int J = J0 + 2 * tx + (j & 1) + 32 * (j >> 1);
             if (J < n_kb) sh[(size_t)I * n_kb + J] = acc[i][j] + 0.0;  // -0 -> +0
         }
@@ -285,6 +295,116 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double *__rest
     for (int J = n_kb + threadIdx.x; J < n_kb_pad; J += kTopkThreads) ar[J] = 0;
 }
 
+// ---------------------------------------------------------------------------
+// top-k selection, one warp per (bh, I) row, keys in registers (J = 32m + lane).
+// Radix select on the order-preserving 64-bit keys, 8 bits per pass, with a
+// warp-private shared histogram; after each pass the bin holding the k_sel-th
+// largest key is found by a warp suffix scan.  It stops early once every key
+// matching the resolved prefix P is selected.  Selected: (key & mask) > P, or
+// == P and among the first R such keys in J order (ties to the lower index),
+// ranked with ballots.  The bitmap words are the ballots themselves.
+// ---------------------------------------------------------------------------
+constexpr int kTopkWarps = 4;
+
+template <int KPL>  // keys per lane: n_kb <= 32 * KPL
+__global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double *__restrict__ scores, int n_rows,
+                                                                    int n_kb, int n_kb_pad, int k_sel, int subtract,
+                                                                    int32_t *__restrict__ idx,
+                                                                    uint32_t *__restrict__ bitmap,
+                                                                    uint16_t *__restrict__ amask)
+{
+    __shared__ int hist_all[kTopkWarps][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * kTopkWarps + warp;
+    if (row >= n_rows) return;  // warp-uniform: this kernel has no block-wide synchronisation
+    int *hist = hist_all[warp];
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const double *sr = scores + (size_t)row * n_kb;
+    uint64_t key[KPL];
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) {
+        const int J = 32 * m + lane;
+        key[m] = J < n_kb ? order_key(__ldg(sr + J)) : 0ull;
+    }
+    uint64_t P = 0, mask = 0;
+    int R = k_sel;
+    const bool partial = k_sel > 0 && k_sel < n_kb;
+    if (partial) {
+        for (int shift = 56; shift >= 0; shift -= 8) {
+#pragma unroll
+            for (int b = lane; b < 256; b += 32) hist[b] = 0;
+            __syncwarp();
+#pragma unroll
+            for (int m = 0; m < KPL; ++m)
+                if (32 * m + lane < n_kb && (key[m] & mask) == P) atomicAdd(&hist[(int)((key[m] >> shift) & 255u)], 1);
+            __syncwarp();
+            // lane L covers bins 255-8L .. 248-8L (top first); suffix counts by an inclusive lane scan
+            const int top = 255 - 8 * lane;
+            int h8[8], tot = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                h8[e] = hist[top - e];
+                tot += h8[e];
+            }
+            int incl = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int L = __ffs(__ballot_sync(0xffffffffu, incl >= R)) - 1;  // candidates >= R, so L >= 0
+            int bsel = 0, rn = 0, cnt = 0;
+            if (lane == L) {
+                int cum = incl - tot;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if (cnt == 0 && cum + h8[e] >= R) {
+                        bsel = top - e;
+                        rn = R - cum;
+                        cnt = h8[e];
+                    }
+                    cum += h8[e];
+                }
+            }
+            bsel = __shfl_sync(0xffffffffu, bsel, L);
+            rn = __shfl_sync(0xffffffffu, rn, L);
+            cnt = __shfl_sync(0xffffffffu, cnt, L);
+            P |= (uint64_t)bsel << shift;
+            mask |= (uint64_t)255u << shift;
+            R = rn;
+            __syncwarp();  // every lane has read the histogram before the next pass clears it
+            if (cnt == R) break;  // every key matching P is selected
+        }
+    }
+    int32_t *ir = idx + (size_t)row * k_sel;
+    uint16_t *ar = amask + (size_t)row * n_kb_pad;
+    uint32_t *br = bitmap ? bitmap + (size_t)row * ((n_kb + 31) / 32) : nullptr;
+    const uint16_t one = 0x3F80u;  // bf16 1.0
+    int o = 0, eq_seen = 0;
+#pragma unroll
+    for (int m = 0; m < KPL; ++m) {
+        if (32 * m >= n_kb) break;  // warp-uniform
+        const int J = 32 * m + lane;
+        const bool valid = J < n_kb;
+        bool s;
+        if (!partial) {
+            s = valid && k_sel > 0;
+        } else {
+            const uint64_t km = key[m] & mask;
+            const bool eq = valid && km == P;
+            const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+            s = (valid && km > P) || (eq && eq_seen + __popc(eqb & lt_mask) < R);
+            eq_seen += __popc(eqb);
+        }
+        const unsigned sb = __ballot_sync(0xffffffffu, s);
+        if (s) ir[o + __popc(sb & lt_mask)] = J;
+        o += __popc(sb);
+        if (valid) ar[J] = (s != (subtract == 0)) ? one : (uint16_t)0;
+        if (br && lane == 0) br[m] = sb;
+    }
+    for (int J = n_kb + lane; J < n_kb_pad; J += 32) ar[J] = 0;
+}
+
 // zero the bitmap rows before the atomicOr pass
 __global__ void zero_u32_kernel(uint32_t *p, size_t n)
 {
@@ -398,7 +518,7 @@ cudaError_t launch_kmean(const double *part, int BH, int N, int n_kb, float *kme
 
 cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry &g, double *scores, cudaStream_t s)
 {
-    dim3 grid((g.n_kb + kScTile - 1) / kScTile, (g.n_qb + kScTile - 1) / kScTile, g.BH);
+    dim3 grid((g.n_kb + kScJ - 1) / kScJ, (g.n_qb + kScI - 1) / kScI, g.BH);
     scores_kernel<<<grid, 256, 0, s>>>(qbar, kbar, g.n_qb, g.n_kb, scores);
     return cudaGetLastError();
 }
@@ -406,6 +526,20 @@ cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry
 cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap, uint16_t *amask,
                         cudaStream_t s)
 {
+    const int rows = g.BH * g.n_qb;
+    const unsigned blocks = (unsigned)((rows + kTopkWarps - 1) / kTopkWarps);
+    const int sub = g.subtract ? 1 : 0;
+    // one warp per row while the row's keys fit in registers
+    if (g.n_kb <= 32 * 8) {
+        topk_warp_kernel<8><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx,
+                                                               bitmap, amask);
+        return cudaGetLastError();
+    }
+    if (g.n_kb <= 32 * 40) {
+        topk_warp_kernel<40><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx,
+                                                                bitmap, amask);
+        return cudaGetLastError();
+    }
     if (bitmap) {
         const size_t n = (size_t)g.BH * g.n_qb * ((g.n_kb + 31) / 32);
         zero_u32_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, s>>>(bitmap, n);
@@ -415,8 +549,7 @@ cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, u
         cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    topk_kernel<<<g.BH * g.n_qb, kTopkThreads, smem, s>>>(scores, g.n_qb, g.n_kb, g.n_kb_pad, g.k_sel,
-                                                          g.subtract ? 1 : 0, idx, bitmap, amask);
+    topk_kernel<<<rows, kTopkThreads, smem, s>>>(scores, g.n_qb, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx, bitmap, amask);
     return cudaGetLastError();
 }
 
