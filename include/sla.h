@@ -150,8 +150,10 @@ SLA_API size_t sla_block_mask_noalloc_limit(void);
 
 /* sla_forward with per-stage device timing: enqueues the same launches with a
  * CUDA event between stages, waits for them, and writes 7 floats to the host
- * array stage_ms: milliseconds of {pooling, scores + top-k, quantisation,
- * linear states, per-query-block state, attention, whole call}.  Blocks the
+ * array stage_ms: milliseconds of {Q quantisation (with the pooled Q means;
+ * pooling alone when quant = 0), pooled K means + linear states,
+ * scores + top-k, K smoothing + quantisation, per-query-block state,
+ * attention, whole call}.  Blocks the
  * calling host thread until the call has finished on `stream`. */
 SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
                                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,

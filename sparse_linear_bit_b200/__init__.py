@@ -179,7 +179,7 @@ def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -
                         int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_forward")
 
 
-PROFILE_STAGES = ("pool", "scores_topk", "quantize", "states", "state_reduce", "attention", "total")
+PROFILE_STAGES = ("quantize_q", "states", "scores_topk", "quantize_k", "state_reduce", "attention", "total")
 
 
 def sla_forward_profile(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -> dict:

@@ -209,9 +209,9 @@ sla_status sla_quantize_qk(const void *q, const void *k, int B, int H, int N, in
     double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
     float *mean = k_mean ? k_mean : reinterpret_cast<float *>(ws_at(ws, L.kmean));
     SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, kpart, s));
-    SLA_TRY(launch_kmean(kpart, g.BH, N, g.n_kb, mean, s));
-    SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, s));
-    SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, s));
+    SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), mean, s));
+    SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, nullptr, s));
+    SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, nullptr, s));
     return SLA_OK;
 }
 
@@ -257,24 +257,26 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
 
     SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
     mark();
-    // (1) pooled block means (and the partial sums of K for its per-channel mean)
-    SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
-    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, quant ? kpart : nullptr, s));
+    // (1) Q: INT8 codes and scales, with the pooled block means as a by-product
+    //     (without quantisation: the pooled means alone)
+    if (quant) SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, qbar, s));
+    else SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
     mark();
-    // (2) scores + top-k selection
+    // (2) pooled block means of K (and its partial sums for the smoothing mean),
+    //     per-key-block linear states and the global state
+    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, quant ? kpart : nullptr, s));
+    SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, s));
+    SLA_TRY(launch_htot(partials, g, htot, s));
+    mark();
+    // (3) scores + top-k selection
     SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
     SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
     mark();
-    // (3) smoothing + INT8 quantisation
+    // (4) K: smoothing mean, INT8 codes and scales
     if (quant) {
-        SLA_TRY(launch_kmean(kpart, g.BH, N, g.n_kb, kmean, s));
-        SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, s));
-        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, s));
+        SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), kmean, s));
+        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, nullptr, s));
     }
-    mark();
-    // (4) per-key-block linear states and their global sum
-    SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, s));
-    SLA_TRY(launch_htot(partials, g, htot, s));
     mark();
     // (5) per-query-block state
     SLA_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));

@@ -33,13 +33,14 @@ int topk_count(int n_kb, float topk);
 // block means (and, when part != nullptr, per-CTA partial sums for launch_kmean)
 int pool_parts(int nb);
 cudaError_t launch_pool(const void *x, int BH, int N, int blk, int nb, double *mean, double *part, cudaStream_t s);
-cudaError_t launch_kmean(const double *part, int BH, int N, int n_kb, float *kmean, cudaStream_t s);
+cudaError_t launch_kmean(const double *part, int BH, int N, int n_parts, float *kmean, cudaStream_t s);
 cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry &g, double *scores,
                           cudaStream_t s);
 cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap,
                         uint16_t *amask, cudaStream_t s);
+// INT8 codes and scales; with `bmean` (no smoothing) also the fp64 block means
 cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out,
-                         float *scale, cudaStream_t s);
+                         float *scale, double *bmean, cudaStream_t s);
 
 // linear branch and fused attention (tcgen05)
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states,

@@ -423,15 +423,22 @@ __global__ void zero_u32_kernel(uint32_t *p, size_t n)
 // |x/s| 2^-24, so for |x/s| <= 128 (|x| <= amax = 127 s, up to rounding)
 // |t - fl(x/s)| < 2.3e-5.  Unless t lies within 2^-14 of a half-integer, no
 // rounding boundary of rint separates t from fl(x/s) and rint(t) is the
-// code; otherwise (about 1 element in 8000) the IEEE quotient is taken.
+// code; otherwise (about 1 element in 8000) the IEEE quotient is taken.  On
+// the fast path |t| <= 127 (1 + 3 * 2^-24), so rint(t) needs no clamp, and the
+// low byte of the bits of t + 1.5 * 2^23 (which rounds t to an integer, ties to
+// even) is rint(t) in two's complement.
 // ---------------------------------------------------------------------------
+// When `bmean` is given (Q only), the kernel also writes the block's fp64 mean
+// row, the pooled mean that block selection scores with (exact fp64 sums, so the
+// same values as the pooling kernel's).
 template <bool SMOOTH, int BLK>
 __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
                                                     const float *__restrict__ mean, uint2 *__restrict__ out,
-                                                    float *__restrict__ scale)
+                                                    float *__restrict__ scale, double *__restrict__ bmean)
 {
     constexpr int kVec = BLK * (kD / 8) / 256;  // uint4 per thread
     __shared__ float warp_max[8];
+    __shared__ double part[8][16][8];  // block-mean partials: [warp][channel group][channel]
     const int bh = blockIdx.y, J = blockIdx.x;
     const int t0 = J * BLK;
     const int rows = min(BLK, N - t0);
@@ -454,6 +461,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
         }
     };
     float amax = 0.0f;
+    double bsum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int l = 0; l < kVec; ++l) {
         if (((threadIdx.x + 256 * l) >> 4) < rows) {
@@ -461,12 +469,31 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
             expand(raw[l], f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            if (!SMOOTH && bmean) {  // without smoothing f holds the raw values
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bsum[i] += (double)f[i];
+            }
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+    if (!SMOOTH && bmean) {  // lanes cg and cg + 16 of a warp share a channel group
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bsum[i] += __shfl_xor_sync(0xffffffffu, bsum[i], 16);
+        if ((threadIdx.x & 31) < 16) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) part[threadIdx.x >> 5][cg][i] = bsum[i];
+        }
+    }
     __syncthreads();
+    if (!SMOOTH && bmean && threadIdx.x < kD) {
+        const int c = threadIdx.x;
+        double sum = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += part[w][c >> 3][c & 7];
+        bmean[((size_t)bh * nb + J) * kD + c] = sum / (double)rows;
+    }
     amax = warp_max[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
@@ -474,6 +501,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
     if (threadIdx.x == 0) scale[(size_t)bh * nb + J] = s;
     const float r = s != 0.0f ? __fdiv_rn(1.0f, s) : 0.0f;
     const bool fast = s != 0.0f && isfinite(r);
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: t + kRound rounds t to an integer (ties to even)
     uint2 *ob = out + ((size_t)bh * N + t0) * (kD / 8);
 #pragma unroll
     for (int l = 0; l < kVec; ++l) {
@@ -481,20 +509,30 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
         if ((e >> 4) < rows) {
             float f[8];
             expand(raw[l], f);
-            uint32_t w[2] = {0, 0};
+            // fast path: the low byte of the bits of t + kRound is rint(t) as int8 (|t| <= 127 here)
+            uint32_t cb[8];
+            unsigned slow = fast ? 0u : 0xFFu;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                int c = 0;
-                if (s != 0.0f) {
-                    const float t = f[i] * r;
-                    const float rt = rintf(t);
-                    float q = rt;
-                    if (!fast || fabsf(t - rt) > 0.5f - 6.103515625e-05f) q = rintf(__fdiv_rn(f[i], s));
-                    c = max(-127, min(127, __float2int_rn(q)));
-                }
-                w[i >> 2] |= ((uint32_t)(c & 0xFF)) << (8 * (i & 3));
+                const float t = f[i] * r;
+                const float qf = __fadd_rn(t, kRound);
+                const float rt = __fsub_rn(qf, kRound);
+                if (fabsf(t - rt) > 0.5f - 6.103515625e-05f) slow |= 1u << i;
+                cb[i] = __float_as_uint(qf);
             }
-            ob[e] = make_uint2(w[0], w[1]);
+            if (slow) {  // rare: within 2^-14 of a half-integer, or a zero / tiny scale
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (slow & (1u << i)) {
+                        int c = 0;
+                        if (s != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(f[i], s))));
+                        cb[i] = (uint32_t)c;
+                    }
+                }
+            }
+            const uint32_t w0 = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+            const uint32_t w1 = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
+            ob[e] = make_uint2(w0, w1);
         }
     }
 }
@@ -510,9 +548,9 @@ cudaError_t launch_pool(const void *x, int BH, int N, int blk, int nb, double *m
     return cudaGetLastError();
 }
 
-cudaError_t launch_kmean(const double *part, int BH, int N, int n_kb, float *kmean, cudaStream_t s)
+cudaError_t launch_kmean(const double *part, int BH, int N, int n_parts, float *kmean, cudaStream_t s)
 {
-    kmean_kernel<<<BH, kD, 0, s>>>(part, pool_parts(n_kb), N, kmean);
+    kmean_kernel<<<BH, kD, 0, s>>>(part, n_parts, N, kmean);
     return cudaGetLastError();
 }
 
@@ -554,18 +592,18 @@ cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, u
 }
 
 cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out, float *scale,
-                         cudaStream_t s)
+                         double *bmean, cudaStream_t s)
 {
     dim3 grid(nb, BH);
     const uint4 *xi = static_cast<const uint4 *>(x);
     uint2 *o = reinterpret_cast<uint2 *>(out);
     if (mean) {
-        if (blk != 64) return cudaErrorInvalidValue;
-        quant_kernel<true, 64><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale);
+        if (blk != 64 || bmean) return cudaErrorInvalidValue;
+        quant_kernel<true, 64><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale, nullptr);
     } else if (blk == 128) {
-        quant_kernel<false, 128><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale);
+        quant_kernel<false, 128><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
     } else if (blk == 64) {
-        quant_kernel<false, 64><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale);
+        quant_kernel<false, 64><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
     } else {
         return cudaErrorInvalidValue;
     }
