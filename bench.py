@@ -45,7 +45,7 @@ ATTN_SRC = os.path.join(ROOT, "sparse_linear_bit_b200", "csrc", "sla_attention.c
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = {1: 11, 0: 8}  # our launches per sla_forward call (quant on / off)
+KERNELS_PER_STEP = {1: 10, 0: 8}  # our launches per sla_forward call (quant on / off)
 
 
 def parse():
@@ -61,6 +61,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"])
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling runs)")
     return ap.parse_args()
 
 
@@ -237,8 +238,8 @@ def main():
     import synth
 
     w0 = synth.WORKLOADS[a.workload]
-    w = synth.Workload(w0.name, w0.B, w0.H, w0.grid, blk_q=w0.blk_q, blk_k=w0.blk_k, topk=a.topk, phi=a.phi,
-                       quant=a.quant, seed=w0.seed)
+    w = synth.Workload(w0.name if not a.heads else f"{w0.name}-h{a.heads}", w0.B, a.heads or w0.H, w0.grid,
+                       blk_q=w0.blk_q, blk_k=w0.blk_k, topk=a.topk, phi=a.phi, quant=a.quant, seed=w0.seed)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
