@@ -238,6 +238,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_h);
             tma_prefetch_desc(&tm_qr);
+            // the linear epilogue's operands (H_I, raw Q rows) into L2 now, so that their loads
+            // at the end of the CTA do not wait on HBM
+            for (int c = 0; c < 4; ++c) tma_prefetch_l2_3d(&tm_h, 32 * c, 0, bh * n_qb + I);
+            for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_qr, 64 * c, I * blk_q, bh);
         }
         int issued = 0;
         bool ok = true;

@@ -159,6 +159,14 @@ SLA_DEV void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c
         : "memory");
 }
 
+// Prefetch a TMA tile into L2 (no shared memory, no completion to wait for)
+SLA_DEV void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // TMA tensor store shared -> global (bulk-group completion, issuing thread only)
 SLA_DEV void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1, int c2)
 {
