@@ -65,7 +65,8 @@ def load(path: Optional[str] = None):
     lib.orc_set_threads.argtypes = [i32]
     lib.orc_pool.argtypes = [P, i32, i32, i32, i32, P]
     lib.orc_block_mask.argtypes = [P, P, i32, i32, i32, i32, i32, f64, P, P, P]
-    lib.orc_quantize.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.orc_quantize.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.orc_e4m3_array.argtypes = [P, P, P, i64]
     lib.orc_states.argtypes = [P, P, i32, i32, i32, i32, P, P]
     lib.orc_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, f64, i32, i32, P, P, i64, P, P, P]
     lib.orc_forward.restype = i32
@@ -136,8 +137,11 @@ def block_mask(q, k, blk_q: int, blk_k: int, topk: float, with_scores: bool = Fa
     return (idx, bm, sc) if with_scores else (idx, bm)
 
 
-def quantize(q, k, blk_q: int, blk_k: int, lib=None):
-    """INT8 codes and fp32 scales: (q8, k8, s_q[BH,n_qb], s_k[BH,n_kb], k_mean[BH,d])."""
+def quantize(q, k, blk_q: int, blk_k: int, lib=None, fp8: bool = False):
+    """Codes and fp32 scales: (q8, k8, s_q[BH,n_qb], s_k[BH,n_kb], k_mean[BH,d]).
+
+    INT8 codes by default; with ``fp8`` the codes are FP8 e4m3 bit patterns
+    (stored in int8 arrays; view them as uint8)."""
     lib = lib or load()
     q, k = _bits(q), _bits(k)
     BH, N, d = _shape(q)
@@ -147,8 +151,20 @@ def quantize(q, k, blk_q: int, blk_k: int, lib=None):
     sq = np.zeros((BH, n_qb), dtype=np.float32)
     sk = np.zeros((BH, n_kb), dtype=np.float32)
     km = np.zeros((BH, d), dtype=np.float32)
-    lib.orc_quantize(_ptr(q), _ptr(k), BH, N, d, blk_q, blk_k, _ptr(q8), _ptr(k8), _ptr(sq), _ptr(sk), _ptr(km))
+    lib.orc_quantize(_ptr(q), _ptr(k), BH, N, d, blk_q, blk_k, int(bool(fp8)), _ptr(q8), _ptr(k8), _ptr(sq),
+                     _ptr(sk), _ptr(km))
     return q8, k8, sq, sk, km
+
+
+def e4m3(x, lib=None):
+    """(value, bits): the fp8 e4m3 value nearest to each fp32 x (ties to even, saturated to
+    +-448) and its bit pattern."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    value = np.zeros(x.shape, dtype=np.float32)
+    bits = np.zeros(x.shape, dtype=np.uint8)
+    lib.orc_e4m3_array(_ptr(x), _ptr(value), _ptr(bits), x.size)
+    return value, bits
 
 
 def states(k, v, blk_k: int, phi: int, lib=None):

@@ -23,10 +23,15 @@
  *     K is smoothed by its per-channel mean over all N tokens; per block
  *     scale = amax / 127 in fp32; code = clamp(rint_even(x / scale), -127,
  *     127), every step in IEEE fp32 so that a GPU can reproduce it exactly.
+ *     FP8 variant (quant = 2; the same section names FP8 beside INT8): scale =
+ *     amax / 448 and code = the fp8 e4m3 value nearest to x / scale (ties to
+ *     even, saturating at +-448; e4m3: 4 exponent bits with bias 7, 3
+ *     mantissa bits, subnormals down to 2^-9, no infinities).
  *  5. Sparse branch: for every query row, exact softmax attention
  *     softmax(q k^T / sqrt(d)) v ("TurboDiffusion技术架构解析", §2.1, standard
  *     attention formula) restricted to the tokens of the selected key blocks;
- *     with quantisation on, the logits are (qhat . khat) * s_q * s_k / sqrt(d).
+ *     with quantisation on, the logits are (qhat . khat) * s_q * s_k / sqrt(d)
+ *     (for FP8 the dot product of the decoded e4m3 values, exact in fp64).
  *  6. Linear branch over the remaining (unselected) key blocks: kernelised
  *     linear attention phi(Q)(phi(K)^T V) ("TurboDiffusion技术架构解析", §2.1,
  *     linear attention formula, phi = elu+1 or ReLU), normalised by
@@ -186,11 +191,65 @@ static int8_t code8(float x, float s)
     return (int8_t)r;
 }
 
+/* The fp8 e4m3 value nearest to x (ties to even, sign kept), saturated to +-448.  The
+ * quantum is 2^(e-3) for |x| in [2^e, 2^(e+1)), e >= -6, and 2^-9 below 2^-6. */
+float orc_e4m3(float x)
+{
+    if (isnan(x)) return x;
+    double a = fabs((double)x);
+    if (a > 448.0) return (float)copysign(448.0, (double)x);
+    int E;
+    frexp(a, &E);                      /* a = f * 2^E, f in [0.5, 1): floor(log2 a) = E - 1 */
+    int qexp = a < ldexp(1.0, -6) ? -9 : (E - 1) - 3;
+    double r = nearbyint(ldexp(a, -qexp)); /* a / quantum, rounded half to even */
+    double v = ldexp(r, qexp);
+    if (v > 448.0) v = 448.0;
+    return (float)copysign(v, (double)x); /* the sign survives rounding to zero */
+}
+
+/* The e4m3 bit pattern of a value that e4m3 represents exactly (orc_e4m3's output). */
+uint8_t orc_e4m3_bits(float v)
+{
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -6)) return (uint8_t)(sign | (int)ldexp(a, 9)); /* subnormal: m * 2^-9 */
+    int E;
+    double f = frexp(a, &E);           /* a = (2f) * 2^(E-1), 2f in [1, 2) */
+    int e = E - 1 + 7;                 /* biased exponent, 1..15 */
+    int m = (int)((2.0 * f - 1.0) * 8.0);
+    return (uint8_t)(sign | (e << 3) | m);
+}
+
+static double e4m3_value(uint8_t b)
+{
+    int e = (b >> 3) & 15, m = b & 7;
+    double a = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (b & 0x80) ? -a : a;
+}
+
+/* orc_e4m3 and orc_e4m3_bits over an array (for the pins). */
+void orc_e4m3_array(const float *x, float *value, uint8_t *bits, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        value[i] = orc_e4m3(x[i]);
+        bits[i] = orc_e4m3_bits(value[i]);
+    }
+}
+
+/* Symmetric per-block FP8 code of x with scale s (both fp32): e4m3 bits. */
+static uint8_t code_fp8(float x, float s)
+{
+    if (s == 0.0f) return 0;
+    return orc_e4m3_bits(orc_e4m3(x / s));
+}
+
 /* Quantise one head.  K is smoothed by its fp32-rounded per-channel mean. */
-static void quant_head(const uint16_t *q, const uint16_t *k, int N, int d, int blk_q, int blk_k,
+static void quant_head(const uint16_t *q, const uint16_t *k, int N, int d, int blk_q, int blk_k, int fp8,
                        int8_t *q8, int8_t *k8, float *sq, float *sk, float *kmean)
 {
     int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    const float qmax = fp8 ? 448.0f : 127.0f;
     float *mu = (float *)malloc(sizeof(float) * (size_t)d);
     for (int c = 0; c < d; ++c) {
         double s = 0.0;
@@ -202,30 +261,35 @@ static void quant_head(const uint16_t *q, const uint16_t *k, int N, int d, int b
         int t0 = I * blk_q, t1 = t0 + blk_q < N ? t0 + blk_q : N;
         float amax = 0.0f;
         for (size_t e = (size_t)t0 * d; e < (size_t)t1 * d; ++e) amax = fmaxf(amax, fabsf(bf32(q[e])));
-        float s = amax / 127.0f;
+        float s = amax / qmax;
         sq[I] = s;
-        for (size_t e = (size_t)t0 * d; e < (size_t)t1 * d; ++e) q8[e] = code8(bf32(q[e]), s);
+        for (size_t e = (size_t)t0 * d; e < (size_t)t1 * d; ++e)
+            q8[e] = fp8 ? (int8_t)code_fp8(bf32(q[e]), s) : code8(bf32(q[e]), s);
     }
     for (int J = 0; J < n_kb; ++J) {
         int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
         float amax = 0.0f;
         for (int t = t0; t < t1; ++t)
             for (int c = 0; c < d; ++c) amax = fmaxf(amax, fabsf(bf32(k[(size_t)t * d + c]) - mu[c]));
-        float s = amax / 127.0f;
+        float s = amax / qmax;
         sk[J] = s;
         for (int t = t0; t < t1; ++t)
-            for (int c = 0; c < d; ++c) k8[(size_t)t * d + c] = code8(bf32(k[(size_t)t * d + c]) - mu[c], s);
+            for (int c = 0; c < d; ++c) {
+                float x = bf32(k[(size_t)t * d + c]) - mu[c];
+                k8[(size_t)t * d + c] = fp8 ? (int8_t)code_fp8(x, s) : code8(x, s);
+            }
     }
     free(mu);
 }
 
-void orc_quantize(const uint16_t *q, const uint16_t *k, int BH, int N, int d, int blk_q, int blk_k,
+/* fp8 = 0: INT8 codes; fp8 = 1: FP8 e4m3 codes (bit patterns in the int8 arrays). */
+void orc_quantize(const uint16_t *q, const uint16_t *k, int BH, int N, int d, int blk_q, int blk_k, int fp8,
                   int8_t *q8, int8_t *k8, float *sq, float *sk, float *kmean)
 {
     int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
 #pragma omp parallel for schedule(dynamic)
     for (int bh = 0; bh < BH; ++bh)
-        quant_head(q + (size_t)bh * N * d, k + (size_t)bh * N * d, N, d, blk_q, blk_k,
+        quant_head(q + (size_t)bh * N * d, k + (size_t)bh * N * d, N, d, blk_q, blk_k, fp8,
                    q8 + (size_t)bh * N * d, k8 + (size_t)bh * N * d, sq + (size_t)bh * n_qb,
                    sk + (size_t)bh * n_kb, kmean ? kmean + (size_t)bh * d : NULL);
 }
@@ -302,11 +366,16 @@ static void row_out(int i, const uint16_t *q, const uint16_t *k, const uint16_t 
         int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
         for (int j = t0; j < t1; ++j) {
             double l;
-            if (quant) {
+            if (quant == 1) {
                 int64_t acc = 0;
                 for (int c = 0; c < d; ++c)
                     acc += (int64_t)q8[(size_t)i * d + c] * (int64_t)k8[(size_t)j * d + c];
                 l = (double)acc * (double)sq[I] * (double)sk[J] * inv_sqrt_d;
+            } else if (quant == 2) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc += e4m3_value((uint8_t)q8[(size_t)i * d + c]) * e4m3_value((uint8_t)k8[(size_t)j * d + c]);
+                l = acc * (double)sq[I] * (double)sk[J] * inv_sqrt_d;
             } else {
                 double acc = 0.0;
                 for (int c = 0; c < d; ++c) acc += bf(q[(size_t)i * d + c]) * bf(k[(size_t)j * d + c]);
@@ -350,7 +419,8 @@ static int cmp_i64(const void *a, const void *b)
 }
 
 /*
- * Forward for a list of rows.  rows: [nrows][2] pairs (bh, i); when rows is
+ * Forward for a list of rows (quant: 0 = none, 1 = INT8, 2 = FP8 e4m3).
+ * rows: [nrows][2] pairs (bh, i); when rows is
  * NULL every row of every head is produced in [BH][N] order (nrows ignored).
  * idx_in (nullable, [BH][n_qb][k_sel]) replaces the oracle's own selection.
  * out, out_s, out_l: [nrows][d] (out_s / out_l nullable).  Returns 0, or -1
@@ -395,7 +465,7 @@ int orc_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int BH,
             memcpy(idx, idx_in + (size_t)bh * n_qb * k_sel, sizeof(int32_t) * (size_t)n_qb * k_sel);
         else
             mask_head(qh, kh, N, d, blk_q, blk_k, k_sel, idx, NULL, NULL);
-        if (quant) quant_head(qh, kh, N, d, blk_q, blk_k, q8, k8, sq, sk, NULL);
+        if (quant) quant_head(qh, kh, N, d, blk_q, blk_k, quant == 2, q8, k8, sq, sk, NULL);
 #pragma omp parallel for schedule(dynamic)
         for (int J = 0; J < n_kb; ++J) {
             int t0 = J * blk_k;

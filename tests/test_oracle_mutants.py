@@ -27,7 +27,13 @@ MUTANTS = {
     "tie_prefers_higher_block": ("return (x->j > y->j) - (x->j < y->j);", "return (x->j < y->j) - (x->j > y->j);"),
     "ceil_count": ("double x = floor(topk * (double)n_kb + 1e-4);", "double x = ceil(topk * (double)n_kb - 1e-4);"),
     "pool_divides_by_block": ("mean[(size_t)J * d + c] = s / (double)(t1 - t0);", "mean[(size_t)J * d + c] = s / (double)blk;"),
-    "scale_over_128_q": ("        float s = amax / 127.0f;\n        sq[I] = s;", "        float s = amax / 128.0f;\n        sq[I] = s;"),
+    "scale_over_128": ("const float qmax = fp8 ? 448.0f : 127.0f;", "const float qmax = fp8 ? 448.0f : 128.0f;"),
+    "fp8_scale_over_240": ("const float qmax = fp8 ? 448.0f : 127.0f;", "const float qmax = fp8 ? 240.0f : 127.0f;"),
+    "e4m3_exponent_bias_8": ("int e = E - 1 + 7;", "int e = E - 1 + 8;"),
+    "e4m3_round_half_up": ("double r = nearbyint(ldexp(a, -qexp));", "double r = floor(ldexp(a, -qexp) + 0.5);"),
+    "e4m3_no_subnormals": ("int qexp = a < ldexp(1.0, -6) ? -9 : (E - 1) - 3;", "int qexp = (E - 1) - 3;"),
+    "fp8_logits_raw_bytes": ("acc += e4m3_value((uint8_t)q8[(size_t)i * d + c]) * e4m3_value((uint8_t)k8[(size_t)j * d + c]);",
+                             "acc += (double)q8[(size_t)i * d + c] * e4m3_value((uint8_t)k8[(size_t)j * d + c]);"),
     "no_smoothing": ("mu[c] = (float)(s / (double)N);", "mu[c] = 0.0f;"),
     "softmax_unnormalised": ("for (int e = 0; e < d; ++e) os[e] /= den;", "(void)den;"),
     "elu_without_plus_one": ("return x > 0.0 ? x + 1.0 : exp(x);", "return x > 0.0 ? x : exp(x) - 1.0;"),

@@ -13,6 +13,11 @@ of the oracle) and raises AssertionError on a mismatch.  What pins what:
 * quantisation     -- a block whose values are exact multiples of the scale;
   range, amax -> +-127 and half-step error bounds; zero block; smoothing
   invariance to a per-channel shift of K; Q is not smoothed
+* FP8 e4m3         -- the encoder equals torch's float8_e4m3fn conversion (round to
+  nearest even) below the saturation point and saturates at +-448 above it; per
+  block the amax element maps to +-448 and every element lies within half an e4m3
+  step of its code; with quant = 2, topk = 1 equals softmax attention on the
+  decoded codes and general topk equals the dense brute force on them
 * forward          -- topk = 1 equals dense softmax attention from
   torch's float64 scaled_dot_product_attention; topk = 0 equals closed-form
   linear attention phi(Q)(phi(K)^T V) / phi(Q)(phi(K)^T 1) ("TurboDiffusion
@@ -235,6 +240,96 @@ def pin_quant_smoothing(lib):
 
 
 # --------------------------------------------------------------------------
+# FP8 e4m3
+# --------------------------------------------------------------------------
+
+def _torch_e4m3(x):
+    torch = pytest.importorskip("torch")
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.float().numpy(), t.view(torch.uint8).numpy()
+
+
+def _e4m3_grid():
+    """All finite e4m3 values (decoded from every bit pattern but the NaNs)."""
+    torch = pytest.importorskip("torch")
+    b = torch.arange(256, dtype=torch.uint8)
+    v = b.view(torch.float8_e4m3fn).float().numpy()
+    return np.unique(v[np.isfinite(v)])
+
+
+def pin_fp8_encoder(lib):
+    rng = np.random.default_rng(21)
+    grid = _e4m3_grid()
+    pos = grid[grid > 0]
+    mids = ((pos[:-1].astype(np.float64) + pos[1:]) / 2).astype(np.float32)  # exact in fp32: ties
+    xs = [rng.standard_normal(20000).astype(np.float32) * np.float32(sc) for sc in (1e-4, 3e-3, 0.1, 1, 30, 150)]
+    xs += [grid, mids, -mids, np.array([447.9, 448.0, 455.0, 463.99, 0.0, -0.0], dtype=np.float32)]
+    x = np.concatenate(xs).astype(np.float32)
+    x = x[np.abs(x) < 464]
+    val, bits = oracle.e4m3(x, lib=lib)
+    tv, tb = _torch_e4m3(x)
+    assert np.array_equal(val, tv)
+    assert np.array_equal(bits, tb)
+    # ties go to the even mantissa: both neighbours of a midpoint are taken, in turn
+    mv, _ = oracle.e4m3(mids, lib=lib)
+    assert 0.3 < np.mean(mv == pos[1:]) < 0.7
+    # saturation (what the conversion to e4m3 with satfinite does)
+    big = np.array([464.0, 480.0, 1000.0, 3e38, -464.0, -1e9], dtype=np.float32)
+    bv, bb = oracle.e4m3(big, lib=lib)
+    assert np.array_equal(bv, np.sign(big) * 448.0)
+    assert np.array_equal(bb, np.where(big > 0, 0x7E, 0xFE).astype(np.uint8))
+
+
+def pin_fp8_quant(lib):
+    torch = pytest.importorskip("torch")
+    q, k, _ = _qkv((3, 10, 7), d=128, seed=22, adversarial=("outliers",))   # N = 210, ragged
+    dec = lambda c: torch.from_numpy(np.ascontiguousarray(c).view(np.uint8)).view(torch.float8_e4m3fn).float().numpy()
+    for blk_q, blk_k in ((128, 64), (64, 64)):
+        q8, k8, sq, sk, km = oracle.quantize(q, k, blk_q, blk_k, lib=lib, fp8=True)
+        _, _, _, _, km_i8 = oracle.quantize(q, k, blk_q, blk_k, lib=lib)
+        assert np.array_equal(km, km_i8)                      # same smoothing mean as INT8
+        N = q.shape[2]
+        qf = synth.bf16_bits_to_f64(q[0, 0]).astype(np.float32)
+        kf = synth.bf16_bits_to_f64(k[0, 0]).astype(np.float32) - km[0]
+        for name, x, codes, s, blk in (("q", qf, q8, sq, blk_q), ("k", kf, k8, sk, blk_k)):
+            c = dec(codes[0, 0]).astype(np.float64)
+            assert np.isfinite(c).all() and np.abs(c).max() <= 448
+            for I in range(-(-N // blk)):
+                xb = x[I * blk:(I + 1) * blk].astype(np.float64)
+                cb = c[I * blk:(I + 1) * blk]
+                sc = float(s[0, I])
+                assert sc == np.float32(np.float32(np.abs(xb).max()) / np.float32(448.0))
+                a = np.unravel_index(np.argmax(np.abs(xb)), xb.shape)
+                assert abs(cb[a]) == 448 and np.sign(cb[a]) == np.sign(xb[a]), (name, I)
+                # within half an e4m3 step: 2^-4 relative for normal codes, 2^-10 absolute below 2^-6
+                step = np.where(np.abs(cb) >= 2.0 ** -6, np.abs(cb) * 2.0 ** -3, 2.0 ** -9)
+                assert (np.abs(xb / sc - cb) <= 0.5 * step * (1 + 1e-6) + 1e-7).all(), (name, I)
+
+
+def pin_fp8_forward(lib):
+    torch = pytest.importorskip("torch")
+    dec = lambda c: torch.from_numpy(np.ascontiguousarray(c).view(np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+    q, k, v = _qkv((3, 10, 7), d=64, H=2, seed=23)           # N = 210, ragged
+    for blk_q, blk_k, topk, ph in ((64, 64, 1.0, 0), (128, 64, 0.5, 1), (64, 32, 0.3, 0)):
+        out, os_, ol = oracle.forward(q, k, v, blk_q, blk_k, topk, phi=ph, quant=2, branches=True, lib=lib)
+        idx, _ = oracle.block_mask(q, k, blk_q, blk_k, topk, lib=lib)
+        q8, k8, sq, sk, _ = oracle.quantize(q, k, blk_q, blk_k, lib=lib, fp8=True)
+        N, d = q.shape[2], q.shape[3]
+        for h in range(2):
+            rs = np.repeat(sq[h].astype(np.float64), blk_q)[:N]
+            cs = np.repeat(sk[h].astype(np.float64), blk_k)[:N]
+            lg = (dec(q8[0, h]) @ dec(k8[0, h]).T) * rs[:, None] * cs[None, :] / np.sqrt(d)
+            ref, rs_, rl = sla_dense(q[0, h], k[0, h], v[0, h], idx[h], blk_q, blk_k, ph, logits=lg)
+            for a, b in ((out[0, h], ref), (os_[0, h], rs_), (ol[0, h], rl)):
+                err = np.abs(a - b).max() / max(np.abs(b).max(), 1e-300)
+                assert err < 1e-10, (blk_q, topk, h, err)
+            if topk == 1.0:  # all selected: softmax attention on the decoded codes
+                P = torch.softmax(torch.from_numpy(lg), dim=-1).numpy()
+                dense = P @ synth.bf16_bits_to_f64(v[0, h])
+                assert np.abs(out[0, h] - dense).max() / np.abs(dense).max() < 1e-12
+
+
+# --------------------------------------------------------------------------
 # forward
 # --------------------------------------------------------------------------
 
@@ -331,7 +426,7 @@ def pin_forward_rows(lib):
 PINS = [pin_topk_count, pin_mask_exhaustive, pin_mask_invariances, pin_mask_degenerate,
         pin_quant_exact_block, pin_quant_bounds, pin_quant_smoothing, pin_forward_dense_limit,
         pin_forward_linear_limit, pin_forward_bruteforce, pin_forward_constant_v, pin_forward_hull,
-        pin_forward_relu_zero, pin_forward_rows]
+        pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
