@@ -45,7 +45,7 @@ ATTN_SRC = os.path.join(ROOT, "sparse_linear_bit_b200", "csrc", "sla_attention.c
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = {1: 10, 0: 8}  # our launches per sla_forward call (quant on / off)
+KERNELS_PER_STEP = {2: 10, 1: 10, 0: 8}  # our launches per sla_forward call (fp8 / int8 / off)
 
 
 def parse():
@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b-720p")
     ap.add_argument("--topk", type=float, default=0.10)
-    ap.add_argument("--quant", type=int, default=1)
+    ap.add_argument("--quant", type=int, default=1, choices=[0, 1, 2], help="0 none, 1 INT8, 2 FP8 e4m3")
     ap.add_argument("--phi", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,7 +85,7 @@ def workload_config(w, a):
     nbytes = w.B * w.H * w.N * w.d * 2
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "grid_thw": list(w.grid),
             "blk_q": w.blk_q, "blk_k": w.blk_k, "topk": a.topk, "phi": ["elu+1", "relu"][a.phi],
-            "quant": "int8 Q/K, bf16 P.V" if a.quant else "bf16 Q.K^T, fp16 P.V",
+            "quant": {1: "int8 Q/K, bf16 P.V", 2: "fp8 e4m3 Q/K, bf16 P.V"}.get(a.quant, "bf16 Q.K^T, fp16 P.V"),
             "l2": ("inputs (3 x %.2f GB) exceed the 126 MB L2; no flush between steps" if 3 * nbytes > 126e6 else
                    "inputs (3 x %.3f GB) fit in L2: steps run warm") % (nbytes / 1e9)}
 
@@ -359,7 +359,7 @@ def main():
     ops_qk, ops_pv = 2.0 * macs, 2.0 * macs
     ops_lin = 2.0 * wl.B * wl.H * n_qb * 128.0 * w.d * w.d  # phi(Q_I) H_I, tf32
     p_bf16 = float(peaks["bf16_tflops"]) * 1e12
-    p_qk = 2.0 * p_bf16 if a.quant else p_bf16  # int8 = 2x bf16 (nominal ratio)
+    p_qk = 2.0 * p_bf16 if a.quant else p_bf16  # int8 and fp8 = 2x bf16 (nominal ratio)
     p_tf32 = 0.5 * p_bf16
     t_attn = stage_ms["attention"] * 1e-3
     ideal = ops_qk / p_qk + ops_pv / p_bf16 + ops_lin / p_tf32
@@ -369,8 +369,8 @@ def main():
     traffic = recorded_traffic(w.name, a.topk, a.quant)
     roofline = {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s (burst); int8 = 2x, tf32 = 0.5x",
-                "ops_per_launch": {"qk_int8" if a.quant else "qk_bf16": ops_qk, "pv_bf16": ops_pv,
+                "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s (burst); int8/fp8 = 2x, tf32 = 0.5x",
+                "ops_per_launch": {{0: "qk_bf16", 1: "qk_int8", 2: "qk_fp8"}[a.quant]: ops_qk, "pv_bf16": ops_pv,
                                    "linear_tf32": ops_lin},
                 "launch_ms": stage_ms["attention"]}
 
@@ -386,7 +386,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": a.steps,
                 "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": a.scaling,
-                "vs_baseline": None, "dtype": "i8+bf16" if a.quant else "bf16+fp16", "data": "synthetic",
+                "vs_baseline": None, "dtype": {0: "bf16+fp16", 1: "i8+bf16", 2: "fp8e4m3+bf16"}[a.quant],
+                "data": "synthetic",
                 "config": dict(workload_config(w, a), parallelism=(
                     f"{world} rank(s), one per GPU; " + ("each runs the whole workload" if a.scaling == "weak"
                                                          else "B*H heads split in contiguous ranges"))),

@@ -18,14 +18,18 @@
  *      with one fused multiply-add per channel; per query block I the k_sel key
  *      blocks first in the order (score descending, block index ascending) are
  *      selected, k_sel = sla_topk_count(n_kb, topk);
- *   3. (quant = 1) K smoothed by its per-channel mean over all N tokens; Q and
- *      the smoothed K quantised to INT8 with one fp32 scale per block
- *      (scale = amax/127, code = clamp(rint_even(x/scale), +-127), IEEE fp32);
+ *   3. (quant = 1 or 2) K smoothed by its per-channel mean over all N tokens;
+ *      Q and the smoothed K quantised with one fp32 scale per block: INT8 with
+ *      quant = 1 (scale = amax/127, code = clamp(rint_even(x/scale), +-127)),
+ *      FP8 e4m3 with quant = 2 (scale = amax/448, code = the e4m3 value
+ *      nearest to x/scale, ties to even, saturating at +-448; the same section
+ *      names FP8 beside INT8); every step in IEEE fp32;
  *   4. sparse branch: per query row, exact softmax attention over the tokens of
  *      the selected key blocks; logits (qhat.khat)*s_q*s_k/sqrt(d) with
- *      quant = 1, (q.k)/sqrt(d) in bf16 x bf16 -> fp32 with quant = 0; P.V
- *      with P rounded to bf16 (quant = 1) or to fp16 against an fp16 copy of
- *      V (quant = 0; V entries beyond +-65504 saturate), fp32 accumulation;
+ *      quant = 1 or 2 (INT8 MMA with int32 sums, or FP8 MMA with fp32 sums),
+ *      (q.k)/sqrt(d) in bf16 x bf16 -> fp32 with quant = 0; P.V with P
+ *      rounded to bf16 (quant = 1, 2) or to fp16 against an fp16 copy of V
+ *      (quant = 0; V entries beyond +-65504 saturate), fp32 accumulation;
  *   5. linear branch over the unselected key blocks:
  *      phi(q)^T H_I / (phi(q) . Z_I), H_I = sum_{J unselected} phi(K_J)^T V_J,
  *      Z_I = sum_{J unselected} (column sums of phi(K_J)); phi acts on the raw
@@ -116,7 +120,17 @@ SLA_API sla_status sla_quantize_qk(const void *q_bf16, const void *k_bf16, int B
                            int blk_q, int blk_k, int8_t *q_i8, int8_t *k_i8, float *q_scale,
                            float *k_scale, float *k_mean, void *ws, size_t ws_bytes, void *stream);
 
-/* The whole forward, steps 1-6.  out: bf16 [B, H, N, d]. */
+/* Step 3 with FP8 e4m3 codes (the codes sla_forward uses with quant = 2).
+ *   q_fp8, k_fp8  uint8 [B, H, N, d] e4m3 bit patterns (k_fp8: the smoothed K)
+ *   q_scale, k_scale, k_mean as for sla_quantize_qk (scales are amax / 448).
+ * Codes are bit-exact with the fp32 definition above (a code that rounds to
+ * zero keeps the sign of x). */
+SLA_API sla_status sla_quantize_qk_fp8(const void *q_bf16, const void *k_bf16, int B, int H, int N, int d,
+                               int blk_q, int blk_k, uint8_t *q_fp8, uint8_t *k_fp8, float *q_scale,
+                               float *k_scale, float *k_mean, void *ws, size_t ws_bytes, void *stream);
+
+/* The whole forward, steps 1-6.  quant: 0 = none, 1 = INT8, 2 = FP8 e4m3.
+ * out: bf16 [B, H, N, d]. */
 SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                        size_t ws_bytes, void *stream);

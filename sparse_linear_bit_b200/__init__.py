@@ -25,7 +25,7 @@ from typing import Optional
 
 __all__ = [
     "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
-    "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_forward", "sla_check", "workspace",
+    "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_quantize_qk_fp8", "sla_forward", "sla_check", "workspace",
     "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
     "sla_block_mask_noalloc_limit", "head_shard", "shard_heads",
 ]
@@ -54,6 +54,8 @@ lib.sla_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _
 lib.sla_block_mask.restype = _I
 lib.sla_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]
 lib.sla_quantize_qk.restype = _I
+lib.sla_quantize_qk_fp8.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _SZ, _P]
+lib.sla_quantize_qk_fp8.restype = _I
 lib.sla_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P]
 lib.sla_forward.restype = _I
 lib.sla_forward_profile.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P,
@@ -171,6 +173,13 @@ def sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws
     _ok(lib.sla_quantize_qk(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, _ptr(q_i8), _ptr(k_i8), _ptr(q_scale),
                             _ptr(k_scale), _ptr(k_mean), _ptr(ws), ws.numel() * ws.element_size(),
                             _stream(stream)), "sla_quantize_qk")
+
+
+def sla_quantize_qk_fp8(q, k, blk_q, blk_k, q_fp8, k_fp8, q_scale, k_scale, k_mean, ws, stream=None) -> None:
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_quantize_qk_fp8(_ptr(q), _ptr(k), B, H, N, d, blk_q, blk_k, _ptr(q_fp8), _ptr(k_fp8),
+                                _ptr(q_scale), _ptr(k_scale), _ptr(k_mean), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)), "sla_quantize_qk_fp8")
 
 
 def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -> None:

@@ -129,6 +129,34 @@ char *ws_at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
 
 }  // namespace
 
+namespace sla {
+sla_status quantize_qk(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k, int fp8,
+                           int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale, float *k_mean, void *ws,
+                           size_t ws_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, 0.0f);
+    if (st != SLA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(ws) || !aligned16(q_i8) || !aligned16(k_i8))
+        return SLA_ERR_INVALID_ARG;
+    if (!q_scale || !k_scale || ((uintptr_t)q_scale & 3u) || ((uintptr_t)k_scale & 3u) ||
+        (k_mean && ((uintptr_t)k_mean & 3u)))
+        return SLA_ERR_INVALID_ARG;
+    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, 0.0f, 1);
+    const Layout L = make_layout(g);
+    if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
+    double *kbar = reinterpret_cast<double *>(ws_at(ws, L.kbar));
+    double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
+    float *mean = k_mean ? k_mean : reinterpret_cast<float *>(ws_at(ws, L.kmean));
+    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, kpart, s));
+    SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), mean, s));
+    SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, nullptr, fp8, s));
+    SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, nullptr, fp8, s));
+    return SLA_OK;
+}
+}  // namespace sla
+
 extern "C" {
 
 const char *sla_version(void) { return "sla-b200 0.1.0 (sm_100a)"; }
@@ -150,14 +178,14 @@ int sla_topk_count(int n_kb, float topk) { return topk_count(n_kb, topk); }
 
 size_t sla_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant)
 {
-    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || quant < 0 || quant > 2) return 0;
     return make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant)).total;
 }
 
 int sla_workspace_layout(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant, size_t *offsets,
                          int n)
 {
-    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || (quant != 0 && quant != 1)) return 0;
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || quant < 0 || quant > 2) return 0;
     const Layout L = make_layout(make_geometry(B, H, N, d, blk_q, blk_k, topk, quant));
     const size_t v[17] = {L.status, L.qbar,  L.kbar,   L.scores,   L.idx,  L.amask, L.q8,  L.k8,   L.qscale,
                           L.kscale, L.kmean, L.states, L.partials, L.htot, L.hq,    L.v16, L.kpart};
@@ -193,26 +221,15 @@ sla_status sla_quantize_qk(const void *q, const void *k, int B, int H, int N, in
                            int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale, float *k_mean, void *ws,
                            size_t ws_bytes, void *stream)
 {
-    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, 0.0f);
-    if (st != SLA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(ws) || !aligned16(q_i8) || !aligned16(k_i8))
-        return SLA_ERR_INVALID_ARG;
-    if (!q_scale || !k_scale || ((uintptr_t)q_scale & 3u) || ((uintptr_t)k_scale & 3u) ||
-        (k_mean && ((uintptr_t)k_mean & 3u)))
-        return SLA_ERR_INVALID_ARG;
-    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, 0.0f, 1);
-    const Layout L = make_layout(g);
-    if (ws_bytes < L.total) return SLA_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SLA_TRY(cudaMemsetAsync(ws_at(ws, L.status), 0, sizeof(int), s));
-    double *kbar = reinterpret_cast<double *>(ws_at(ws, L.kbar));
-    double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
-    float *mean = k_mean ? k_mean : reinterpret_cast<float *>(ws_at(ws, L.kmean));
-    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, kpart, s));
-    SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), mean, s));
-    SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q_i8, q_scale, nullptr, s));
-    SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, mean, k_i8, k_scale, nullptr, s));
-    return SLA_OK;
+    return quantize_qk(q, k, B, H, N, d, blk_q, blk_k, 0, q_i8, k_i8, q_scale, k_scale, k_mean, ws, ws_bytes, stream);
+}
+
+sla_status sla_quantize_qk_fp8(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k,
+                               uint8_t *q_fp8, uint8_t *k_fp8, float *q_scale, float *k_scale, float *k_mean,
+                               void *ws, size_t ws_bytes, void *stream)
+{
+    return quantize_qk(q, k, B, H, N, d, blk_q, blk_k, 1, reinterpret_cast<int8_t *>(q_fp8),
+                       reinterpret_cast<int8_t *>(k_fp8), q_scale, k_scale, k_mean, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -229,7 +246,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
     if (st != SLA_OK) return st;
     if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_RELU) return SLA_ERR_INVALID_ARG;
-    if (quant != 0 && quant != 1) return SLA_ERR_INVALID_ARG;
+    if (quant < 0 || quant > 2) return SLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
         return SLA_ERR_INVALID_ARG;
     const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, topk, quant);
@@ -259,7 +276,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     mark();
     // (1) Q: INT8 codes and scales, with the pooled block means as a by-product
     //     (without quantisation: the pooled means alone)
-    if (quant) SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, qbar, s));
+    if (quant) SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, qbar, quant == 2, s));
     else SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
     mark();
     // (2) pooled block means of K (and its partial sums for the smoothing mean),
@@ -275,7 +292,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     // (4) K: smoothing mean, INT8 codes and scales
     if (quant) {
         SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), kmean, s));
-        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, nullptr, s));
+        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, nullptr, quant == 2, s));
     }
     mark();
     // (5) per-query-block state

@@ -5,8 +5,9 @@
 // ("TurboDiffusion技术架构解析" §2.1, standard attention formula) over the tokens
 // of the key blocks the query block selected, computed SageAttention-style
 // ("清华开源TurboDiffusion加速框架", SageAttention与稀疏计算): INT8 Q.K^T on the
-// tensor cores with per-block fp32 dequantisation scales, online softmax in
-// fp32, P rounded to bf16 for a bf16 P.V with fp32 accumulation.  With
+// tensor cores with per-block fp32 dequantisation scales (or FP8 e4m3 codes
+// on the f8f6f4 tensor-core path with fp32 sums), online softmax in fp32, P
+// rounded to bf16 for a bf16 P.V with fp32 accumulation.  With
 // quantisation off, Q.K^T runs in bf16 and P.V in fp16 (P and an fp16 copy of
 // V, 8x finer rounding than bf16), both with fp32 accumulation.
 //
@@ -63,7 +64,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: P may grow to 2^8 before O is rescaled
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 
-template <bool QUANT>
+template <bool QUANT>  // QUANT: 8-bit Q/K codes (INT8 or FP8)
 struct AttnCfg {
     static constexpr uint32_t kKBytes = QUANT ? 2 * kBox : 4 * kBox;        // K of a pair of key blocks
     static constexpr uint32_t kVBytes = 4 * kBox;                           // V of a pair of key blocks
@@ -112,12 +113,13 @@ SLA_DEV void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, u
 }
 
 // Row max over this thread's 64 tile columns, in logit units (log2 domain).
-// QUANT: raw int32 dot products; adding the 1.5 * 2^23 bias to the bits makes them
+// INT_S: raw int32 dot products; adding the 1.5 * 2^23 bias to the bits makes them
 // floats 12582912 + d (exact for |d| < 2^22), which is also how tile_exp reads them.
-template <bool QUANT, bool MASKED>
+// Otherwise the logits are fp32 already.
+template <bool INT_S, bool MASKED>
 SLA_DEV float tile_max(uint32_t (&sv)[64], int valid, float c)
 {
-    if (QUANT) {
+    if (INT_S) {
 #pragma unroll
         for (int k = 0; k < 64; ++k) sv[k] += 0x4B400000u;
     }
@@ -135,11 +137,11 @@ SLA_DEV float tile_max(uint32_t (&sv)[64], int valid, float c)
 #pragma unroll
     for (int k = 0; k < 7; ++k) tt[k] = fmax3f(tt[3 * k], tt[3 * k + 1], tt[3 * k + 2]);
     const float xmax = fmax3f(fmax3f(tt[0], tt[1], tt[2]), fmax3f(tt[3], tt[4], tt[5]), fmaxf(tt[6], tt[21]));
-    return (QUANT ? (xmax - 12582912.0f) : xmax) * c;  // c >= 0
+    return (INT_S ? (xmax - 12582912.0f) : xmax) * c;  // c >= 0
 }
 
 // P = exp2(x * c + off) for the 64 columns, packed two per 32-bit word; returns the row sum.
-template <bool QUANT, bool MASKED>
+template <bool P_BF16, bool MASKED>
 SLA_DEV float tile_exp(const uint32_t (&sv)[64], int valid, float c, float off, uint32_t (&pk)[32])
 {
     const uint64_t c2 = f2pack(c, c), off2 = f2pack(off, off);
@@ -153,10 +155,19 @@ SLA_DEV float tile_exp(const uint32_t (&sv)[64], int valid, float c, float off, 
             if (k + 1 >= valid) p1 = 0.0f;
         }
         acc2[(k >> 1) & 3] = add2(acc2[(k >> 1) & 3], f2pack(p0, p1));
-        pk[k >> 1] = QUANT ? pack_bf16x2(p0, p1) : pack_f16x2_sat(p0, p1);
+        pk[k >> 1] = P_BF16 ? pack_bf16x2(p0, p1) : pack_f16x2_sat(p0, p1);
     }
     const float2 s01 = f2unpack(add2(add2(acc2[0], acc2[1]), add2(acc2[2], acc2[3])));
     return s01.x + s01.y;
+}
+
+SLA_DEV void mma_f8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc_, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc_), "r"(accumulate)
+        : "memory");
 }
 
 SLA_DEV void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc_, uint32_t accumulate)
@@ -171,7 +182,9 @@ SLA_DEV void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, ui
 // descriptor + byte offset (the start-address field is the low 14 bits, in 16 B units)
 SLA_DEV uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
 
-template <bool QUANT>
+// MODE 0: bf16 Q.K^T, fp16 P.V; 1: INT8 Q.K^T (int32 logits); 2: FP8 e4m3 Q.K^T (fp32
+// logits); P.V in bf16 for both quantised modes.
+template <int MODE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
             const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_qr,
@@ -180,6 +193,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const int32_t *__restrict__ idx, const float *__restrict__ hq, int N, int blk_q, int n_qb, int n_kb,
             int k_sel, int phi, uint16_t *__restrict__ out, int *status)
 {
+    constexpr bool QUANT = MODE != 0, INT_S = MODE == 1;
     using Cfg = AttnCfg<QUANT>;
     constexpr int NS = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -317,7 +331,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     } else if (warp >= 10) {
         // ------------------------------------------------------------ Q.K^T + P.V issuer of group g
         const int g = warp - 10;
-        constexpr uint32_t id_qk = QUANT ? idesc(2, 1, 1, 0, 0, 128, 64) : idesc(1, 1, 1, 0, 0, 128, 64);
+        // S32 <- s8 x s8 (INT8), F32 <- e4m3 x e4m3 (FP8), F32 <- bf16 x bf16
+        constexpr uint32_t id_qk = MODE == 1   ? idesc(2, 1, 1, 0, 0, 128, 64)
+                                   : MODE == 2 ? idesc(1, 0, 0, 0, 0, 128, 64)
+                                               : idesc(1, 1, 1, 0, 0, 128, 64);
         constexpr uint32_t id_pv = QUANT ? idesc(1, 1, 1, 0, 1, 128, 128) : idesc(1, 0, 0, 0, 1, 128, 128);
         const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
         const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), 2 * kBox, 1024);
@@ -331,9 +348,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tc_fence_after();
             const uint64_t kd = dadd(kd0, (t % NS) * Cfg::kStageBytes + g * kBox);
             if (elect_one()) {
-                if (QUANT) {  // K-step of 32 int8 = 8 TMEM columns of Q
+                if (MODE == 1) {  // K-step of 32 int8 = 8 TMEM columns of Q
 #pragma unroll
                     for (int k = 0; k < 4; ++k) mma_i8_tmem_a(s_g, t_q + 8 * k, kd + 2 * k, id_qk, k > 0 ? 1u : 0u);
+                } else if (MODE == 2) {  // K-step of 32 e4m3 = 8 TMEM columns of Q
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma_f8_tmem_a(s_g, t_q + 8 * k, kd + 2 * k, id_qk, k > 0 ? 1u : 0u);
                 } else {  // K-step of 16 bf16 = 8 TMEM columns of Q
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
@@ -455,7 +475,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const bool tok_ready = mbar_test(&sm.tok[g][quarter], t & 1);
             const int valid = min(64, N - J * 64);
             // the two paths are separate instantiations so the full-tile path carries no masking
-            const float tmax = valid == 64 ? tile_max<QUANT, false>(sv, 64, c) : tile_max<QUANT, true>(sv, valid, c);
+            const float tmax = valid == 64 ? tile_max<INT_S, false>(sv, 64, c) : tile_max<INT_S, true>(sv, valid, c);
             const float m_new = fmaxf(m_used, tmax);
             const bool need = m_new > m_used + kRescaleThreshold;  // also true on the first block
             float alpha = 1.0f;
@@ -468,7 +488,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             if (!__all_sync(0xffffffffu, tok_ready) && !(ok = wait_all(&sm.tok[g][quarter], t & 1))) break;
             const bool pv_ready = t == 0 || mbar_test(&sm.bar_pv[g], (t - 1) & 1);
             uint32_t pk[32];
-            const float off = QUANT ? -fmaf(kBias, c, m_used) : -m_used;
+            const float off = INT_S ? -fmaf(kBias, c, m_used) : -m_used;
             if (valid == 64) l += tile_exp<QUANT, false>(sv, 64, c, off, pk);
             else l += tile_exp<QUANT, true>(sv, valid, c, off, pk);
             __syncwarp();
@@ -578,11 +598,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     }
 }
 
-template <bool QUANT>
+template <int MODE>
 cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int8_t *q8, const int8_t *k8,
                           const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
                           const Geometry &g, int phi, void *out, int *status, cudaStream_t s)
 {
+    constexpr bool QUANT = MODE != 0;
     CUtensorMap tk, tv, th, tq;
     const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
     if (QUANT) {
@@ -613,10 +634,10 @@ cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int
         if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, st, bq)) return cudaErrorInvalidValue;
     }
     const size_t smem = sizeof(AttnSmem<QUANT>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<QUANT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(g.n_qb, g.BH);
-    attn_kernel<QUANT><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, tq, static_cast<const uint16_t *>(q), q8, qscale,
+    attn_kernel<MODE><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, tq, static_cast<const uint16_t *>(q), q8, qscale,
                                                         kscale, idx, hq, g.N, g.blk_q, g.n_qb, g.n_kb, g.k_sel, phi,
                                                         static_cast<uint16_t *>(out), status);
     return cudaGetLastError();
@@ -628,8 +649,9 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
                              const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
                              const Geometry &g, int phi, void *out, int *status, cudaStream_t s)
 {
-    if (g.quant) return launch_attn_t<true>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
-    return launch_attn_t<false>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
+    if (g.quant == 2) return launch_attn_t<2>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
+    if (g.quant == 1) return launch_attn_t<1>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
+    return launch_attn_t<0>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
 }
 
 }  // namespace sla

@@ -38,9 +38,10 @@ cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry
                           cudaStream_t s);
 cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap,
                         uint16_t *amask, cudaStream_t s);
-// INT8 codes and scales; with `bmean` (no smoothing) also the fp64 block means
+// INT8 (fp8 = 0) or FP8 e4m3 (fp8 = 1) codes and scales; with `bmean` (no smoothing) also the
+// fp64 block means
 cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out,
-                         float *scale, double *bmean, cudaStream_t s);
+                         float *scale, double *bmean, int fp8, cudaStream_t s);
 
 // linear branch and fused attention (tcgen05)
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states,

@@ -27,6 +27,14 @@
 namespace sla {
 namespace {
 
+// two fp32 -> packed fp8 e4m3 (lo in the low byte), round to nearest even, saturating at +-448
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8])
 {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -427,11 +435,16 @@ __global__ void zero_u32_kernel(uint32_t *p, size_t n)
 // the fast path |t| <= 127 (1 + 3 * 2^-24), so rint(t) needs no clamp, and the
 // low byte of the bits of t + 1.5 * 2^23 (which rounds t to an integer, ties to
 // even) is rint(t) in two's complement.
+//
+// FP8 (e4m3) codes: s = amax / 448 and code = e4m3(fl(x / s)), round to nearest
+// even with saturation (SageAttention's FP8 option beside INT8).  The same
+// reciprocal product is used; |t - fl(x/s)| < 2^-22 |t|, so when t (1 - 2^-20)
+// and t (1 + 2^-20) convert to the same code it is the quotient's code.
 // ---------------------------------------------------------------------------
 // When `bmean` is given (Q only), the kernel also writes the block's fp64 mean
 // row, the pooled mean that block selection scores with (exact fp64 sums, so the
 // same values as the pooling kernel's).
-template <bool SMOOTH, int BLK>
+template <bool SMOOTH, int BLK, bool FP8>
 __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
                                                     const float *__restrict__ mean, uint2 *__restrict__ out,
                                                     float *__restrict__ scale, double *__restrict__ bmean)
@@ -497,7 +510,7 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
     amax = warp_max[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
-    const float s = __fdiv_rn(amax, 127.0f);
+    const float s = __fdiv_rn(amax, FP8 ? 448.0f : 127.0f);
     if (threadIdx.x == 0) scale[(size_t)bh * nb + J] = s;
     const float r = s != 0.0f ? __fdiv_rn(1.0f, s) : 0.0f;
     const bool fast = s != 0.0f && isfinite(r);
@@ -509,29 +522,53 @@ __global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x,
         if ((e >> 4) < rows) {
             float f[8];
             expand(raw[l], f);
-            // fast path: the low byte of the bits of t + kRound is rint(t) as int8 (|t| <= 127 here)
-            uint32_t cb[8];
-            unsigned slow = fast ? 0u : 0xFFu;
+            uint32_t w0, w1;
+            if (FP8) {
+                // The e4m3 code of t = fl(x * r) is that of the IEEE quotient unless a rounding
+                // boundary of e4m3 lies within 2^-22 |t| of t (see above): t (1 -+ 2^-20) bracket
+                // that interval, so equal codes at both ends settle it.
+                uint32_t c[4], slow = fast ? 0u : 0xFu;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float t = f[i] * r;
-                const float qf = __fadd_rn(t, kRound);
-                const float rt = __fsub_rn(qf, kRound);
-                if (fabsf(t - rt) > 0.5f - 6.103515625e-05f) slow |= 1u << i;
-                cb[i] = __float_as_uint(qf);
-            }
-            if (slow) {  // rare: within 2^-14 of a half-integer, or a zero / tiny scale
+                for (int i = 0; i < 4; ++i) {
+                    const float t0 = f[2 * i] * r, t1 = f[2 * i + 1] * r;
+                    const uint32_t lo = e4m3x2(t0 * (1.0f - 9.5367431640625e-07f), t1 * (1.0f - 9.5367431640625e-07f));
+                    const uint32_t hi = e4m3x2(t0 * (1.0f + 9.5367431640625e-07f), t1 * (1.0f + 9.5367431640625e-07f));
+                    if (lo != hi) slow |= 1u << i;
+                    c[i] = lo;
+                }
+                if (slow) {  // rare: near an e4m3 rounding boundary, or a zero / tiny scale
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (slow & (1u << i))
+                            c[i] = s != 0.0f ? e4m3x2(__fdiv_rn(f[2 * i], s), __fdiv_rn(f[2 * i + 1], s)) : 0u;
+                }
+                w0 = c[0] | (c[1] << 16);
+                w1 = c[2] | (c[3] << 16);
+            } else {
+                // fast path: the low byte of the bits of t + kRound is rint(t) as int8 (|t| <= 127 here)
+                uint32_t cb[8];
+                unsigned slow = fast ? 0u : 0xFFu;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    if (slow & (1u << i)) {
-                        int c = 0;
-                        if (s != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(f[i], s))));
-                        cb[i] = (uint32_t)c;
+                    const float t = f[i] * r;
+                    const float qf = __fadd_rn(t, kRound);
+                    const float rt = __fsub_rn(qf, kRound);
+                    if (fabsf(t - rt) > 0.5f - 6.103515625e-05f) slow |= 1u << i;
+                    cb[i] = __float_as_uint(qf);
+                }
+                if (slow) {  // rare: within 2^-14 of a half-integer, or a zero / tiny scale
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (slow & (1u << i)) {
+                            int c = 0;
+                            if (s != 0.0f) c = max(-127, min(127, __float2int_rn(__fdiv_rn(f[i], s))));
+                            cb[i] = (uint32_t)c;
+                        }
                     }
                 }
+                w0 = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+                w1 = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
             }
-            const uint32_t w0 = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
-            const uint32_t w1 = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
             ob[e] = make_uint2(w0, w1);
         }
     }
@@ -592,18 +629,21 @@ cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, u
 }
 
 cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out, float *scale,
-                         double *bmean, cudaStream_t s)
+                         double *bmean, int fp8, cudaStream_t s)
 {
     dim3 grid(nb, BH);
     const uint4 *xi = static_cast<const uint4 *>(x);
     uint2 *o = reinterpret_cast<uint2 *>(out);
     if (mean) {
         if (blk != 64 || bmean) return cudaErrorInvalidValue;
-        quant_kernel<true, 64><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale, nullptr);
+        if (fp8) quant_kernel<true, 64, true><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale, nullptr);
+        else quant_kernel<true, 64, false><<<grid, 256, 0, s>>>(xi, N, nb, mean, o, scale, nullptr);
     } else if (blk == 128) {
-        quant_kernel<false, 128><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
+        if (fp8) quant_kernel<false, 128, true><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
+        else quant_kernel<false, 128, false><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
     } else if (blk == 64) {
-        quant_kernel<false, 64><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
+        if (fp8) quant_kernel<false, 64, true><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
+        else quant_kernel<false, 64, false><<<grid, 256, 0, s>>>(xi, N, nb, nullptr, o, scale, bmean);
     } else {
         return cudaErrorInvalidValue;
     }

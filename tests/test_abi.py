@@ -110,6 +110,16 @@ def test_block_mask_and_quant_host_validation():
     assert L.sla_quantize_qk(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, None, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
                              None) == 1
     assert L.sla_quantize_qk(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16, None) == 3
+    # the FP8 variant validates the same way
+    assert L.sla_quantize_qk_fp8(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, None, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                                 None) == 1
+    assert L.sla_quantize_qk_fp8(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE, 16,
+                                 None) == 3
+    assert L.sla_quantize_qk_fp8(FAKE, FAKE, 1, 2, 2048, 128, 96, 64, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                                 None) == 2
+    # quant = 2 (FP8) needs the same workspace as INT8
+    assert sla.sla_workspace_bytes(1, 2, 2048, 128, 64, 64, 0.1, 2) == sla.sla_workspace_bytes(1, 2, 2048, 128, 64,
+                                                                                              64, 0.1, 1)
     assert L.sla_check(None, None) == 1
 
 

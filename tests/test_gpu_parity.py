@@ -157,7 +157,38 @@ FWD_CASES = {
     "topk1_fp": ((1, 2, (8, 16, 16)), 128, 1.0, 0, 0),
     "topk_0p6_fp": ((1, 2, (8, 16, 16)), 128, 0.6, 0, 0),
     "ties_quant": ((1, 3, (8, 16, 16)), 128, 0.1, 0, 1),
+    # FP8 e4m3 Q.K^T (quant = 2), against the FP8 oracle
+    "tiny_fp8_elu": ((1, 2, (8, 16, 16)), 64, 0.1, 0, 2),
+    "ragged_fp8_relu": ((2, 2, (5, 9, 13)), 128, 0.2, 1, 2),
+    "multi_tile_fp8": ((1, 2, (8, 32, 32)), 128, 0.1, 0, 2),
+    "topk1_fp8": ((1, 2, (8, 16, 16)), 128, 1.0, 0, 2),
 }
+
+
+@pytest.mark.parametrize("blk_q,grid,H,adv", [
+    (128, (8, 16, 16), 2, ()),
+    (64, (3, 10, 7), 3, ("outliers",)),     # ragged N = 210, heavy-tailed K channels
+    (128, (5, 9, 13), 2, ("ties",)),
+])
+def test_quantize_fp8_bit_exact(blk_q, grid, H, adv):
+    q, k, _ = synth.make_qkv(1, H, grid, seed=17, adversarial=adv)
+    B, _, N, d = q.shape
+    n_qb, n_kb = -(-N // blk_q), -(-N // 64)
+    q8o, k8o, sqo, sko, kmo = oracle.quantize(q, k, blk_q, 64, fp8=True)
+    qd, kd = to_dev(q, torch), to_dev(k, torch)
+    q8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
+    k8 = torch.empty(q.shape, dtype=torch.uint8, device="cuda")
+    sq = torch.empty((B, H, n_qb), dtype=torch.float32, device="cuda")
+    sk = torch.empty((B, H, n_kb), dtype=torch.float32, device="cuda")
+    km = torch.empty((B, H, d), dtype=torch.float32, device="cuda")
+    ws = sla.workspace(B, H, N, d, blk_q, 64, 0.0, 2)
+    sla.sla_quantize_qk_fp8(qd, kd, blk_q, 64, q8, k8, sq, sk, km, ws)
+    sla.sla_check(ws)
+    assert np.array_equal(km.cpu().numpy().reshape(B * H, d), kmo)
+    assert np.array_equal(sq.cpu().numpy().reshape(B * H, -1), sqo)
+    assert np.array_equal(sk.cpu().numpy().reshape(B * H, -1), sko)
+    assert np.array_equal(q8.cpu().numpy(), q8o.view(np.uint8))
+    assert np.array_equal(k8.cpu().numpy(), k8o.view(np.uint8))
 
 
 @pytest.mark.parametrize("name", sorted(FWD_CASES))
