@@ -94,10 +94,13 @@ SLA_DEV float ex2(float x)
     return y;
 }
 
-SLA_DEV float phi_f(float x, int phi)
+// phi of one Q element, rounded to tf32 for the linear branch's MMA.  exp(x) for
+// x <= 0 is ex2(x log2 e) on the MUFU unit (the result is rounded to 10 mantissa
+// bits next).
+SLA_DEV float phi_tf32(float x, int phi)
 {
-    if (phi == 1) return fmaxf(x, 0.0f);
-    return x > 0.0f ? x + 1.0f : __expf(x);  // rounded to tf32 next
+    const float e = ex2(fminf(x, 0.0f) * kLog2e);  // unconditional, so both cases are a select
+    return to_tf32(phi == 1 ? fmaxf(x, 0.0f) : (x > 0.0f ? x + 1.0f : e));
 }
 
 SLA_DEV void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -528,8 +531,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 float f[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    f[2 * e] = row_valid ? to_tf32(phi_f(__uint_as_float(ww[e] << 16), phi)) : 0.0f;
-                    f[2 * e + 1] = row_valid ? to_tf32(phi_f(__uint_as_float(ww[e] & 0xFFFF0000u), phi)) : 0.0f;
+                    f[2 * e] = row_valid ? phi_tf32(__uint_as_float(ww[e] << 16), phi) : 0.0f;
+                    f[2 * e + 1] = row_valid ? phi_tf32(__uint_as_float(ww[e] & 0xFFFF0000u), phi) : 0.0f;
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) den = fmaf(f[e], sm.z[8 * u + e], den);

@@ -62,7 +62,8 @@ struct StatesSmem {
 __device__ __forceinline__ float phi_f(float x, int phi)
 {
     if (phi == 1) return fmaxf(x, 0.0f);
-    return x > 0.0f ? x + 1.0f : __expf(x);  // the result is rounded to fp16 next
+    const float e = ex2_approx(fminf(x, 0.0f) * 1.4426950408889634f);  // unconditional: a select, no branch
+    return x > 0.0f ? x + 1.0f : e;  // rounded to fp16 next
 }
 
 __global__ void __launch_bounds__(kStatesThreads, 1) states_kernel(const __grid_constant__ CUtensorMap tm_k,

@@ -342,13 +342,19 @@ SLA_DEV bool bar_and(int id, int count, bool v)
 SLA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 SLA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// round-to-nearest (ties away) fp32 -> tf32, kept in a 32-bit container
-SLA_DEV float to_tf32(float x)
+// 2^x on the MUFU unit (flushes subnormal results to zero)
+SLA_DEV float ex2_approx(float x)
 {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+
+// fp32 -> tf32 (10 mantissa bits), round to nearest with ties away from zero,
+// kept in a 32-bit container: add half the weight of the 13 dropped bits to the
+// magnitude bits (a carry moves to the next binade, as rounding up should), then
+// clear them.  Integer ALU work only (finite inputs).
+SLA_DEV float to_tf32(float x) { return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u); }
 
 SLA_DEV uint32_t pack_bf16x2(float lo, float hi)
 {
