@@ -67,6 +67,8 @@ def load(path: Optional[str] = None):
     lib.orc_block_mask.argtypes = [P, P, i32, i32, i32, i32, i32, f64, P, P, P]
     lib.orc_quantize.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P, P, P, P, P]
     lib.orc_e4m3_array.argtypes = [P, P, P, i64]
+    lib.orc_rowquant.argtypes = [P, i32, i32, i32, P, ctypes.c_float, P, P]
+    lib.orc_w8a8_linear.argtypes = [P, P, P, P, P, i32, i32, i32, P]
     lib.orc_states.argtypes = [P, P, i32, i32, i32, i32, P, P]
     lib.orc_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, f64, i32, i32, P, P, i64, P, P, P]
     lib.orc_forward.restype = i32
@@ -209,3 +211,33 @@ def forward(q, k, v, blk_q: int, blk_k: int, topk: float, phi: int = 0, quant: i
     if rc != 0:
         raise MemoryError("oracle forward failed (out of memory or bad row index)")
     return (out, os_, ol_) if branches else out
+
+
+# --------------------------------------------------------------------------
+# W8A8 INT8 linear layer with FusedNorm
+# --------------------------------------------------------------------------
+
+def rowquant(x, norm: bool = False, gamma=None, eps: float = 1e-6, lib=None):
+    """Per-row symmetric INT8 codes and fp32 scales of a bf16 matrix [rows, cols]
+    (uint16 bits), optionally after the row's RMS normalisation times gamma."""
+    lib = lib or load()
+    x = _bits(x)
+    rows, cols = x.shape
+    q = np.zeros((rows, cols), dtype=np.int8)
+    s = np.zeros(rows, dtype=np.float32)
+    g = None if gamma is None else np.ascontiguousarray(gamma, dtype=np.float32)
+    lib.orc_rowquant(_ptr(x), rows, cols, int(bool(norm)), _ptr(g), float(np.float32(eps)), _ptr(q), _ptr(s))
+    return q, s
+
+
+def w8a8_linear(qx, sx, qw, sw, bias=None, lib=None):
+    """out[m][n] = (sum_k qx[m][k] qw[n][k]) * sx[m] * sw[n] (+ bias[n]) in fp64."""
+    lib = lib or load()
+    qx, qw = np.ascontiguousarray(qx, dtype=np.int8), np.ascontiguousarray(qw, dtype=np.int8)
+    sx, sw = np.ascontiguousarray(sx, dtype=np.float32), np.ascontiguousarray(sw, dtype=np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    M, K = qx.shape
+    N = qw.shape[0]
+    out = np.zeros((M, N), dtype=np.float64)
+    lib.orc_w8a8_linear(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(b), M, N, K, _ptr(out))
+    return out

@@ -510,3 +510,65 @@ int orc_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int BH,
     free(key); free(gstart); free(idx); free(q8); free(k8); free(sq); free(sk); free(h); free(z);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架":
+ * W8A8 quantises the weights and activations of the linear layers to 8-bit
+ * integers and runs them on the INT8 units, with a FusedNorm operator; the
+ * "TurboDiffusion" GitHub summary, 主要特点 3: W8A8 accelerates the linear
+ * layers).  Granularity, rounding and the norm are not stated; the readings:
+ *   - activations: one symmetric scale per token (row), weights: one per
+ *     output channel (row of W [N, K]); scale = amax / 127 and code =
+ *     clamp(rint_even(y / scale), +-127) in IEEE fp32, the SageSLA rule;
+ *   - FusedNorm: the row's RMS normalisation fused into its quantisation:
+ *     ms = (fp64 sum of x^2) / cols rounded to fp32, r = 1 / sqrt(ms + eps)
+ *     (IEEE fp32 add, sqrt and divide), y = fp32(x * r) * gamma[c] (two fp32
+ *     products; gamma nullable = 1);
+ *   - out[m][n] = (sum_k qx[m][k] qw[n][k]) * sx[m] * sw[n] (+ bias[n]),
+ *     exact integer sum, the rest in fp64.
+ * ------------------------------------------------------------------------ */
+void orc_rowquant(const uint16_t *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,
+                  float *s)
+{
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < rows; ++m) {
+        const uint16_t *xr = x + (size_t)m * cols;
+        float *y = (float *)malloc(sizeof(float) * (size_t)cols);
+        float r = 1.0f;
+        if (norm) {
+            double ss = 0.0;
+            for (int c = 0; c < cols; ++c) ss += bf(xr[c]) * bf(xr[c]);
+            float ms = (float)(ss / (double)cols);
+            float den = sqrtf(ms + eps);
+            r = 1.0f / den;
+        }
+        float amax = 0.0f;
+        for (int c = 0; c < cols; ++c) {
+            float v = bf32(xr[c]);
+            if (norm) {
+                v = v * r;
+                if (gamma) v = v * gamma[c];
+            }
+            y[c] = v;
+            amax = fmaxf(amax, fabsf(v));
+        }
+        float sc = amax / 127.0f;
+        s[m] = sc;
+        for (int c = 0; c < cols; ++c) q[(size_t)m * cols + c] = code8(y[c], sc);
+        free(y);
+    }
+}
+
+void orc_w8a8_linear(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, const float *bias, int M,
+                     int N, int K, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int m = 0; m < M; ++m)
+        for (int n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int k = 0; k < K; ++k) acc += (int64_t)qx[(size_t)m * K + k] * (int64_t)qw[(size_t)n * K + k];
+            double v = (double)acc * (double)sx[m] * (double)sw[n];
+            if (bias) v += (double)bias[n];
+            out[(size_t)m * N + n] = v;
+        }
+}

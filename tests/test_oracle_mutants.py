@@ -32,6 +32,11 @@ MUTANTS = {
     "e4m3_exponent_bias_8": ("int e = E - 1 + 7;", "int e = E - 1 + 8;"),
     "e4m3_round_half_up": ("double r = nearbyint(ldexp(a, -qexp));", "double r = floor(ldexp(a, -qexp) + 0.5);"),
     "e4m3_no_subnormals": ("int qexp = a < ldexp(1.0, -6) ? -9 : (E - 1) - 3;", "int qexp = (E - 1) - 3;"),
+    "rowquant_sum_not_mean": ("float ms = (float)(ss / (double)cols);", "float ms = (float)ss;"),
+    "rowquant_eps_outside_sqrt": ("float den = sqrtf(ms + eps);", "float den = sqrtf(ms) + eps;"),
+    "rowquant_gamma_dropped": ("if (gamma) v = v * gamma[c];", "(void)gamma;"),
+    "w8a8_weight_scale_dropped": ("double v = (double)acc * (double)sx[m] * (double)sw[n];", "double v = (double)acc * (double)sx[m];"),
+    "w8a8_bias_subtracted": ("if (bias) v += (double)bias[n];", "if (bias) v -= (double)bias[n];"),
     "fp8_logits_raw_bytes": ("acc += e4m3_value((uint8_t)q8[(size_t)i * d + c]) * e4m3_value((uint8_t)k8[(size_t)j * d + c]);",
                              "acc += (double)q8[(size_t)i * d + c] * e4m3_value((uint8_t)k8[(size_t)j * d + c]);"),
     "no_smoothing": ("mu[c] = (float)(s / (double)N);", "mu[c] = 0.0f;"),

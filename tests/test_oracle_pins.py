@@ -18,6 +18,11 @@ of the oracle) and raises AssertionError on a mismatch.  What pins what:
   block the amax element maps to +-448 and every element lies within half an e4m3
   step of its code; with quant = 2, topk = 1 equals softmax attention on the
   decoded codes and general topk equals the dense brute force on them
+* W8A8 linear      -- per-row codes: amax -> +-127, half-step bounds, zero rows; with
+  FusedNorm the decoded rows equal torch's float32 rms_norm (eps and gamma included,
+  rows small enough for eps to matter) within half a step; the linear layer equals
+  numpy's int64 matmul of the codes times both scales plus bias, and the decoded
+  product stays within the quantisation error bound of the fp64 x w^T
 * forward          -- topk = 1 equals dense softmax attention from
   torch's float64 scaled_dot_product_attention; topk = 0 equals closed-form
   linear attention phi(Q)(phi(K)^T V) / phi(Q)(phi(K)^T 1) ("TurboDiffusion
@@ -330,6 +335,65 @@ def pin_fp8_forward(lib):
 
 
 # --------------------------------------------------------------------------
+# W8A8 INT8 linear with FusedNorm
+# --------------------------------------------------------------------------
+
+def _w8a8_inputs(seed, rows, cols, tiny_rows=0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)) * rng.uniform(0.2, 3.0, size=(rows, 1))
+    if tiny_rows:  # RMS ~ 1e-3: eps = 1e-6 is no longer negligible against the mean square
+        x[:tiny_rows] *= 1e-3
+    x[rows // 2] = 0.0  # an all-zero row
+    return _bits_from_f64(x)
+
+
+def pin_w8a8_rowquant(lib):
+    torch = pytest.importorskip("torch")
+    rows, cols = 24, 96
+    x = _w8a8_inputs(31, rows, cols, tiny_rows=4)
+    xf = synth.bf16_bits_to_f64(x)
+    gamma = np.random.default_rng(32).uniform(0.5, 1.5, cols).astype(np.float32)
+    for norm, g in ((False, None), (True, None), (True, gamma)):
+        q, s = oracle.rowquant(x, norm=norm, gamma=g, eps=1e-6, lib=lib)
+        c = q.astype(np.int64)
+        assert c.min() >= -127 and c.max() <= 127
+        if norm:
+            y = torch.nn.functional.rms_norm(torch.from_numpy(xf.astype(np.float32)), (cols,),
+                                             weight=None if g is None else torch.from_numpy(g), eps=1e-6)
+            y = y.double().numpy()
+        else:
+            y = xf
+        for m in range(rows):
+            if not np.any(xf[m]):
+                assert s[m] == 0 and not np.any(c[m])
+                continue
+            a = np.argmax(np.abs(y[m]))
+            assert abs(c[m, a]) == 127 and np.sign(c[m, a]) == np.sign(y[m, a]), (norm, m)
+            tol = 0.5 * float(s[m]) * (1 + 1e-5) + 2e-6 * np.abs(y[m]).max()
+            assert (np.abs(y[m] - c[m] * float(s[m])) <= tol).all(), (norm, m)
+
+
+def pin_w8a8_linear(lib):
+    M, N, K = 20, 12, 96
+    x = _w8a8_inputs(33, M, K)
+    w = _w8a8_inputs(34, N, K)
+    bias = np.random.default_rng(35).standard_normal(N).astype(np.float32)
+    qx, sx = oracle.rowquant(x, lib=lib)
+    qw, sw = oracle.rowquant(w, lib=lib)
+    out = oracle.w8a8_linear(qx, sx, qw, sw, bias, lib=lib)
+    ref = (qx.astype(np.int64) @ qw.astype(np.int64).T).astype(np.float64) * sx.astype(np.float64)[:, None] \
+        * sw.astype(np.float64)[None, :] + bias.astype(np.float64)[None, :]
+    assert np.allclose(out, ref, rtol=1e-14, atol=1e-14)
+    # the decoded product against the fp64 product, within the quantisation error bound
+    xf, wf = synth.bf16_bits_to_f64(x), synth.bf16_bits_to_f64(w)
+    exact = xf @ wf.T + bias.astype(np.float64)[None, :]
+    dx, dw = 0.5 * sx.astype(np.float64)[:, None], 0.5 * sw.astype(np.float64)[:, None]
+    bound = (np.abs(xf).sum(1)[:, None] * dw.T + dx * np.abs(wf).sum(1)[None, :] + K * dx * dw.T) * (1 + 1e-6)
+    assert (np.abs(out - exact) <= bound + 1e-12).all()
+    assert not np.allclose(oracle.w8a8_linear(qx, sx, qw, sw, None, lib=lib), out)
+
+
+# --------------------------------------------------------------------------
 # forward
 # --------------------------------------------------------------------------
 
@@ -426,7 +490,7 @@ def pin_forward_rows(lib):
 PINS = [pin_topk_count, pin_mask_exhaustive, pin_mask_invariances, pin_mask_degenerate,
         pin_quant_exact_block, pin_quant_bounds, pin_quant_smoothing, pin_forward_dense_limit,
         pin_forward_linear_limit, pin_forward_bruteforce, pin_forward_constant_v, pin_forward_hull,
-        pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward]
+        pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward, pin_w8a8_rowquant, pin_w8a8_linear]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
