@@ -173,6 +173,37 @@ SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void 
                                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                                        size_t ws_bytes, void *stream, float *stage_ms);
 
+/* ---- W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架",
+ * W8A8 section; "TurboDiffusion" GitHub summary, 主要特点 3: the linear layers'
+ * weights and activations quantised to 8-bit integers on the INT8 units, with
+ * a FusedNorm operator).  This is not part of the attention forward. */
+
+/* Per-row symmetric INT8 quantisation of a bf16 matrix x [rows, cols]
+ * (row-major): one fp32 scale per row, scale = amax / 127, code =
+ * clamp(rint_even(y / scale), +-127), IEEE fp32.  With norm = 1 the row is
+ * first RMS-normalised (FusedNorm): ms = (fp64 sum of x^2) / cols rounded to
+ * fp32, r = 1 / sqrt(ms + eps), y = fp32(x * r) * gamma[c] (gamma nullable =
+ * all ones; ignored when norm = 0).  Use it per token for activations and per
+ * output channel (row of W [N, K]) for weights.
+ *   q      int8 [rows, cols];  scale  fp32 [rows]
+ * Requires cols % 8 == 0 and cols <= 16384 (else SLA_ERR_UNSUPPORTED); x and q
+ * 16-byte aligned.  Codes are bit-exact with the definition above (the fp64
+ * sum of squares is exact, as for the smoothing mean). */
+SLA_API sla_status sla_w8a8_quantize(const void *x_bf16, int rows, int cols, int norm, const float *gamma,
+                             float eps, int8_t *q, float *scale, void *stream);
+
+/* Bytes of workspace sla_w8a8_linear needs (its status word, read by sla_check). */
+SLA_API size_t sla_w8a8_workspace_bytes(void);
+
+/* out[m][n] = bf16( float(sum_k qx[m][k] * qw[n][k]) * sx[m] * sw[n] + bias[n] )
+ * with qx int8 [M, K] (per-token codes), sx fp32 [M], qw int8 [N, K] (per
+ * output channel), sw fp32 [N], bias fp32 [N] (nullable), out bf16 [M, N]:
+ * an INT8 tensor-core GEMM with int32 accumulation.  Requires K % 16 == 0 and
+ * N % 8 == 0 (else SLA_ERR_UNSUPPORTED); qx, qw, out and ws 16-byte aligned. */
+SLA_API sla_status sla_w8a8_linear(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw,
+                           const float *bias, int M, int N, int K, void *out_bf16, void *ws, size_t ws_bytes,
+                           void *stream);
+
 /* Synchronises `stream` and returns the device-side status word of `ws`
  * (SLA_OK, or SLA_ERR_TIMEOUT when a bounded wait ran out), or SLA_ERR_CUDA
  * if the synchronisation itself failed. */

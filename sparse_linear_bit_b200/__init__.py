@@ -27,7 +27,8 @@ __all__ = [
     "SlaError", "lib", "sla_version", "sla_status_string", "sla_topk_count", "sla_workspace_bytes",
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_quantize_qk_fp8", "sla_forward", "sla_check", "workspace",
     "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
-    "sla_block_mask_noalloc_limit", "head_shard", "shard_heads",
+    "sla_block_mask_noalloc_limit", "head_shard", "shard_heads", "sla_w8a8_quantize", "sla_w8a8_linear",
+    "w8a8_workspace",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -64,6 +65,11 @@ lib.sla_forward_profile.restype = _I
 lib.sla_block_mask_noalloc.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]
 lib.sla_block_mask_noalloc.restype = _I
 lib.sla_block_mask_noalloc_limit.restype = _SZ
+lib.sla_w8a8_quantize.argtypes = [_P, _I, _I, _I, _P, _F, _P, _P, _P]
+lib.sla_w8a8_quantize.restype = _I
+lib.sla_w8a8_workspace_bytes.restype = _SZ
+lib.sla_w8a8_linear.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]
+lib.sla_w8a8_linear.restype = _I
 lib.sla_check.argtypes = [_P, _P]
 lib.sla_check.restype = _I
 
@@ -204,3 +210,28 @@ def sla_forward_profile(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream
 def sla_check(ws, stream=None) -> None:
     """Synchronise the stream and raise if a kernel recorded a device-side failure."""
     _ok(lib.sla_check(_ptr(ws), _stream(stream)), "sla_check")
+
+
+# --------------------------------------------------------------------------
+# W8A8 INT8 linear layer with FusedNorm
+# --------------------------------------------------------------------------
+
+def sla_w8a8_quantize(x, q, scale, norm: bool = False, gamma=None, eps: float = 1e-6, stream=None) -> None:
+    """Per-row INT8 codes of a bf16 [rows, cols] tensor into q (int8, same shape) and scale
+    (fp32 [rows]); with ``norm`` the rows are RMS-normalised (times ``gamma``) first."""
+    rows, cols = x.shape
+    _ok(lib.sla_w8a8_quantize(_ptr(x), rows, cols, int(bool(norm)), _ptr(gamma), float(eps), _ptr(q), _ptr(scale),
+                              _stream(stream)), "sla_w8a8_quantize")
+
+
+def w8a8_workspace(device=None):
+    import torch
+    return torch.zeros(int(lib.sla_w8a8_workspace_bytes()), dtype=torch.uint8, device=device or "cuda")
+
+
+def sla_w8a8_linear(qx, sx, qw, sw, bias, out, ws, stream=None) -> None:
+    """out (bf16 [M, N]) = (qx [M, K] int8) (qw [N, K] int8)^T * sx[M] * sw[N] (+ bias[N])."""
+    M, K = qx.shape
+    N = qw.shape[0]
+    _ok(lib.sla_w8a8_linear(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), _ptr(bias), M, N, K, _ptr(out), _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "sla_w8a8_linear")

@@ -55,6 +55,11 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
                              const Geometry &g, int phi, void *out, int *status, cudaStream_t s);
 
 // TMA descriptor encoding (driver entry point fetched once through the runtime)
+// W8A8 linear layer (sla_w8a8.cu)
+cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,
+                            float *scale, cudaStream_t s);
+cudaError_t launch_w8a8_gemm(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, const float *bias,
+                             int M, int N, int K, void *out, int *status, cudaStream_t s);
 bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const uint64_t *dims,
                  const uint64_t *strides_bytes /* rank-1 entries */, const uint32_t *box);
 

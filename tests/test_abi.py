@@ -120,6 +120,18 @@ def test_block_mask_and_quant_host_validation():
     # quant = 2 (FP8) needs the same workspace as INT8
     assert sla.sla_workspace_bytes(1, 2, 2048, 128, 64, 64, 0.1, 2) == sla.sla_workspace_bytes(1, 2, 2048, 128, 64,
                                                                                               64, 0.1, 1)
+    # W8A8: shapes the kernels do not cover, null or misaligned pointers, a small workspace
+    assert L.sla_w8a8_quantize(FAKE, 4, 100, 0, None, ctypes.c_float(1e-6), FAKE, FAKE, None) == 2   # cols % 8
+    assert L.sla_w8a8_quantize(FAKE, 4, 16392, 0, None, ctypes.c_float(1e-6), FAKE, FAKE, None) == 2
+    assert L.sla_w8a8_quantize(None, 4, 128, 0, None, ctypes.c_float(1e-6), FAKE, FAKE, None) == 1
+    assert L.sla_w8a8_quantize(FAKE, 4, 128, 2, None, ctypes.c_float(1e-6), FAKE, FAKE, None) == 1     # norm
+    assert L.sla_w8a8_quantize(FAKE, 4, 128, 1, None, ctypes.c_float(-1.0), FAKE, FAKE, None) == 1    # eps
+    assert L.sla_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 8, 24, FAKE, FAKE, 256, None) == 2      # K % 16
+    assert L.sla_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 12, 32, FAKE, FAKE, 256, None) == 2     # N % 8
+    assert L.sla_w8a8_linear(FAKE, FAKE, FAKE + 8, FAKE, None, 4, 8, 32, FAKE, FAKE, 256, None) == 1  # align
+    assert L.sla_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, 4, 8, 32, FAKE, FAKE, 16, None) == 3       # ws
+    assert L.sla_w8a8_linear(FAKE, FAKE, FAKE, FAKE, None, 0, 8, 32, FAKE, FAKE, 256, None) == 1
+    assert sla.lib.sla_w8a8_workspace_bytes() == 256
     assert L.sla_check(None, None) == 1
 
 
