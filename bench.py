@@ -60,6 +60,7 @@ def parse():
     ap.add_argument("--phi", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w8a8", action="store_true", help="skip the W8A8 linear-layer measurement")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong"])
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling runs)")
     return ap.parse_args()
@@ -374,6 +375,47 @@ def main():
                                    "linear_tf32": ops_lin},
                 "launch_ms": stage_ms["attention"]}
 
+    # ---- W8A8 INT8 linear layer (+ FusedNorm) at the DiT projection shape of this workload:
+    #      the N tokens of one sample x hidden 5120 -> 5120 (the 14B model's width)
+    w8a8 = None
+    if rank == 0 and not a.no_w8a8:
+        M_, N_, K_ = w.N, 5120, 5120
+        gen = torch.Generator(device=dev).manual_seed(7)
+        xw = torch.randn(M_, K_, device=dev, generator=gen).bfloat16()
+        ww = (torch.randn(N_, K_, device=dev, generator=gen) * 0.02).bfloat16()
+        gam = torch.ones(K_, device=dev)
+        qx_ = torch.empty((M_, K_), dtype=torch.int8, device=dev)
+        sx_ = torch.empty(M_, dtype=torch.float32, device=dev)
+        qw_ = torch.empty((N_, K_), dtype=torch.int8, device=dev)
+        sw_ = torch.empty(N_, dtype=torch.float32, device=dev)
+        yw = torch.empty((M_, N_), dtype=torch.bfloat16, device=dev)
+        wsw = sla.w8a8_workspace(dev)
+        sla.sla_w8a8_quantize(ww, qw_, sw_, stream=stream)
+        layer = lambda: (sla.sla_w8a8_quantize(xw, qx_, sx_, norm=True, gamma=gam, stream=stream),
+                         sla.sla_w8a8_linear(qx_, sx_, qw_, sw_, None, yw, wsw, stream=stream))
+        for _ in range(3):
+            layer()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        tq_, tg_ = [], []
+        for _ in range(10):
+            evs[0].record(stream)
+            sla.sla_w8a8_quantize(xw, qx_, sx_, norm=True, gamma=gam, stream=stream)
+            evs[1].record(stream)
+            sla.sla_w8a8_linear(qx_, sx_, qw_, sw_, None, yw, wsw, stream=stream)
+            evs[2].record(stream)
+            torch.cuda.synchronize(dev)
+            tq_.append(evs[0].elapsed_time(evs[1]))
+            tg_.append(evs[1].elapsed_time(evs[2]))
+        sla.sla_check(wsw, stream=stream)
+        gq, gg = float(np.median(tq_)), float(np.median(tg_))
+        ops_w = 2.0 * M_ * N_ * K_
+        p_i8 = 2.0 * float(peaks["bf16_tflops"])
+        w8a8 = {"shape": {"M_tokens": M_, "N": N_, "K": K_}, "fused_norm_quantize_ms": gq,
+                "quantize_gbs": M_ * K_ * 3 / gq / 1e6, "gemm_ms": gg, "gemm_tops": ops_w / gg / 1e9,
+                "gemm_frac_of_int8_peak": ops_w / gg / 1e9 / p_i8,
+                "int8_peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal int8 ratio)"}
+        del xw, ww, qx_, qw_, yw
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, single GPU only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -392,7 +434,7 @@ def main():
                     f"{world} rank(s), one per GPU; " + ("each runs the whole workload" if a.scaling == "weak"
                                                          else "B*H heads split in contiguous ranges"))),
                 "stages_ms": stage_ms, "roofline": roofline,
-                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "w8a8_linear": w8a8,
                 "gpu_launches": KERNELS_PER_STEP[a.quant] * a.steps,
                 "dense_equiv_ops_per_step_per_gpu": ops}
         print(json.dumps(line), flush=True)

@@ -186,8 +186,8 @@ SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void 
  * all ones; ignored when norm = 0).  Use it per token for activations and per
  * output channel (row of W [N, K]) for weights.
  *   q      int8 [rows, cols];  scale  fp32 [rows]
- * Requires cols % 8 == 0 and cols <= 16384 (else SLA_ERR_UNSUPPORTED); x and q
- * 16-byte aligned.  Codes are bit-exact with the definition above (the fp64
+ * Requires cols % 8 == 0 and cols <= 16384 (else SLA_ERR_UNSUPPORTED); x, q and
+ * gamma 16-byte aligned.  Codes are bit-exact with the definition above (the fp64
  * sum of squares is exact, as for the smoothing mean). */
 SLA_API sla_status sla_w8a8_quantize(const void *x_bf16, int rows, int cols, int norm, const float *gamma,
                              float eps, int8_t *q, float *scale, void *stream);

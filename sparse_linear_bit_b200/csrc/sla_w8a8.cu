@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "sla_internal.h"
 #include "sla_ptx.cuh"
@@ -33,9 +34,11 @@ namespace {
 // per-row quantisation (+ FusedNorm)
 // ---------------------------------------------------------------------------
 constexpr int kRqThreads = 256;
-constexpr int kRqChunks = 8;  // uint4 (8 bf16) per thread: cols <= 256 * 8 * 8 = 16384
+constexpr int kRqMaxChunks = 8;  // uint4 (8 bf16) per thread: cols <= 256 * 8 * 8 = 16384
 
-template <bool NORM>
+// kRqChunks: uint4 per thread, the smallest instantiation that holds the row, so that
+// short rows keep few registers and many CTAs (rows) in flight per SM
+template <bool NORM, int kRqChunks>
 __global__ void __launch_bounds__(kRqThreads) rowquant_kernel(const uint4 *__restrict__ x, int cols,
                                                               const float *__restrict__ gamma, float eps,
                                                               uint2 *__restrict__ q, float *__restrict__ scale)
@@ -84,11 +87,14 @@ __global__ void __launch_bounds__(kRqThreads) rowquant_kernel(const uint4 *__res
     auto norm_chunk = [&](int l, float (&f)[8]) {
         expand(raw[l], f);
         if (NORM) {
-            const int c0 = 8 * (tid + kRqThreads * l);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                f[i] = __fmul_rn(f[i], r);
-                if (gamma) f[i] = __fmul_rn(f[i], __ldg(gamma + c0 + i));
+            for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], r);
+            if (gamma) {  // 8 consecutive channels: two 16-byte loads (gamma is 16-byte aligned)
+                const float4 *g4 = reinterpret_cast<const float4 *>(gamma) + 2 * (tid + kRqThreads * l);
+                const float4 ga = __ldg(g4), gb = __ldg(g4 + 1);
+                const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(f[i], gg[i]);
             }
         }
     };
@@ -329,11 +335,20 @@ __global__ void __launch_bounds__(kGmThreads, 1) w8a8_gemm_kernel(const __grid_c
 cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,
                             float *scale, cudaStream_t s)
 {
-    if (cols % 8 != 0 || cols > kRqThreads * kRqChunks * 8) return cudaErrorInvalidValue;
+    if (cols % 8 != 0 || cols > kRqThreads * kRqMaxChunks * 8) return cudaErrorInvalidValue;
     const uint4 *xi = static_cast<const uint4 *>(x);
     uint2 *qo = reinterpret_cast<uint2 *>(q);
-    if (norm) rowquant_kernel<true><<<rows, kRqThreads, 0, s>>>(xi, cols, gamma, eps, qo, scale);
-    else rowquant_kernel<false><<<rows, kRqThreads, 0, s>>>(xi, cols, nullptr, 0.0f, qo, scale);
+    const int ch = (cols / 8 + kRqThreads - 1) / kRqThreads;
+    auto go = [&](auto chunks) {
+        constexpr int C = decltype(chunks)::value;
+        if (norm) rowquant_kernel<true, C><<<rows, kRqThreads, 0, s>>>(xi, cols, gamma, eps, qo, scale);
+        else rowquant_kernel<false, C><<<rows, kRqThreads, 0, s>>>(xi, cols, nullptr, 0.0f, qo, scale);
+    };
+    if (ch <= 1) go(std::integral_constant<int, 1>{});
+    else if (ch <= 2) go(std::integral_constant<int, 2>{});
+    else if (ch <= 3) go(std::integral_constant<int, 3>{});
+    else if (ch <= 4) go(std::integral_constant<int, 4>{});
+    else go(std::integral_constant<int, 8>{});
     return cudaGetLastError();
 }
 
@@ -386,7 +401,7 @@ sla_status sla_w8a8_quantize(const void *x, int rows, int cols, int norm, const 
     if (rows < 1 || cols < 8 || (norm != 0 && norm != 1)) return SLA_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SLA_ERR_INVALID_ARG;
     if (cols % 8 != 0 || cols > 16384) return SLA_ERR_UNSUPPORTED;
-    if (!al(x, 16) || !al(q, 16) || !al(scale, 4) || (gamma && !al(gamma, 4))) return SLA_ERR_INVALID_ARG;
+    if (!al(x, 16) || !al(q, 16) || !al(scale, 4) || (gamma && !al(gamma, 16))) return SLA_ERR_INVALID_ARG;
     if (sla::launch_rowquant(x, rows, cols, norm, norm ? gamma : nullptr, eps, q, scale,
                              static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return SLA_ERR_CUDA;
