@@ -18,6 +18,9 @@ collective since every (batch, head) is independent:
                    element; the job grows with the number of GPUs.
   --scaling strong the workload's B*H heads are split into contiguous ranges, one
                    per rank (sparse_linear_bit_b200.head_shard).
+  --scaling ulysses every rank holds N/P tokens of every head (context
+                   parallelism); a step is the all-to-all to head shards, the
+                   forward on H/P heads and the all-to-all back (NCCL).
 Times are taken on the device and the max over ranks is reported.  Rank 0
 prints one JSON line.
 """
@@ -61,7 +64,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w8a8", action="store_true", help="skip the W8A8 linear-layer measurement")
-    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"])
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong", "ulysses"])
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling runs)")
     return ap.parse_args()
 
@@ -230,6 +233,47 @@ def selected_work(idx, w, k_sel):
     return float((keys * rows[None, :]).sum()) * w.d
 
 
+def run_ulysses(a, w, q, k, v, rank, world, dev, ops_job):
+    """Context-parallel step: token-sharded inputs, all-to-all, forward on H/P heads, all-to-all back."""
+    import torch
+    import torch.distributed as dist
+    from sparse_linear_bit_b200 import ulysses
+    if w.H % world or w.N % world:
+        raise SystemExit(f"--scaling ulysses needs H and N divisible by {world}")
+    n = w.N // world
+    to_dev = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, :, rank * n:(rank + 1) * n]).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    import sparse_linear_bit_b200 as sla
+    ws = sla.workspace(w.B, w.H // world, w.N, w.d, w.blk_q, w.blk_k, a.topk, a.quant, device=dev)
+    step = lambda: ulysses.sla_forward_ulysses(qd, kd, vd, w.blk_q, w.blk_k, a.topk, a.phi, a.quant, ws=ws)
+    for _ in range(max(3, a.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    sla.sla_check(ws)
+    ms = max_over_ranks(e0.elapsed_time(e1) / a.steps, dev, world)
+    if rank == 0:
+        line = {"metric": METRIC, "value": ops_job / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world,
+                "steps": a.steps, "warmup": max(3, a.warmup), "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None,
+                "dtype": {0: "bf16+fp16", 1: "i8+bf16", 2: "fp8e4m3+bf16"}[a.quant], "data": "synthetic",
+                "config": dict(workload_config(w, a), parallelism=f"{world} ranks, Ulysses context parallelism: "
+                               f"{n} tokens of every head per rank, all-to-all to {w.H // world} heads per rank"),
+                "gpu_launches": None}
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+    return 0
+
+
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
@@ -272,6 +316,8 @@ def main():
     # ---- this rank's share: the whole workload (weak) or a contiguous head range (strong)
     ops_job = dense_equiv_ops(w.B, w.H, w.N, w.d) * (world if a.scaling == "weak" else 1)
     wl = w
+    if a.scaling == "ulysses" and world > 1:
+        return run_ulysses(a, w, q, k, v, rank, world, dev, ops_job)
     if a.scaling == "strong" and world > 1:
         first, count = sla.head_shard(w.B, w.H, world, rank)
         q, k, v = (np.ascontiguousarray(sla.shard_heads(x, world, rank)) for x in (q, k, v))

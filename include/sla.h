@@ -204,6 +204,23 @@ SLA_API sla_status sla_w8a8_linear(const int8_t *qx, const float *sx, const int8
                            const float *bias, int M, int N, int K, void *out_bf16, void *ws, size_t ws_bytes,
                            void *stream);
 
+/* ---- Ulysses context parallelism (the "TurboDiffusion" GitHub summary,
+ * 主要特点: the training code supports Ulysses CP).  Each of P ranks holds
+ * n_local = N / P consecutive tokens of every head; an all-to-all regroups them
+ * into every token of H / P heads, the attention runs per head, and a second
+ * all-to-all restores the token sharding.  This call does the block
+ * permutation around each all-to-all (the exchange itself is the caller's, e.g.
+ * NCCL's all_to_all_single on the [P][B][H/P][n_local][d] buffer, slice r to /
+ * from rank r):
+ *   mode 0  [B][H][n_local][d]        -> buffer   (tokens -> heads, send side)
+ *   mode 1  buffer                    -> [B][H/P][P*n_local][d]  (receive side)
+ *   mode 2  [B][H/P][P*n_local][d]    -> buffer   (heads -> tokens, send side)
+ *   mode 3  buffer                    -> [B][H][n_local][d]      (receive side)
+ * elem_bytes: 1, 2, 4 or 8.  H % P == 0; n_local * d * elem_bytes % 16 == 0 (else
+ * SLA_ERR_UNSUPPORTED); src, dst 16-byte aligned and distinct. */
+SLA_API sla_status sla_ulysses_permute(const void *src, void *dst, int B, int H, int P, int n_local, int d,
+                               int elem_bytes, int mode, void *stream);
+
 /* Synchronises `stream` and returns the device-side status word of `ws`
  * (SLA_OK, or SLA_ERR_TIMEOUT when a bounded wait ran out), or SLA_ERR_CUDA
  * if the synchronisation itself failed. */
