@@ -146,7 +146,7 @@ SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void
  * file-scope device array of sla_block_mask_noalloc_limit() bytes (16 MiB),
  * which every GPU that loads the library holds until the process exits.
  * Problems whose scratch would exceed it return SLA_ERR_WORKSPACE before any
- * launch (about B*H*n_qb*(8*n_kb + 2*n_kb_pad) + 1 KiB*B*H*(n_qb + n_kb)
+ * launch (about B*H*n_qb*(8*n_kb + 8*ceil(n_kb/64)) + 1 KiB*B*H*(n_qb + n_kb)
  * bytes are needed).  It allocates nothing.
  *
  * The first call on a device resolves the array's device address for that

@@ -30,7 +30,7 @@ Geometry make_geometry(int B, int H, int N, int d, int blk_q, int blk_k, float t
     g.BH = B * H;
     g.n_qb = (N + blk_q - 1) / blk_q;
     g.n_kb = (N + blk_k - 1) / blk_k;
-    g.n_kb_pad = (g.n_kb + 7) / 8 * 8;
+    g.n_aw = 2 * ((g.n_kb + 63) / 64);  // whole 64-block k-steps of the state reduction
     g.k_sel = topk_count(g.n_kb, topk);
     g.subtract = 2 * g.k_sel <= g.n_kb;
     g.n_chunks = (g.n_kb + kStateChunk - 1) / kStateChunk;
@@ -51,7 +51,7 @@ Layout make_layout(const Geometry &g)
     L.kpart = take(BH * (size_t)pool_parts(g.n_kb) * kD * sizeof(double));
     L.scores = take(BH * g.n_qb * g.n_kb * sizeof(double));
     L.idx = take(BH * g.n_qb * (size_t)(g.k_sel > 0 ? g.k_sel : 1) * sizeof(int32_t));
-    L.amask = take(BH * g.n_qb * g.n_kb_pad * sizeof(uint16_t));
+    L.amask = take(BH * g.n_qb * (size_t)g.n_aw * sizeof(uint32_t));
     const size_t none = (size_t)-1;
     L.q8 = g.quant ? take(BH * N * kD) : none;
     L.k8 = g.quant ? take(BH * N * kD) : none;
@@ -213,7 +213,7 @@ sla_status sla_block_mask(const void *q, const void *k, int B, int H, int N, int
     SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, nullptr, s));
     SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
     int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
-    SLA_TRY(launch_topk(scores, g, idx, bitmap_out, reinterpret_cast<uint16_t *>(ws_at(ws, L.amask)), s));
+    SLA_TRY(launch_topk(scores, g, idx, bitmap_out, reinterpret_cast<uint32_t *>(ws_at(ws, L.amask)), s));
     return SLA_OK;
 }
 
@@ -258,7 +258,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     double *kpart = reinterpret_cast<double *>(ws_at(ws, L.kpart));
     double *scores = reinterpret_cast<double *>(ws_at(ws, L.scores));
     int32_t *idx = reinterpret_cast<int32_t *>(ws_at(ws, L.idx));
-    uint16_t *amask = reinterpret_cast<uint16_t *>(ws_at(ws, L.amask));
+    uint32_t *amask = reinterpret_cast<uint32_t *>(ws_at(ws, L.amask));
     float *kmean = reinterpret_cast<float *>(ws_at(ws, L.kmean));
     int8_t *q8 = quant ? reinterpret_cast<int8_t *>(ws_at(ws, L.q8)) : nullptr;
     int8_t *k8 = quant ? reinterpret_cast<int8_t *>(ws_at(ws, L.k8)) : nullptr;

@@ -15,7 +15,7 @@ constexpr int kStateChunk = 32;          // key blocks per partial sum of the gl
 
 struct Geometry {
     int B, H, N, d, blk_q, blk_k;
-    int BH, n_qb, n_kb, n_kb_pad, k_sel, quant;
+    int BH, n_qb, n_kb, n_aw, k_sel, quant;  // n_aw: 32-bit words of a state-reduction mask row
     bool subtract;  // H_I = H_total - sum(selected); otherwise sum(unselected)
     int n_chunks;   // partial sums of the global state per head
 };
@@ -37,7 +37,7 @@ cudaError_t launch_kmean(const double *part, int BH, int N, int n_parts, float *
 cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry &g, double *scores,
                           cudaStream_t s);
 cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap,
-                        uint16_t *amask, cudaStream_t s);
+                        uint32_t *amask, cudaStream_t s);
 // INT8 (fp8 = 0) or FP8 e4m3 (fp8 = 1) codes and scales; with `bmean` (no smoothing) also the
 // fp64 block means
 cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const float *mean, int8_t *out,
@@ -47,7 +47,7 @@ cudaError_t launch_quant(const void *x, int BH, int N, int blk, int nb, const fl
 cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int phi, uint16_t *states,
                           float *partials, uint16_t *v16, int *status, cudaStream_t s);
 cudaError_t launch_htot(const float *partials, const Geometry &g, float *htot, cudaStream_t s);
-cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, const float *htot,
+cudaError_t launch_state_reduce(const uint32_t *amask, const uint16_t *states, const float *htot,
                                 const Geometry &g, float *hq, int *status, cudaStream_t s);
 // v: bf16 V with quant = 1, the fp16 copy of V with quant = 0
 cudaError_t launch_attention(const void *q, const void *k, const void *v, const int8_t *q8, const int8_t *k8,

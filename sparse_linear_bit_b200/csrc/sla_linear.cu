@@ -14,8 +14,9 @@
 //                 is off.
 //  htot_kernel    global state per head = fixed-order sum of the chunk sums.
 //  reduce_kernel  per query block I: C_I = sum_J A[I][J] S_J as a dense GEMM
-//                 (M = 128 query blocks, N = 256 state columns, K = key
-//                 blocks) with a 0/1 mask A.  When at most half the key blocks
+//                 (M = 128 query blocks, N = 192 state columns, K = key
+//                 blocks) with a 0/1 mask A, expanded from bits into tensor
+//                 memory.  When at most half the key blocks
 //                 are selected A marks the selected blocks and the state is
 //                 H_total - C_I (only the selected ~10% go through bf16); else A
 //                 marks the unselected blocks and the state is C_I (exact zeros
@@ -330,23 +331,38 @@ __global__ void htot_kernel(const float *__restrict__ partials, int n_chunks, fl
 }
 
 // ---------------------------------------------------------------------------
-// per-query-block state: persistent GEMM over tiles (bh, 256 state columns,
-// 128 query blocks), m fastest so the 5 query-block tiles of one column tile
-// run together and share the state columns through L2.  Warp 0 = TMA producer,
-// warp 1 = MMA issuer, warps 2..5 = epilogue (TMEM lanes by warp index % 4).
-// Two TMEM accumulators: the epilogue of one tile overlaps the next tile's MMAs.
+// per-query-block state: persistent GEMM over tiles (bh, 192 state columns,
+// 128 query blocks), m fastest so the query-block tiles of one column tile run
+// together and share the state columns through L2.  The 0/1 mask never goes
+// through shared memory: top-k writes it as bits, and four builder warps expand
+// each row's 64 bits of a k-step into bf16 pairs stored straight into tensor
+// memory, where the MMA takes its A operand.  Only the states (B, MN-major)
+// stream in by TMA, 24 KB per k-step.
+//   warp 0      TMA producer (B ring, kRedBStages)
+//   warp 1      MMA issuer
+//   warps 2..5  epilogue (TMEM lane quarter = warp index % 4): 32 x 32 fp32
+//               chunks staged swizzled in shared memory and written by TMA stores
+//   warps 6..9  A builders (same lane quarters)
+// TMEM: two accumulators [0, 384) so the epilogue of one tile overlaps the
+// next tile's MMAs, and the A ring [384, 512): kRedAStages x 32 columns (one
+// k-step of 64 key blocks as 16-bit pairs).  16512 state columns = 86 x 192.
 // ---------------------------------------------------------------------------
-constexpr int kRedStages = 4;
-constexpr int kRedThreads = 192;
-constexpr uint32_t kRedA = 128 * 128;      // 128 query blocks x 64 key blocks (bf16)
-constexpr uint32_t kRedB = 4 * kTileBytes; // 64 key blocks x 256 columns (bf16), four 64-column boxes
+constexpr int kRedBStages = 6;
+constexpr int kRedAStages = 4;
+constexpr int kRedThreads = 320;
+constexpr int kRedN = 192;
+constexpr uint32_t kRedB = 3 * kTileBytes;  // 64 key blocks x 192 columns (bf16), three 64-column boxes
+constexpr uint32_t kRedACol = 2 * kRedN;    // first TMEM column of the A ring
+constexpr int kRedEpiBufs = 3;              // 4 KB output staging buffers per epilogue warp
+static_assert(kStateCols % kRedN == 0, "state columns split into whole tiles");
+static_assert(kRedACol + 32 * kRedAStages <= 512, "TMEM budget");
 
 struct ReduceSmem {
-    alignas(1024) uint8_t a[kRedStages][kRedA];
-    alignas(1024) uint8_t b[kRedStages][kRedB];
-    float ht[4][256];  // global-state columns of the tile in the epilogue, one copy per epilogue warp
-    uint64_t full[kRedStages];
-    uint64_t empty[kRedStages];
+    alignas(1024) uint8_t b[kRedBStages][kRedB];
+    alignas(1024) uint8_t out[4][kRedEpiBufs][32 * 128];  // [epilogue warp][buffer]: 32 rows x 32 fp32, SW128
+    float ht[4][kRedN];  // global-state columns of the tile in the epilogue, one copy per epilogue warp
+    uint64_t full[kRedBStages], empty[kRedBStages];
+    uint64_t a_full[kRedAStages], a_empty[kRedAStages];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -355,16 +371,40 @@ struct ReduceSmem {
 
 __device__ __forceinline__ uint64_t dadd16(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
 
-__global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_constant__ CUtensorMap tm_a,
-                                                                const __grid_constant__ CUtensorMap tm_s, int n_qb,
+// bf16 MMA with A in tensor memory (rows = lanes, two K elements per 32-bit column, the lower K
+// in the low half)
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc_,
+                                                uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc_), "r"(accumulate)
+        : "memory");
+}
+
+// the mask words of k-steps kt .. kt+3 of one row (zeros past the row's end or for a padding row)
+__device__ __forceinline__ void load_mask4(const uint32_t *row, int kt, int nk, uint32_t (&w)[8])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint2 v = make_uint2(0u, 0u);
+        if (row && kt + i < nk) v = __ldg(reinterpret_cast<const uint2 *>(row) + kt + i);
+        w[2 * i] = v.x;
+        w[2 * i + 1] = v.y;
+    }
+}
+
+__global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const uint32_t *__restrict__ amask, int n_aw,
+                                                                const __grid_constant__ CUtensorMap tm_s,
+                                                                const __grid_constant__ CUtensorMap tm_hq, int n_qb,
                                                                 int n_kb, int n_tiles, int subtract,
-                                                                const float *__restrict__ htot,
-                                                                float *__restrict__ hq, int *status)
+                                                                const float *__restrict__ htot, int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     ReduceSmem &sm = *reinterpret_cast<ReduceSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_mt = (n_qb + 127) / 128, n_nt = (kStateCols + 255) / 256;
+    const int n_mt = (n_qb + 127) / 128, n_nt = kStateCols / kRedN;
     const int nk = (n_kb + 63) / 64;
     volatile int *abort_flag = &sm.abort_flag;
     if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
@@ -372,9 +412,13 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_con
     if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
 
     if (tid == 0) {
-        for (int s = 0; s < kRedStages; ++s) {
+        for (int s = 0; s < kRedBStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
+        }
+        for (int s = 0; s < kRedAStages; ++s) {
+            mbar_init(&sm.a_full[s], 128);
+            mbar_init(&sm.a_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
@@ -382,8 +426,8 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_con
         }
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
-        tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_s);
+        tma_prefetch_desc(&tm_hq);
     }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, 512);
@@ -396,107 +440,168 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const __grid_con
     auto tile_coords = [&](int t, int &bh, int &I0, int &n0) {
         const int m = t % n_mt, rest = t / n_mt;
         bh = rest / n_nt;
-        n0 = (rest % n_nt) * 256;
+        n0 = (rest % n_nt) * kRedN;
         I0 = m * 128;
     };
 
     if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ producer (states)
         int kc = 0;  // k-steps issued over all tiles of this CTA
         bool ok = true;
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
             int bh, I0, n0;
             tile_coords(t, bh, I0, n0);
-            const int n_groups = min(256, kStateCols - n0) / 64;
             for (int kt = 0; kt < nk; ++kt, ++kc) {
-                const int s = kc % kRedStages, u = kc / kRedStages;
+                const int s = kc % kRedBStages, u = kc / kRedBStages;
                 if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
-                mbar_expect_tx(&sm.full[s], kRedA + (uint32_t)n_groups * kTileBytes);
-                tma_load_3d(sm.a[s], &tm_a, &sm.full[s], kt * 64, I0, bh);
-                for (int g = 0; g < n_groups; ++g)
+                mbar_expect_tx(&sm.full[s], kRedB);
+#pragma unroll
+                for (int g = 0; g < 3; ++g)
                     tma_load_3d(sm.b[s] + g * kTileBytes, &tm_s, &sm.full[s], n0 + 64 * g, kt * 64, bh);
             }
         }
         if (!ok) {  // let in-flight loads land before the CTA exits
-            for (int s = 0; s < kRedStages; ++s) {
+            for (int s = 0; s < kRedBStages; ++s) {
                 int jl = -1;
-                for (int j = s; j < kc; j += kRedStages) jl = j;
-                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedStages) & 1);
+                for (int j = s; j < kc; j += kRedBStages) jl = j;
+                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedBStages) & 1);
             }
         }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        const uint64_t ad0 = sdesc_sw128(smem_u32(sm.a[0]), 16, 1024);
         const uint64_t bd0 = sdesc_sw128(smem_u32(sm.b[0]), kTileBytes, 1024);
+        const uint32_t id = idesc(1, 1, 1, 0, 1, 128, kRedN);  // A from TMEM, B MN-major
         int kc = 0, lt = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
-            int bh, I0, n0;
-            tile_coords(t, bh, I0, n0);
-            const uint32_t id = idesc(1, 1, 1, 0, 1, 128, (uint32_t)min(256, kStateCols - n0));  // A K-, B MN-major
             const int buf = lt & 1;
-            const uint32_t acc = tmem + 256 * buf;
+            const uint32_t acc = tmem + kRedN * buf;
             if (lt >= 2 && !(ok = mbar_wait(&sm.acc_empty[buf], ((lt >> 1) - 1) & 1, status, abort_flag))) break;
             tc_fence_after();
             for (int kt = 0; kt < nk; ++kt, ++kc) {
-                const int s = kc % kRedStages, u = kc / kRedStages;
-                if (!(ok = mbar_wait(&sm.full[s], u & 1, status, abort_flag))) break;
+                const int sb = kc % kRedBStages, sa = kc % kRedAStages;
+                const uint32_t pa = (kc / kRedAStages) & 1, pb = (kc / kRedBStages) & 1;
+                const bool ra = mbar_test(&sm.a_full[sa], pa);  // both tests in flight together
+                const bool rb = mbar_test(&sm.full[sb], pb);
+                if (!ra && !(ok = mbar_wait(&sm.a_full[sa], pa, status, abort_flag))) break;
+                if (!rb && !(ok = mbar_wait(&sm.full[sb], pb, status, abort_flag))) break;
                 tc_fence_after();
+                const uint32_t a_t = tmem + kRedACol + 32 * sa;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(acc, dadd16(ad0, s * kRedA + 32 * k), dadd16(bd0, s * kRedB + 2048 * k), id,
-                             (kt > 0 || k > 0) ? 1u : 0u);
-                mma_commit(&sm.empty[s]);
+                    mma_bf16_tmem_a(acc, a_t + 8 * k, dadd16(bd0, sb * kRedB + 2048 * k), id,
+                                    (kt > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.empty[sb]);
+                mma_commit(&sm.a_empty[sa]);
             }
             if (!ok) break;
             mma_commit(&sm.acc_full[buf]);
         }
         mma_commit(&sm.drain);
         mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ A builders
+        // Thread = one query block (TMEM lane); column c of a k-step holds the mask of key
+        // blocks 64 kt + 2c (low half) and 64 kt + 2c + 1 (high half): bf16 1.0 or 0.
+        const int q = warp & 3;
+        const uint32_t a_lane = (uint32_t)(q * 32) << 16;
+        auto row_of = [&](int t) -> const uint32_t * {
+            if (t >= n_tiles) return nullptr;
+            int bh, I0, n0;
+            tile_coords(t, bh, I0, n0);
+            const int I = I0 + q * 32 + lane;
+            return I < n_qb ? amask + ((size_t)bh * n_qb + I) * n_aw : nullptr;
+        };
+        int kc = 0;
+        bool ok = true;
+        uint32_t w[8];
+        load_mask4(row_of(blockIdx.x), 0, nk, w);
+        for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+            const uint32_t *row = row_of(t), *next_row = row_of(t + gridDim.x);
+            for (int kt0 = 0; ok && kt0 < nk; kt0 += 4) {
+                uint32_t nx[8];  // one group ahead, into the next tile at the end of this one
+                if (kt0 + 4 < nk)
+                    load_mask4(row, kt0 + 4, nk, nx);
+                else
+                    load_mask4(next_row, 0, nk, nx);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (kt0 + j < nk) {  // warp-uniform
+                        const int sa = kc % kRedAStages, u = kc / kRedAStages;
+                        if (u > 0 && !(ok = mbar_wait_warp(&sm.a_empty[sa], (u - 1) & 1, status, abort_flag)))
+                            break;
+                        tc_fence_after();
+                        uint32_t r[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) {
+                            const uint32_t b = (w[2 * j + (c >> 4)] >> (2 * (c & 15))) & 3u;
+                            r[c] = (b & 1u) * 0x3F80u + (b >> 1) * 0x3F800000u;
+                        }
+                        tmem_st32(tmem + a_lane + kRedACol + 32 * sa, r);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&sm.a_full[sa]);
+                        ++kc;
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = nx[i];
+            }
+        }
     } else if (warp >= 2) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        int lt = 0;
+        int lt = 0, ec = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++lt) {
             int bh, I0, n0;
             tile_coords(t, bh, I0, n0);
-            const int n_valid = min(256, kStateCols - n0);
             const int buf = lt & 1;
             // global-state columns of this tile (subtract mode), staged per warp so that only
             // warp-local synchronisation is needed
             float *ht = sm.ht[q];
             if (subtract) {
                 __syncwarp();
-                for (int c = lane; c < n_valid; c += 32) ht[c] = __ldg(htot + (size_t)bh * kStateCols + n0 + c);
+                for (int c = lane; c < kRedN; c += 32) ht[c] = __ldg(htot + (size_t)bh * kStateCols + n0 + c);
                 __syncwarp();
             }
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[buf], (lt >> 1) & 1, status, abort_flag))))
-                break;
+            if (!(ok = mbar_wait_warp(&sm.acc_full[buf], (lt >> 1) & 1, status, abort_flag))) break;
             tc_fence_after();
-            const int I = I0 + q * 32 + lane;
-            float *dst = hq + ((size_t)bh * n_qb + I) * kStateCols + n0;
-            const uint32_t acc = tmem + 256 * buf + ((uint32_t)(q * 32) << 16);
-            for (int c0 = 0; c0 < n_valid; c0 += 32) {
+            const uint32_t acc = tmem + kRedN * buf + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < kRedN; c0 += 32, ++ec) {
                 uint32_t r[32];
                 tmem_ld32(acc + c0, r);
                 tmem_wait_ld();
-                if (I < n_qb) {
-                    float v[32];
+                if (c0 + 32 == kRedN) {  // the accumulator is read: the next tile may start on it
+                    tc_fence_before();
+                    mbar_arrive(&sm.acc_empty[buf]);
+                }
+                uint8_t *stage = sm.out[q][ec % kRedEpiBufs];
+                if (lane == 0) bulk_wait_read<kRedEpiBufs - 1>();  // the store that used this buffer has read it
+                __syncwarp();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float x = __uint_as_float(r[i]);
-                        if (subtract) x = ht[c0 + i] - x;
-                        v[i] = (n0 + c0 + i < kD * kD) ? to_tf32(x) : x;
+                for (int u = 0; u < 8; ++u) {
+                    float v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = c0 + 4 * u + i;
+                        float x = __uint_as_float(r[4 * u + i]);
+                        if (subtract) x = ht[c] - x;
+                        v[i] = (n0 + c < kD * kD) ? to_tf32(x) : x;
                     }
-                    float4 *o = reinterpret_cast<float4 *>(dst + c0);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                    *reinterpret_cast<float4 *>(stage + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+                        make_float4(v[0], v[1], v[2], v[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {  // rows past n_qb fall outside the tensor map and are not written
+                    tma_store_3d(&tm_hq, stage, n0 + c0, I0 + 32 * q, bh);
+                    bulk_commit();
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&sm.acc_empty[buf]);
         }
+        if (lane == 0) bulk_wait<0>();  // stores complete before the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -545,15 +650,16 @@ cudaError_t launch_htot(const float *partials, const Geometry &g, float *htot, c
     return cudaGetLastError();
 }
 
-cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, const float *htot, const Geometry &g,
+cudaError_t launch_state_reduce(const uint32_t *amask, const uint16_t *states, const float *htot, const Geometry &g,
                                 float *hq, int *status, cudaStream_t s)
 {
-    CUtensorMap ta, ts;
+    if (g.n_aw != 2 * ((g.n_kb + 63) / 64)) return cudaErrorInvalidValue;
+    CUtensorMap ts, th;
     {
-        const uint64_t dims[3] = {(uint64_t)g.n_kb_pad, (uint64_t)g.n_qb, (uint64_t)g.BH};
-        const uint64_t strides[2] = {(uint64_t)g.n_kb_pad * 2, (uint64_t)g.n_qb * g.n_kb_pad * 2};
-        const uint32_t box[3] = {64, 128, 1};
-        if (!encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, amask, dims, strides, box))
+        const uint64_t dims[3] = {(uint64_t)kStateCols, (uint64_t)g.n_qb, (uint64_t)g.BH};
+        const uint64_t strides[2] = {(uint64_t)kStateCols * 4, (uint64_t)g.n_qb * kStateCols * 4};
+        const uint32_t box[3] = {32, 32, 1};
+        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, dims, strides, box))
             return cudaErrorInvalidValue;
     }
     {
@@ -569,9 +675,9 @@ cudaError_t launch_state_reduce(const uint16_t *amask, const uint16_t *states, c
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int n_tiles = g.BH * ((g.n_qb + 127) / 128) * ((kStateCols + 255) / 256);
-    reduce_kernel<<<n_tiles < sms ? n_tiles : sms, kRedThreads, smem, s>>>(ta, ts, g.n_qb, g.n_kb, n_tiles,
-                                                                         g.subtract ? 1 : 0, htot, hq, status);
+    const int n_tiles = g.BH * ((g.n_qb + 127) / 128) * (kStateCols / kRedN);
+    reduce_kernel<<<n_tiles < sms ? n_tiles : sms, kRedThreads, smem, s>>>(amask, g.n_aw, ts, th, g.n_qb, g.n_kb,
+                                                                         n_tiles, g.subtract ? 1 : 0, htot, status);
     return cudaGetLastError();
 }
 

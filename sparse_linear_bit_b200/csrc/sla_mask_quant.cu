@@ -214,17 +214,19 @@ __device__ int block_exclusive_scan(int v, int *total, int *warp_tmp)
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double *__restrict__ scores, int n_qb, int n_kb,
-                                                            int n_kb_pad, int k_sel, int subtract,
+                                                            int n_aw, int k_sel, int subtract,
                                                             int32_t *__restrict__ idx, uint32_t *__restrict__ bitmap,
-                                                            uint16_t *__restrict__ amask)
+                                                            uint32_t *__restrict__ amask)
 {
-    extern __shared__ uint64_t keys[];  // [n_kb]
+    extern __shared__ uint64_t keys[];  // [n_kb], then the selection bits [n_aw] (32-bit words)
     __shared__ int hist[256];
     __shared__ int warp_tmp[kTopkThreads / 32];
     __shared__ int s_bin, s_remaining;
     const int row = blockIdx.x;  // bh * n_qb + I
     const double *sr = scores + (size_t)row * n_kb;
+    uint32_t *sel_bits = reinterpret_cast<uint32_t *>(keys + n_kb);
     for (int J = threadIdx.x; J < n_kb; J += kTopkThreads) keys[J] = order_key(sr[J]);
+    for (int w = threadIdx.x; w < n_aw; w += kTopkThreads) sel_bits[w] = 0u;
 
     // radix select for the k_sel-th largest key
     uint64_t prefix = 0, mask = 0;
@@ -275,12 +277,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double *__rest
         n_sel += s;
     }
     const int sel_before = block_exclusive_scan(n_sel, &tot, warp_tmp);
-    // write the ascending index list, the bitmap and the state-reduction mask row
+    // write the ascending index list; gather the selection bits in shared memory
     int32_t *ir = idx + (size_t)row * k_sel;
-    const int words = (n_kb + 31) / 32;
-    uint32_t *br = bitmap ? bitmap + (size_t)row * words : nullptr;
-    uint16_t *ar = amask + (size_t)row * n_kb_pad;
-    const uint16_t one = 0x3F80u;  // bf16 1.0
     int o = sel_before;
     e = eq_before;
     uint32_t word = 0;
@@ -289,18 +287,26 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const double *__rest
         int s = base_sel(J);
         if (!s && k_sel > 0 && k_sel < n_kb && keys[J] == T) s = (e++ < remaining);
         if (s) ir[o++] = J;
-        ar[J] = (s ^ (subtract ? 0 : 1)) ? one : (uint16_t)0;
-        if (br) {
-            if ((J >> 5) != cur_w) {
-                if (word) atomicOr(&br[cur_w], word);
-                word = 0;
-                cur_w = J >> 5;
-            }
-            if (s) word |= 1u << (J & 31);
+        if ((J >> 5) != cur_w) {
+            if (word) atomicOr(&sel_bits[cur_w], word);
+            word = 0;
+            cur_w = J >> 5;
         }
+        if (s) word |= 1u << (J & 31);
     }
-    if (br && word) atomicOr(&br[cur_w], word);
-    for (int J = n_kb + threadIdx.x; J < n_kb_pad; J += kTopkThreads) ar[J] = 0;
+    if (word) atomicOr(&sel_bits[cur_w], word);
+    __syncthreads();
+    // the bitmap (selected) and the state-reduction mask row (selected, or its valid complement)
+    const int words = (n_kb + 31) / 32;
+    uint32_t *br = bitmap ? bitmap + (size_t)row * words : nullptr;
+    uint32_t *ar = amask + (size_t)row * n_aw;
+    for (int w = threadIdx.x; w < n_aw; w += kTopkThreads) {
+        const uint32_t sb = sel_bits[w];
+        const int valid_bits = min(32, max(0, n_kb - 32 * w));
+        const uint32_t valid = valid_bits == 32 ? 0xFFFFFFFFu : (1u << valid_bits) - 1u;
+        ar[w] = subtract ? sb : (~sb & valid);
+        if (br && w < words) br[w] = sb;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -316,10 +322,10 @@ constexpr int kTopkWarps = 4;
 
 template <int KPL>  // keys per lane: n_kb <= 32 * KPL
 __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double *__restrict__ scores, int n_rows,
-                                                                    int n_kb, int n_kb_pad, int k_sel, int subtract,
+                                                                    int n_kb, int n_aw, int k_sel, int subtract,
                                                                     int32_t *__restrict__ idx,
                                                                     uint32_t *__restrict__ bitmap,
-                                                                    uint16_t *__restrict__ amask)
+                                                                    uint32_t *__restrict__ amask)
 {
     __shared__ int hist_all[kTopkWarps][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -385,9 +391,8 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double
         }
     }
     int32_t *ir = idx + (size_t)row * k_sel;
-    uint16_t *ar = amask + (size_t)row * n_kb_pad;
+    uint32_t *ar = amask + (size_t)row * n_aw;
     uint32_t *br = bitmap ? bitmap + (size_t)row * ((n_kb + 31) / 32) : nullptr;
-    const uint16_t one = 0x3F80u;  // bf16 1.0
     int o = 0, eq_seen = 0;
 #pragma unroll
     for (int m = 0; m < KPL; ++m) {
@@ -405,19 +410,15 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double
             eq_seen += __popc(eqb);
         }
         const unsigned sb = __ballot_sync(0xffffffffu, s);
+        const unsigned ab = __ballot_sync(0xffffffffu, valid && (s != (subtract == 0)));
         if (s) ir[o + __popc(sb & lt_mask)] = J;
         o += __popc(sb);
-        if (valid) ar[J] = (s != (subtract == 0)) ? one : (uint16_t)0;
-        if (br && lane == 0) br[m] = sb;
+        if (lane == 0) {
+            ar[m] = ab;
+            if (br) br[m] = sb;
+        }
     }
-    for (int J = n_kb + lane; J < n_kb_pad; J += 32) ar[J] = 0;
-}
-
-// zero the bitmap rows before the atomicOr pass
-__global__ void zero_u32_kernel(uint32_t *p, size_t n)
-{
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-        p[i] = 0;
+    for (int w = (n_kb + 31) / 32 + lane; w < n_aw; w += 32) ar[w] = 0u;  // the last k-step's padding
 }
 
 // ---------------------------------------------------------------------------
@@ -598,7 +599,7 @@ cudaError_t launch_scores(const double *qbar, const double *kbar, const Geometry
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap, uint16_t *amask,
+cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, uint32_t *bitmap, uint32_t *amask,
                         cudaStream_t s)
 {
     const int rows = g.BH * g.n_qb;
@@ -606,25 +607,21 @@ cudaError_t launch_topk(const double *scores, const Geometry &g, int32_t *idx, u
     const int sub = g.subtract ? 1 : 0;
     // one warp per row while the row's keys fit in registers
     if (g.n_kb <= 32 * 8) {
-        topk_warp_kernel<8><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx,
+        topk_warp_kernel<8><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_aw, g.k_sel, sub, idx,
                                                                bitmap, amask);
         return cudaGetLastError();
     }
     if (g.n_kb <= 32 * 40) {
-        topk_warp_kernel<40><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx,
+        topk_warp_kernel<40><<<blocks, 32 * kTopkWarps, 0, s>>>(scores, rows, g.n_kb, g.n_aw, g.k_sel, sub, idx,
                                                                 bitmap, amask);
         return cudaGetLastError();
     }
-    if (bitmap) {
-        const size_t n = (size_t)g.BH * g.n_qb * ((g.n_kb + 31) / 32);
-        zero_u32_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, s>>>(bitmap, n);
-    }
-    const size_t smem = sizeof(uint64_t) * (size_t)g.n_kb;
+    const size_t smem = sizeof(uint64_t) * (size_t)g.n_kb + sizeof(uint32_t) * (size_t)g.n_aw;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    topk_kernel<<<rows, kTopkThreads, smem, s>>>(scores, g.n_qb, g.n_kb, g.n_kb_pad, g.k_sel, sub, idx, bitmap, amask);
+    topk_kernel<<<rows, kTopkThreads, smem, s>>>(scores, g.n_qb, g.n_kb, g.n_aw, g.k_sel, sub, idx, bitmap, amask);
     return cudaGetLastError();
 }
 

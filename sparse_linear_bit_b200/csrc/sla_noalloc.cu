@@ -60,7 +60,7 @@ sla_status sla_block_mask_noalloc(const void *q, const void *k, int B, int H, in
     // the scratch the mask path uses is the prefix of the forward's workspace layout, up to the mask rows
     const sla::Geometry g = sla::make_geometry(B, H, N, d, blk_q, blk_k, topk, 0);
     const sla::Layout L = sla::make_layout(g);
-    const size_t need = L.amask + (size_t)g.BH * g.n_qb * g.n_kb_pad * sizeof(uint16_t);
+    const size_t need = L.amask + (size_t)g.BH * g.n_qb * g.n_aw * sizeof(uint32_t);
     if (need > kStaticScratchBytes) return SLA_ERR_WORKSPACE;  // problem too large for the static scratch
     auto misaligned = [](const void *p, uintptr_t a) { return p == nullptr || ((uintptr_t)p & (a - 1)) != 0; };
     if (misaligned(q, 16) || misaligned(k, 16)) return SLA_ERR_INVALID_ARG;
@@ -74,7 +74,7 @@ sla_status sla_block_mask_noalloc(const void *q, const void *k, int B, int H, in
     double *kbar = reinterpret_cast<double *>(scratch + L.kbar);
     double *scores = reinterpret_cast<double *>(scratch + L.scores);
     int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(scratch + L.idx);
-    uint16_t *amask = reinterpret_cast<uint16_t *>(scratch + L.amask);
+    uint32_t *amask = reinterpret_cast<uint32_t *>(scratch + L.amask);
     if (sla::launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla::launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla::launch_scores(qbar, kbar, g, scores, s) != cudaSuccess) return SLA_ERR_CUDA;

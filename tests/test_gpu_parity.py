@@ -54,6 +54,7 @@ MASK_CASES = {
     "outliers_topk0": ((2, 2, (16, 16, 16)), 128, 64, 0.0, ("outliers",)),
     "topk1": ((1, 2, (8, 16, 16)), 128, 64, 1.0, ()),
     "topk_half": ((1, 2, (8, 16, 16)), 128, 64, 0.5, ()),
+    "block_topk_1313": ((1, 1, (21, 40, 100)), 128, 64, 0.1, ()),
 }
 
 
@@ -217,11 +218,21 @@ def test_forward_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_linear_states_match_oracle():
+LINEAR_CASES = {
+    # name: (grid, topk): subtract mode (H_total - selected), complement mode, several
+    # query-block tiles and key-block steps with ragged tails
+    "ragged_subtract": ((3, 10, 7), 0.3),
+    "ragged_complement": ((3, 10, 7), 0.7),
+    "multi_tile_subtract": ((16, 32, 36), 0.1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(LINEAR_CASES))
+def test_linear_states_match_oracle(name):
     """Intermediate check: per-key-block states and per-query-block states."""
-    q, k, v = synth.make_qkv(1, 1, (3, 10, 7), seed=11)
+    grid, topk = LINEAR_CASES[name]
+    q, k, v = synth.make_qkv(1, 1, grid, seed=11 + len(name))
     N = q.shape[2]
-    topk = 0.3
     out, ws = run_forward(q, k, v, 128, 64, topk, 0, 1)
     lay = sla.sla_workspace_layout(1, 1, N, 128, 128, 64, topk, 1)
     n_kb, n_qb = -(-N // 64), -(-N // 128)
@@ -233,13 +244,45 @@ def test_linear_states_match_oracle():
     assert rel_l2(st[:, :16384], hT) < 5e-3
     assert rel_l2(st[:, 16384:], z) < 5e-3
     hq = wsn[lay["hq"]:lay["hq"] + n_qb * 16512 * 4].view(np.float32).reshape(n_qb, 16512).astype(np.float64)
-    idx, _ = oracle.block_mask(q, k, 128, 64, f32(topk))
+    _, bm = oracle.block_mask(q, k, 128, 64, f32(topk))
+    sel = np.unpackbits(bm[0].view(np.uint8), axis=-1, bitorder="little")[:, :n_kb].astype(np.float64)
+    HI = (1.0 - sel) @ hT  # unselected key blocks of each query block
+    ZI = (1.0 - sel) @ z
     for I in range(n_qb):
-        un = [J for J in range(n_kb) if J not in set(idx[0, I].tolist())]
-        HI = hT[un].sum(axis=0)
-        ZI = z[un].sum(axis=0)
-        assert rel_l2(hq[I, :16384], HI) < 5e-3, I
-        assert rel_l2(hq[I, 16384:], ZI) < 5e-3, I
+        assert rel_l2(hq[I, :16384], HI[I]) < 5e-3, I
+        assert rel_l2(hq[I, 16384:], ZI[I]) < 5e-3, I
+
+
+REDUCE_MASK_CASES = {
+    # name: ((B, H, grid), blk_q, topk); n_kb = 1313 takes the block-wide top-k kernel
+    "ragged_subtract": ((1, 2, (3, 10, 7)), 128, 0.3),
+    "ragged_complement": ((1, 2, (3, 10, 7)), 64, 0.7),
+    "multi_step": ((1, 1, (16, 32, 36)), 128, 0.1),
+    "block_topk_1313": ((1, 1, (21, 40, 100)), 128, 0.1),
+    "block_topk_1313_complement": ((1, 1, (21, 40, 100)), 128, 0.6),
+}
+
+
+@pytest.mark.parametrize("name", sorted(REDUCE_MASK_CASES))
+def test_state_reduction_mask_bits(name):
+    """The state-reduction mask rows in the workspace, bit-exact: bit J of row I is set for the
+    selected key blocks when at most half of them are selected, else for the unselected ones;
+    the bits past n_kb (to a whole 64-block step) are zero."""
+    (B, H, grid), blk_q, topk = REDUCE_MASK_CASES[name]
+    q, k, v = synth.make_qkv(B, H, grid, seed=300 + len(name))
+    N = q.shape[2]
+    n_qb, n_kb = -(-N // blk_q), -(-N // 64)
+    n_aw = 2 * (-(-n_kb // 64))
+    _, ws = run_forward(q, k, v, blk_q, 64, topk, 0, 1)
+    lay = sla.sla_workspace_layout(B, H, N, 128, blk_q, 64, topk, 1)
+    raw = ws[lay["amask"]:lay["amask"] + B * H * n_qb * n_aw * 4].cpu().numpy()
+    bits = np.unpackbits(raw, bitorder="little").reshape(B * H, n_qb, 32 * n_aw)
+    _, bm = oracle.block_mask(q, k, blk_q, 64, f32(topk))
+    sel = np.unpackbits(np.ascontiguousarray(bm).view(np.uint8), axis=-1, bitorder="little")[..., :n_kb]
+    ks = oracle.topk_count(n_kb, f32(topk))
+    expect = sel if 2 * ks <= n_kb else 1 - sel
+    assert np.array_equal(bits[..., :n_kb], expect)
+    assert not bits[..., n_kb:].any()
 
 
 @pytest.mark.parametrize("topk", [0.1])
