@@ -20,6 +20,10 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   library routine; topk=0 equals closed-form linear attention; an independent
   attention-form brute force with a dense token mask; constant-V identity;
   convex-hull bounds; a hand-worked golden case).
+* ``backward``  -- pinned (float64 autograd of an independent PyTorch
+  statement of the unquantised forward, whose values are checked against
+  ``forward``; topk=1 against the gradient of a library attention routine;
+  central differences of ``forward`` along random directions).
 * Which block-score criterion, combine rule and quantisation granularity the
   pages' own SageSLA uses cannot be pinned from the pages: parity unpinned for
   that question; this oracle implements the stated reading.
@@ -72,6 +76,8 @@ def load(path: Optional[str] = None):
     lib.orc_states.argtypes = [P, P, i32, i32, i32, i32, P, P]
     lib.orc_forward.argtypes = [P, P, P, i32, i32, i32, i32, i32, f64, i32, i32, P, P, i64, P, P, P]
     lib.orc_forward.restype = i32
+    lib.orc_backward.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, P, P, P, P]
+    lib.orc_backward.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -211,6 +217,26 @@ def forward(q, k, v, blk_q: int, blk_k: int, topk: float, phi: int = 0, quant: i
     if rc != 0:
         raise MemoryError("oracle forward failed (out of memory or bad row index)")
     return (out, os_, ol_) if branches else out
+
+
+def backward(q, k, v, dout, blk_q: int, blk_k: int, topk: float, phi: int = 0,
+             idx: Optional[np.ndarray] = None, lib=None):
+    """fp64 gradients (dq, dk, dv) of the unquantised SLA forward for the output
+    gradient ``dout`` (bf16 bits, same shape as q), with the block selection held
+    fixed (the oracle's own, or ``idx``).  Results have the input's shape."""
+    lib = lib or load()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    BH, N, d = _shape(q)
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(q.shape, dtype=np.float64)
+    dv = np.zeros(q.shape, dtype=np.float64)
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    rc = lib.orc_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), BH, N, d, blk_q, blk_k, float(topk), int(phi),
+                          _ptr(idx), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise MemoryError("oracle backward failed (out of memory)")
+    return dq, dk, dv
 
 
 # --------------------------------------------------------------------------

@@ -512,6 +512,201 @@ int orc_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int BH,
 }
 
 /* ------------------------------------------------------------------------
+ * Backward: gradients of the unquantised forward (steps 1-3, 5-7 with
+ * quant = 0) with respect to q, k and v, for SLA fine-tuning
+ * ("清华开源TurboDiffusion加速框架", 方法论: full attention is replaced by SLA
+ * and the pretrained model is fine-tuned for the sparsity; the "TurboDiffusion"
+ * summary page, 主要特点: SLA white-box training).  The block selection is a
+ * piecewise-constant function of (q, k), so it is held fixed; everything else
+ * is differentiated exactly (chain rule, fp64).  With do = dL/dO:
+ *
+ *  sparse branch, row i, selected tokens j, s_ij = q_i.k_j / sqrt(d),
+ *  p_ij = softmax_j(s_ij), os_i = sum_j p_ij v_j:
+ *    dv_j += p_ij do_i;  dp_ij = do_i.v_j;  D_i = do_i.os_i;
+ *    ds_ij = p_ij (dp_ij - D_i);
+ *    dq_i += ds_ij k_j / sqrt(d);  dk_j += ds_ij q_i / sqrt(d).
+ *  linear branch, row i of query block I, f = phi(q_i), a = f H_I, b = f.Z_I,
+ *  ol_i = a / b (a zero b gives a zero output and no gradient):
+ *    da = do_i / b;  db = -(do_i.ol_i) / b;
+ *    dq_i += (H_I da + Z_I db) * phi'(q_i);
+ *    dH_I += f (outer) da;  dZ_I += f db.
+ *  key side, per key block J: G_J = sum of dH_I and g_J = sum of dZ_I over the
+ *  query blocks I that did not select J; for each token j of J:
+ *    dk_j += (G_J v_j + g_J) * phi'(k_j);  dv_j += G_J^T phi(k_j).
+ * phi'(x) = 1 for x > 0, else exp(x) (elu+1) or 0 (ReLU).
+ * ------------------------------------------------------------------------ */
+static double dphi_f(double x, int phi)
+{
+    if (phi == 1) return x > 0.0 ? 1.0 : 0.0;
+    return x > 0.0 ? 1.0 : exp(x);
+}
+
+static int backward_head(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int N,
+                         int d, int blk_q, int blk_k, int k_sel, const int32_t *idx, int phi, double *dq,
+                         double *dk, double *dv)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    const double rsd = 1.0 / sqrt((double)d); /* softmax scale 1/sqrt(d) */
+    size_t dd = (size_t)d * d;
+    double *h = (double *)malloc(sizeof(double) * (size_t)n_kb * dd);
+    double *z = (double *)malloc(sizeof(double) * (size_t)n_kb * d);
+    double *dH = (double *)calloc((size_t)n_qb * dd, sizeof(double));
+    double *dZ = (double *)calloc((size_t)n_qb * d, sizeof(double));
+    double *HI = (double *)malloc(sizeof(double) * dd);
+    double *ZI = (double *)malloc(sizeof(double) * (size_t)d);
+    double *G = (double *)malloc(sizeof(double) * dd);
+    double *gz = (double *)malloc(sizeof(double) * (size_t)d);
+    double *p = (double *)malloc(sizeof(double) * ((size_t)k_sel * blk_k + 1));
+    double *vec = (double *)malloc(sizeof(double) * 8 * (size_t)d);
+    unsigned char *selected = (unsigned char *)calloc((size_t)n_qb * n_kb + 1, 1);
+    if (!h || !z || !dH || !dZ || !HI || !ZI || !G || !gz || !p || !vec || !selected) {
+        free(h); free(z); free(dH); free(dZ); free(HI); free(ZI); free(G); free(gz); free(p); free(vec);
+        free(selected);
+        return -1;
+    }
+    double *qi = vec, *doi = vec + d, *os = vec + 2 * d, *f = vec + 3 * d, *a = vec + 4 * d, *ol = vec + 5 * d,
+           *da = vec + 6 * d, *w = vec + 7 * d;
+    states_head(k, v, N, d, blk_k, phi, h, z);
+    for (int I = 0; I < n_qb; ++I)
+        for (int r = 0; r < k_sel; ++r) selected[(size_t)I * n_kb + idx[(size_t)I * k_sel + r]] = 1;
+    memset(dq, 0, sizeof(double) * (size_t)N * d);
+    memset(dk, 0, sizeof(double) * (size_t)N * d);
+    memset(dv, 0, sizeof(double) * (size_t)N * d);
+
+    for (int I = 0; I < n_qb; ++I) {
+        const int32_t *sel = idx + (size_t)I * k_sel;
+        unselected_state(sel, k_sel, n_kb, d, h, z, HI, ZI);
+        double *dHI = dH + (size_t)I * dd, *dZI = dZ + (size_t)I * d;
+        int i1 = (I + 1) * blk_q < N ? (I + 1) * blk_q : N;
+        for (int i = I * blk_q; i < i1; ++i) {
+            for (int c = 0; c < d; ++c) {
+                qi[c] = bf(q[(size_t)i * d + c]);
+                doi[c] = bf(dout[(size_t)i * d + c]);
+            }
+            /* ---- sparse branch: recompute p and os, then the softmax gradient ---- */
+            int nk = 0;
+            double mx = -INFINITY;
+            for (int r = 0; r < k_sel; ++r) {
+                int J = sel[r], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                for (int j = t0; j < t1; ++j) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += qi[c] * bf(k[(size_t)j * d + c]);
+                    p[nk] = s * rsd;
+                    if (p[nk] > mx) mx = p[nk];
+                    ++nk;
+                }
+            }
+            if (nk > 0) {
+                double den = 0.0;
+                for (int n = 0; n < nk; ++n) {
+                    p[n] = exp(p[n] - mx);
+                    den += p[n];
+                }
+                for (int n = 0; n < nk; ++n) p[n] /= den;
+                for (int e = 0; e < d; ++e) os[e] = 0.0;
+                int n = 0;
+                for (int r = 0; r < k_sel; ++r) {
+                    int J = sel[r], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                    for (int j = t0; j < t1; ++j, ++n)
+                        for (int e = 0; e < d; ++e) os[e] += p[n] * bf(v[(size_t)j * d + e]);
+                }
+                double D = 0.0;
+                for (int e = 0; e < d; ++e) D += doi[e] * os[e];
+                n = 0;
+                for (int r = 0; r < k_sel; ++r) {
+                    int J = sel[r], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                    for (int j = t0; j < t1; ++j, ++n) {
+                        double dp = 0.0;
+                        for (int e = 0; e < d; ++e) dp += doi[e] * bf(v[(size_t)j * d + e]);
+                        double ds = p[n] * (dp - D);
+                        for (int c = 0; c < d; ++c) {
+                            dq[(size_t)i * d + c] += ds * bf(k[(size_t)j * d + c]) * rsd;
+                            dk[(size_t)j * d + c] += ds * qi[c] * rsd;
+                            dv[(size_t)j * d + c] += p[n] * doi[c];
+                        }
+                    }
+                }
+            }
+            /* ---- linear branch ---- */
+            double b = 0.0;
+            for (int c = 0; c < d; ++c) {
+                f[c] = phi_f(qi[c], phi);
+                b += f[c] * ZI[c];
+            }
+            if (b == 0.0) continue;
+            for (int e = 0; e < d; ++e) {
+                a[e] = 0.0;
+                for (int c = 0; c < d; ++c) a[e] += f[c] * HI[(size_t)c * d + e];
+                ol[e] = a[e] / b;
+            }
+            double dol = 0.0;
+            for (int e = 0; e < d; ++e) dol += doi[e] * ol[e];
+            double db = -dol / b;
+            for (int e = 0; e < d; ++e) da[e] = doi[e] / b;
+            for (int c = 0; c < d; ++c) {
+                double df = ZI[c] * db;
+                for (int e = 0; e < d; ++e) df += HI[(size_t)c * d + e] * da[e];
+                dq[(size_t)i * d + c] += df * dphi_f(qi[c], phi);
+                for (int e = 0; e < d; ++e) dHI[(size_t)c * d + e] += f[c] * da[e];
+                dZI[c] += f[c] * db;
+            }
+        }
+    }
+    /* ---- key side of the linear branch ---- */
+    for (int J = 0; J < n_kb; ++J) {
+        memset(G, 0, sizeof(double) * dd);
+        memset(gz, 0, sizeof(double) * (size_t)d);
+        for (int I = 0; I < n_qb; ++I) {
+            if (selected[(size_t)I * n_kb + J]) continue;
+            for (size_t e = 0; e < dd; ++e) G[e] += dH[(size_t)I * dd + e];
+            for (int c = 0; c < d; ++c) gz[c] += dZ[(size_t)I * d + c];
+        }
+        int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+        for (int j = t0; j < t1; ++j) {
+            for (int e = 0; e < d; ++e) w[e] = bf(v[(size_t)j * d + e]);
+            for (int c = 0; c < d; ++c) {
+                double kc = bf(k[(size_t)j * d + c]), fk = phi_f(kc, phi);
+                double dfk = gz[c];
+                for (int e = 0; e < d; ++e) {
+                    dfk += G[(size_t)c * d + e] * w[e];
+                    dv[(size_t)j * d + e] += G[(size_t)c * d + e] * fk;
+                }
+                dk[(size_t)j * d + c] += dfk * dphi_f(kc, phi);
+            }
+        }
+    }
+    free(h); free(z); free(dH); free(dZ); free(HI); free(ZI); free(G); free(gz); free(p); free(vec); free(selected);
+    return 0;
+}
+
+/* Gradients of every head ([BH][N][d] bf16 q, k, v, dout -> fp64 dq, dk, dv).
+ * idx_in (nullable, [BH][n_qb][k_sel]) replaces the oracle's own selection.
+ * Returns 0, or -1 when memory runs out. */
+int orc_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int BH, int N,
+                 int d, int blk_q, int blk_k, double topk, int phi, const int32_t *idx_in, double *dq, double *dk,
+                 double *dv)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int k_sel = orc_topk_count(n_kb, topk);
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : fail)
+    for (int bh = 0; bh < BH; ++bh) {
+        size_t hd = (size_t)N * d;
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * ((size_t)n_qb * k_sel + 1));
+        if (!idx) { fail |= 1; continue; }
+        if (idx_in)
+            memcpy(idx, idx_in + (size_t)bh * n_qb * k_sel, sizeof(int32_t) * (size_t)n_qb * k_sel);
+        else
+            mask_head(q + bh * hd, k + bh * hd, N, d, blk_q, blk_k, k_sel, idx, NULL, NULL);
+        if (backward_head(q + bh * hd, k + bh * hd, v + bh * hd, dout + bh * hd, N, d, blk_q, blk_k, k_sel, idx,
+                          phi, dq + bh * hd, dk + bh * hd, dv + bh * hd))
+            fail |= 1;
+        free(idx);
+    }
+    return fail ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------
  * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架":
  * W8A8 quantises the weights and activations of the linear layers to 8-bit
  * integers and runs them on the INT8 units, with a FusedNorm operator; the

@@ -48,6 +48,18 @@ MUTANTS = {
     "truncating_round": ("float r = rintf(x / s);", "float r = truncf(x / s);"),
     "score_key_index_swap": ("s = fma(qm[(size_t)I * d + c], km[(size_t)J * d + c], s);",
                              "s = fma(qm[(size_t)I * d + c], km[(size_t)((J + 1) % n_kb) * d + c], s);"),
+    "bwd_softmax_drops_D": ("double ds = p[n] * (dp - D);", "double ds = p[n] * dp;"),
+    "bwd_dk_unscaled": ("dk[(size_t)j * d + c] += ds * qi[c] * rsd;", "dk[(size_t)j * d + c] += ds * qi[c];"),
+    "bwd_db_sign": ("double db = -dol / b;", "double db = dol / b;"),
+    "bwd_dH_transposed": ("dHI[(size_t)c * d + e] += f[c] * da[e];", "dHI[(size_t)e * d + c] += f[c] * da[e];"),
+    "bwd_key_side_over_selected": ("if (selected[(size_t)I * n_kb + J]) continue;",
+                                   "if (!selected[(size_t)I * n_kb + J]) continue;"),
+    "bwd_dv_linear_transposed": ("dv[(size_t)j * d + e] += G[(size_t)c * d + e] * fk;",
+                                 "dv[(size_t)j * d + e] += G[(size_t)e * d + c] * fk;"),
+    "bwd_elu_derivative_one": ("return x > 0.0 ? 1.0 : exp(x);\n}\n\nstatic int backward_head",
+                               "return 1.0;\n}\n\nstatic int backward_head"),
+    "bwd_dq_linear_without_dphi": ("dq[(size_t)i * d + c] += df * dphi_f(qi[c], phi);", "dq[(size_t)i * d + c] += df;"),
+    "bwd_dz_dropped": ("double dfk = gz[c];", "double dfk = 0.0;"),
     "ragged_tail_dropped": ("int t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;\n        for (int j = t0; j < t1; ++j) {\n            double l;",
                             "int t0 = J * blk_k, t1 = t0 + blk_k <= N ? t0 + blk_k : t0;\n        for (int j = t0; j < t1; ++j) {\n            double l;"),
 }

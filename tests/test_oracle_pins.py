@@ -30,6 +30,13 @@ of the oracle) and raises AssertionError on a mismatch.  What pins what:
   with and without quantisation, with ragged tails; constant V gives 2c
   (c at topk 0 or 1); convex-hull bounds; ReLU rows with phi(q) = 0 give a
   zero linear part; the row-sampled API equals the full forward.
+* backward         -- float64 autograd of an attention-form PyTorch statement of
+  the unquantised forward (dense token mask; the linear branch as masked
+  phi(Q) phi(K)^T weights, not the oracle's state form), whose values are first
+  checked against ``forward``; topk = 1 against autograd of torch's
+  scaled_dot_product_attention; topk = 0 against autograd of closed-form
+  linear attention; ragged blocks, both phi, and ReLU rows with a zero
+  denominator.
 """
 from __future__ import annotations
 
@@ -487,10 +494,106 @@ def pin_forward_rows(lib):
         assert np.array_equal(part[r], BH[bh, i])
 
 
+# --------------------------------------------------------------------------
+# backward
+# --------------------------------------------------------------------------
+
+def _torch_phi(x, ph):
+    torch = pytest.importorskip("torch")
+    if ph == 1:
+        return torch.relu(x)
+    return torch.where(x > 0, x + 1.0, torch.exp(torch.clamp(x, max=0.0)))
+
+
+def _torch_sla(qt, kt, vt, allowed, ph):
+    """Attention-form statement of the unquantised forward of one head, for
+    autograd: ``allowed[i, j]`` marks the tokens of the key blocks that row i's
+    query block selected; the linear branch weighs the other tokens by
+    phi(q_i).phi(k_j)."""
+    torch = pytest.importorskip("torch")
+    d = qt.shape[-1]
+    any_row = allowed.any(dim=-1, keepdim=True)
+    s = (qt @ kt.T) / math.sqrt(d)
+    s = torch.where(any_row, s.masked_fill(~allowed, float("-inf")), torch.zeros_like(s))
+    p = torch.where(any_row, torch.softmax(s, dim=-1), torch.zeros_like(s))
+    w = (_torch_phi(qt, ph) @ _torch_phi(kt, ph).T) * (~allowed)
+    den = w.sum(dim=-1, keepdim=True)
+    ol = torch.where(den != 0, (w @ vt) / torch.where(den != 0, den, torch.ones_like(den)), torch.zeros_like(qt))
+    return p @ vt + ol
+
+
+def _grads(fn, q, k, v, dout):
+    """float64 autograd of sum(fn(q, k, v) * dout) for bf16-bit inputs of one head."""
+    torch = pytest.importorskip("torch")
+    ts = [torch.from_numpy(synth.bf16_bits_to_f64(x)).requires_grad_(True) for x in (q, k, v)]
+    out = fn(*ts)
+    (out * torch.from_numpy(synth.bf16_bits_to_f64(dout))).sum().backward()
+    return out.detach().numpy(), [t.grad.numpy() for t in ts]
+
+
+def _rel(a, b):
+    return np.abs(a - b).max() / max(np.abs(b).max(), 1e-300)
+
+
+def pin_backward_autograd(lib):
+    torch = pytest.importorskip("torch")
+    blk_q, blk_k = 32, 16
+    for (topk, ph, seed) in ((0.3, 0, 30), (0.6, 0, 31), (0.3, 1, 32), (0.0, 0, 33), (1.0, 1, 34)):
+        q, k, v = _qkv((3, 5, 7), d=32, H=2, seed=seed)          # N = 105: 4 x 7 ragged blocks
+        dout = _qkv((3, 5, 7), d=32, H=2, seed=seed + 100)[0]
+        if ph == 1:  # a row whose phi(q) is zero: zero linear denominator
+            qf = synth.bf16_bits_to_f64(q)
+            qf[0, 1, 40] = -np.abs(qf[0, 1, 40]) - 0.25
+            q = _bits_from_f64(qf)
+        N = q.shape[2]
+        idx, _ = oracle.block_mask(q, k, blk_q, blk_k, topk, lib=lib)
+        out_o = oracle.forward(q, k, v, blk_q, blk_k, topk, phi=ph, quant=0, lib=lib)
+        dq, dk, dv = oracle.backward(q, k, v, dout, blk_q, blk_k, topk, phi=ph, lib=lib)
+        n_qb, n_kb = -(-N // blk_q), -(-N // blk_k)
+        for h in range(2):
+            sel = np.zeros((n_qb, n_kb), dtype=bool)
+            for I in range(n_qb):
+                sel[I, idx[h, I]] = True
+            tok = np.arange(N)
+            allowed = torch.from_numpy(sel[(tok // blk_q)[:, None], (tok // blk_k)[None, :]])
+            out_t, (gq, gk, gv) = _grads(lambda a, b, c: _torch_sla(a, b, c, allowed, ph),
+                                         q[0, h], k[0, h], v[0, h], dout[0, h])
+            assert _rel(out_o[0, h], out_t) < 1e-12, (topk, ph, h, "forward statement")
+            for name, mine, ref in (("dq", dq, gq), ("dk", dk, gk), ("dv", dv, gv)):
+                assert _rel(mine[0, h], ref) < 1e-10, (topk, ph, h, name, _rel(mine[0, h], ref))
+
+
+def pin_backward_dense_limit(lib):
+    torch = pytest.importorskip("torch")
+    q, k, v = _qkv((3, 10, 7), d=64, H=1, seed=40)          # N = 210, ragged blocks
+    dout = _qkv((3, 10, 7), d=64, H=1, seed=41)[0]
+    dq, dk, dv = oracle.backward(q, k, v, dout, 64, 64, 1.0, phi=0, lib=lib)
+    _, ref = _grads(lambda a, b, c: torch.nn.functional.scaled_dot_product_attention(a[None], b[None], c[None])[0],
+                    q[0, 0], k[0, 0], v[0, 0], dout[0, 0])
+    for mine, r in zip((dq, dk, dv), ref):
+        assert _rel(mine[0, 0], r) < 1e-12, _rel(mine[0, 0], r)
+
+
+def pin_backward_linear_limit(lib):
+    q, k, v = _qkv((3, 10, 7), d=32, H=1, seed=42)
+    dout = _qkv((3, 10, 7), d=32, H=1, seed=43)[0]
+    for ph in (0, 1):
+        dq, dk, dv = oracle.backward(q, k, v, dout, 128, 64, 0.0, phi=ph, lib=lib)
+
+        def lin(a, b, c):
+            fq, fk = _torch_phi(a, ph), _torch_phi(b, ph)
+            return (fq @ (fk.T @ c)) / (fq @ fk.sum(dim=0))[:, None]
+
+        _, ref = _grads(lin, q[0, 0], k[0, 0], v[0, 0], dout[0, 0])
+        for mine, r in zip((dq, dk, dv), ref):
+            assert _rel(mine[0, 0], r) < 1e-11, (ph, _rel(mine[0, 0], r))
+
+
 PINS = [pin_topk_count, pin_mask_exhaustive, pin_mask_invariances, pin_mask_degenerate,
         pin_quant_exact_block, pin_quant_bounds, pin_quant_smoothing, pin_forward_dense_limit,
         pin_forward_linear_limit, pin_forward_bruteforce, pin_forward_constant_v, pin_forward_hull,
-        pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward, pin_w8a8_rowquant, pin_w8a8_linear]
+        pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward, pin_w8a8_rowquant, pin_w8a8_linear,
+        pin_backward_autograd, pin_backward_dense_limit, pin_backward_linear_limit]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
