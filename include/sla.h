@@ -173,6 +173,29 @@ SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void 
                                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                                        size_t ws_bytes, void *stream, float *stage_ms);
 
+/* ---- Backward, for SLA fine-tuning ("清华开源TurboDiffusion加速框架", 方法论:
+ * full attention is replaced by SLA and the pretrained model fine-tuned for the
+ * sparsity; "TurboDiffusion" summary page, 主要特点: SLA white-box training).
+ *
+ * Gradients of the unquantised forward (sla_forward with quant = 0) with
+ * respect to q, k and v for the output gradient dout:
+ *   q, k, v, dout  bf16 [B, H, N, d] (dout: dL/d out)
+ *   dq, dk, dv     fp32 [B, H, N, d], overwritten (every element written)
+ * The block selection is a piecewise-constant function of (q, k) and is held
+ * fixed (the forward's own selection, recomputed); every other step is the
+ * exact chain rule: the softmax gradient over the selected tokens, and the
+ * linear branch's through phi(q) H_I / (phi(q) . Z_I) (a zero denominator gives
+ * no gradient) and through the key-block states into k and v.  Arithmetic: the
+ * forward's selection and states recomputed as in sla_forward, the gradient
+ * products in fp32, the state gradients summed over query blocks on the tensor
+ * cores in bf16 x bf16 -> fp32.  Same shapes, limits and alignment as
+ * sla_forward; phi as there.  ws: sla_backward_workspace_bytes bytes, 16-byte
+ * aligned (its status word is read by sla_check).  Asynchronous on `stream`. */
+SLA_API size_t sla_backward_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk);
+SLA_API sla_status sla_backward(const void *q_bf16, const void *k_bf16, const void *v_bf16, const void *dout_bf16,
+                                float *dq, float *dk, float *dv, int B, int H, int N, int d, int blk_q, int blk_k,
+                                float topk, int phi, void *ws, size_t ws_bytes, void *stream);
+
 /* ---- W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架",
  * W8A8 section; "TurboDiffusion" GitHub summary, 主要特点 3: the linear layers'
  * weights and activations quantised to 8-bit integers on the INT8 units, with

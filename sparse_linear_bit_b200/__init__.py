@@ -28,7 +28,7 @@ __all__ = [
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_quantize_qk_fp8", "sla_forward", "sla_check", "workspace",
     "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
     "sla_block_mask_noalloc_limit", "head_shard", "shard_heads", "sla_w8a8_quantize", "sla_w8a8_linear",
-    "w8a8_workspace",
+    "w8a8_workspace", "sla_backward_workspace_bytes", "sla_backward", "backward_workspace",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -70,6 +70,10 @@ lib.sla_w8a8_quantize.restype = _I
 lib.sla_w8a8_workspace_bytes.restype = _SZ
 lib.sla_w8a8_linear.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _SZ, _P]
 lib.sla_w8a8_linear.restype = _I
+lib.sla_backward_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _F]
+lib.sla_backward_workspace_bytes.restype = _SZ
+lib.sla_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _SZ, _P]
+lib.sla_backward.restype = _I
 lib.sla_check.argtypes = [_P, _P]
 lib.sla_check.restype = _I
 
@@ -192,6 +196,27 @@ def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -
     B, H, N, d = _bhnd(q)
     _ok(lib.sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk), int(phi),
                         int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_forward")
+
+
+def sla_backward_workspace_bytes(B, H, N, d, blk_q, blk_k, topk) -> int:
+    return int(lib.sla_backward_workspace_bytes(B, H, N, d, blk_q, blk_k, float(topk)))
+
+
+def backward_workspace(B, H, N, d, blk_q, blk_k, topk, device=None):
+    """Allocate a workspace (uint8 CUDA tensor) large enough for sla_backward."""
+    import torch
+    n = sla_backward_workspace_bytes(B, H, N, d, blk_q, blk_k, topk)
+    if n == 0:
+        raise SlaError(1, "sla_backward_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sla_backward(q, k, v, dout, dq, dk, dv, blk_q, blk_k, topk, phi, ws, stream=None) -> None:
+    """Gradients (fp32 dq, dk, dv) of the unquantised forward for the output gradient dout."""
+    B, H, N, d = _bhnd(q)
+    _ok(lib.sla_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, blk_q,
+                         blk_k, float(topk), int(phi), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+        "sla_backward")
 
 
 PROFILE_STAGES = ("quantize_q", "states", "scores_topk", "quantize_k", "state_reduce", "attention", "total")

@@ -315,6 +315,28 @@ sla_status sla_forward(const void *q, const void *k, const void *v, void *out, i
                        static_cast<cudaStream_t>(stream), nullptr);
 }
 
+size_t sla_backward_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk)
+{
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK) return 0;
+    return backward_workspace_bytes(make_geometry(B, H, N, d, blk_q, blk_k, topk, 0));
+}
+
+sla_status sla_backward(const void *q, const void *k, const void *v, const void *dout, float *dq, float *dk, float *dv,
+                        int B, int H, int N, int d, int blk_q, int blk_k, float topk, int phi, void *ws,
+                        size_t ws_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
+    if (st != SLA_OK) return st;
+    if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_RELU) return SLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(ws))
+        return SLA_ERR_INVALID_ARG;
+    const Geometry g = make_geometry(B, H, N, d, blk_q, blk_k, topk, 0);
+    if (ws_bytes < backward_workspace_bytes(g)) return SLA_ERR_WORKSPACE;
+    SLA_TRY(launch_backward(q, k, v, dout, dq, dk, dv, g, phi, ws, static_cast<cudaStream_t>(stream)));
+    return SLA_OK;
+}
+
 sla_status sla_forward_profile(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d,
                                int blk_q, int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes,
                                void *stream, float *stage_ms)

@@ -54,6 +54,11 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
                              const float *qscale, const float *kscale, const int32_t *idx, const float *hq,
                              const Geometry &g, int phi, void *out, int *status, cudaStream_t s);
 
+// backward of the unquantised forward (sla_backward.cu); the workspace begins with the forward's
+// quant = 0 layout
+size_t backward_workspace_bytes(const Geometry &g);
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *dout, float *dq, float *dk,
+                            float *dv, const Geometry &g, int phi, void *ws, cudaStream_t s);
 // TMA descriptor encoding (driver entry point fetched once through the runtime)
 // W8A8 linear layer (sla_w8a8.cu)
 cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,

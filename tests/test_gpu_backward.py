@@ -1,0 +1,96 @@
+"""GPU parity of the backward (sla_backward, through the C ABI) against the
+fp64 CPU oracle's backward.
+
+Tolerance (relative L2 over each of dq, dk, dv): 5e-3.  The gradient products
+run in fp32, but the recomputed forward state is the forward's own: key-block
+states in bf16 (relative rounding 2^-9), H_I rounded to tf32 (2^-11), and the
+per-query-block state gradients enter G = A^T dH as bf16 (2^-9).  Those steps
+feed only the linear branch's terms, so the linear part of a gradient carries
+up to ~2 x 2^-9 ~ 4e-3 relative error and the whole gradient less.
+Every element must also be finite, and two calls must give identical bytes.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_helpers import rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import sparse_linear_bit_b200 as sla  # noqa: E402
+
+TOL = 5e-3
+
+CASES = {
+    # name: ((B, H, grid), blk_q, topk, phi)
+    "ragged_subtract_elu": ((1, 2, (3, 10, 7)), 128, 0.3, 0),
+    "ragged_complement_relu": ((1, 2, (5, 9, 13)), 64, 0.6, 1),
+    "multi_tile_elu": ((1, 2, (8, 16, 16)), 128, 0.1, 0),
+    "linear_only": ((1, 2, (5, 9, 13)), 128, 0.0, 0),
+    "sparse_only_relu": ((1, 2, (5, 9, 13)), 128, 1.0, 1),
+    "two_batches_q64": ((2, 1, (4, 10, 13)), 64, 0.25, 0),
+    # n_kb = 144 > 128: the transposed state reduction spans two row tiles
+    "n_kb_144": ((1, 1, (8, 32, 36)), 128, 0.1, 0),
+}
+
+
+def run_backward(q, k, v, dout, blk_q, topk, phi):
+    B, H, N, d = q.shape
+    qd, kd, vd, dod = (to_dev(x, torch) for x in (q, k, v, dout))
+    dq, dk, dv = (torch.empty(B, H, N, d, dtype=torch.float32, device="cuda") for _ in range(3))
+    ws = sla.backward_workspace(B, H, N, d, blk_q, 64, topk)
+    sla.sla_backward(qd, kd, vd, dod, dq, dk, dv, blk_q, 64, topk, phi, ws)
+    sla.sla_check(ws)
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_backward_parity(name):
+    (B, H, grid), blk_q, topk, phi = CASES[name]
+    q, k, v = synth.make_qkv(B, H, grid, seed=500 + len(name))
+    dout = synth.make_qkv(B, H, grid, seed=600 + len(name))[0]
+    got = [t.cpu().numpy().astype(np.float64) for t in run_backward(q, k, v, dout, blk_q, topk, phi)]
+    ref = oracle.backward(q, k, v, dout, blk_q, 64, float(np.float32(topk)), phi=phi)
+    for nm, g_, r_ in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(g_).all(), (name, nm)
+        err = rel_l2(g_, r_)
+        assert err <= TOL, (name, nm, err)
+
+
+def test_backward_deterministic():
+    q, k, v = synth.make_qkv(1, 2, (8, 16, 16), seed=77)
+    dout = synth.make_qkv(1, 2, (8, 16, 16), seed=78)[0]
+    a = run_backward(q, k, v, dout, 128, 0.1, 0)
+    b = run_backward(q, k, v, dout, 128, 0.1, 0)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+
+
+def test_backward_full_size_scaling():
+    """14B-720P shape (B=1, H=40, N=75600): the gradients are linear in dout, and
+    doubling dout doubles every fp32 operation exactly, so the results must be
+    exactly twice those for dout; all finite."""
+    w = synth.WORKLOADS["wan14b-720p"]
+    q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
+    dout = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed + 1)[0]
+    qd, kd, vd, dod = (to_dev(x, torch) for x in (q, k, v, dout))
+    del q, k, v, dout
+    B, H, N, d = qd.shape
+    ws = sla.backward_workspace(B, H, N, d, w.blk_q, w.blk_k, 0.1)
+    outs = []
+    for scale in (1.0, 2.0):
+        g = [torch.empty(B, H, N, d, dtype=torch.float32, device="cuda") for _ in range(3)]
+        do_s = (dod.float() * scale).bfloat16()
+        sla.sla_backward(qd, kd, vd, do_s, *g, w.blk_q, w.blk_k, 0.1, 0, ws)
+        sla.sla_check(ws)
+        outs.append(g)
+    for x, y in zip(*outs):
+        assert torch.isfinite(x).all()
+        assert torch.equal(x * 2.0, y)
