@@ -64,6 +64,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-w8a8", action="store_true", help="skip the W8A8 linear-layer measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward (fine-tuning) measurement")
     ap.add_argument("--scaling", default="weak", choices=["weak", "strong", "ulysses"])
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiling runs)")
     return ap.parse_args()
@@ -462,6 +463,45 @@ def main():
                 "int8_peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s x 2 (nominal int8 ratio)"}
         del xw, ww, qx_, qw_, yw
 
+    # ---- backward of the unquantised forward (gradients for SLA fine-tuning) on this rank's
+    #      workload; a side measurement like the W8A8 one (not part of the timed step)
+    bwd = None
+    if rank == 0 and not a.no_backward:
+        gen = torch.Generator(device=dev).manual_seed(11)
+        dout = torch.randn(qd.shape, device=dev, generator=gen).bfloat16()
+        grads = [torch.empty(qd.shape, dtype=torch.float32, device=dev) for _ in range(3)]
+        wsb = sla.backward_workspace(*qd.shape, wl.blk_q, wl.blk_k, a.topk, device=dev)
+        bcall = lambda: sla.sla_backward(qd, kd, vd, dout, *grads, wl.blk_q, wl.blk_k, a.topk, a.phi, wsb,
+                                         stream=stream)
+        bcall()
+        torch.cuda.synchronize(dev)
+        tb = []
+        for _ in range(3):
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            bcall()
+            b1.record(stream)
+            torch.cuda.synchronize(dev)
+            tb.append(b0.elapsed_time(b1))
+        sla.sla_check(wsb, stream=stream)
+        ms_b = float(np.median(tb))
+        Bq, Hq, Nq, dq_ = qd.shape
+        n_qb_b, n_kb_b = -(-Nq // wl.blk_q), -(-Nq // wl.blk_k)
+        k_sel_b = sla.sla_topk_count(n_kb_b, a.topk)
+        # algorithmic fp32 work: per (query block, selected key block) tile the five products of the
+        # softmax backward (S, dP, dV, dQ, dK), 2 * 128 x 64 x d each; per query block the three
+        # d x d products of the linear branch; per key block its two
+        fl_sparse = Bq * Hq * n_qb_b * k_sel_b * 5 * 2.0 * wl.blk_q * wl.blk_k * dq_
+        fl_lin = Bq * Hq * (n_qb_b * 3 * 2.0 * wl.blk_q * dq_ * dq_ + n_kb_b * 2 * 2.0 * wl.blk_k * dq_ * dq_)
+        peak_fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
+        ach = (fl_sparse + fl_lin) / (ms_b * 1e-3) / 1e12
+        bwd = {"ms": ms_b, "what": "dq, dk, dv (fp32) of the unquantised forward for a random dout",
+               "roofline": {"bound": "alu", "achieved": ach, "peak": peak_fp32, "unit": "TFLOP/s",
+                            "frac": ach / peak_fp32,
+                            "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 flop x 1.965 GHz (unit counts, max clock)"},
+               "flops_per_call": fl_sparse + fl_lin}
+        del dout, grads, wsb
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, single GPU only)
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -486,7 +526,7 @@ def main():
                     f"{world} rank(s), one per GPU; " + ("each runs the whole workload" if a.scaling == "weak"
                                                          else "B*H heads split in contiguous ranges"))),
                 "stages_ms": stage_ms, "roofline": roofline,
-                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "w8a8_linear": w8a8,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "w8a8_linear": w8a8, "backward": bwd,
                 "gpu_launches": KERNELS_PER_STEP[a.quant] * a.steps,
                 "dense_equiv_ops_per_step_per_gpu": ops}
         print(json.dumps(line), flush=True)
