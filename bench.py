@@ -488,17 +488,18 @@ def main():
         Bq, Hq, Nq, dq_ = qd.shape
         n_qb_b, n_kb_b = -(-Nq // wl.blk_q), -(-Nq // wl.blk_k)
         k_sel_b = sla.sla_topk_count(n_kb_b, a.topk)
-        # algorithmic fp32 work: per (query block, selected key block) tile the five products of the
+        # algorithmic work: per (query block, selected key block) tile the five products of the
         # softmax backward (S, dP, dV, dQ, dK), 2 * 128 x 64 x d each; per query block the three
         # d x d products of the linear branch; per key block its two
         fl_sparse = Bq * Hq * n_qb_b * k_sel_b * 5 * 2.0 * wl.blk_q * wl.blk_k * dq_
         fl_lin = Bq * Hq * (n_qb_b * 3 * 2.0 * wl.blk_q * dq_ * dq_ + n_kb_b * 2 * 2.0 * wl.blk_k * dq_ * dq_)
-        peak_fp32 = 148 * 128 * 2 * 1.965e9 / 1e12
+        # the per-tile products run as bf16 tensor-core MMAs (fp32 accumulation): bf16 tensor peak
         ach = (fl_sparse + fl_lin) / (ms_b * 1e-3) / 1e12
+        p_bf16 = float(peaks["bf16_tflops"])
         bwd = {"ms": ms_b, "what": "dq, dk, dv (fp32) of the unquantised forward for a random dout",
-               "roofline": {"bound": "alu", "achieved": ach, "peak": peak_fp32, "unit": "TFLOP/s",
-                            "frac": ach / peak_fp32,
-                            "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 flop x 1.965 GHz (unit counts, max clock)"},
+               "roofline": {"bound": "tensor", "achieved": ach, "peak": p_bf16, "unit": "TFLOP/s",
+                            "frac": ach / p_bf16, "peak_source": f"{peak_kind} bf16 {p_bf16} TFLOP/s (burst)",
+                            "note": "warp-level mma.sync m16n8k16 bf16 products; the linear branch in fp32"},
                "flops_per_call": fl_sparse + fl_lin}
         del dout, grads, wsb
 

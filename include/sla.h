@@ -186,9 +186,11 @@ SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void 
  * exact chain rule: the softmax gradient over the selected tokens, and the
  * linear branch's through phi(q) H_I / (phi(q) . Z_I) (a zero denominator gives
  * no gradient) and through the key-block states into k and v.  Arithmetic: the
- * forward's selection and states recomputed as in sla_forward, the gradient
- * products in fp32, the state gradients summed over query blocks on the tensor
- * cores in bf16 x bf16 -> fp32.  Same shapes, limits and alignment as
+ * forward's selection and states recomputed as in sla_forward; the sparse
+ * branch's per-tile products on the tensor cores with bf16 operands (P and dS
+ * rounded to bf16) and fp32 accumulation; the linear branch's products in
+ * fp32; the state gradients summed over query blocks on the tensor cores in
+ * bf16 x bf16 -> fp32.  Same shapes, limits and alignment as
  * sla_forward; phi as there.  ws: sla_backward_workspace_bytes bytes, 16-byte
  * aligned (its status word is read by sla_check).  Asynchronous on `stream`. */
 SLA_API size_t sla_backward_workspace_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk);

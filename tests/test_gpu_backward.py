@@ -1,12 +1,14 @@
 """GPU parity of the backward (sla_backward, through the C ABI) against the
 fp64 CPU oracle's backward.
 
-Tolerance (relative L2 over each of dq, dk, dv): 5e-3.  The gradient products
-run in fp32, but the recomputed forward state is the forward's own: key-block
-states in bf16 (relative rounding 2^-9), H_I rounded to tf32 (2^-11), and the
-per-query-block state gradients enter G = A^T dH as bf16 (2^-9).  Those steps
-feed only the linear branch's terms, so the linear part of a gradient carries
-up to ~2 x 2^-9 ~ 4e-3 relative error and the whole gradient less.
+Tolerance (relative L2 over each of dq, dk, dv): 5e-3.  The sparse branch's
+per-tile products take bf16 operands (the inputs themselves, and P and dS
+rounded to bf16: relative 2^-9 per element, with fp32 accumulation, so the
+error of a sum of many such terms stays near 2^-9 or below); the linear branch
+uses the forward's own state: key-block states in bf16 (2^-9), H_I rounded to
+tf32 (2^-11), and the state gradients entering G = A^T dH as bf16 (2^-9).  So
+either branch's part of a gradient carries up to ~2 x 2^-9 ~ 4e-3 relative
+error, and the whole gradient less.
 Every element must also be finite, and two calls must give identical bytes.
 """
 from __future__ import annotations
