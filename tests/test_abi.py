@@ -102,6 +102,39 @@ def test_forward_host_validation():
     assert fwd(ws_bytes=need - 1) == 3
 
 
+def bwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, H=2, N=2048, d=128, blk_q=64,
+             blk_k=64, topk=0.1, phi=0, ws=FAKE, ws_bytes=0, stream=None)
+    a.update(kw)
+    return L.sla_backward(a["q"], a["k"], a["v"], a["dout"], a["dq"], a["dk"], a["dv"], a["B"], a["H"], a["N"],
+                          a["d"], a["blk_q"], a["blk_k"], a["topk"], a["phi"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_backward_host_validation():
+    assert bwd(dout=None) == 1 and bwd(dq=None) == 1 and bwd(dv=None) == 1
+    assert bwd(dk=FAKE + 4) == 1           # misaligned
+    assert bwd(B=0) == 1 and bwd(topk=-0.5) == 1 and bwd(phi=3) == 1
+    assert bwd(d=64) == 2 and bwd(blk_q=256) == 2 and bwd(blk_k=32) == 2
+    assert bwd(ws_bytes=0) == 3            # workspace too small (everything else valid)
+    need = sla.sla_backward_workspace_bytes(1, 2, 2048, 128, 64, 64, 0.1)
+    assert bwd(ws_bytes=need - 1) == 3
+
+
+def test_backward_workspace_bytes():
+    # the backward's workspace starts with the forward's (quantisation off) and adds its own regions
+    for (B, H, N, blk_q, topk) in ((1, 2, 2048, 64, 0.1), (1, 40, 75600, 128, 0.1), (2, 3, 585, 64, 0.6),
+                                   (1, 1, 210, 128, 0.0), (1, 1, 210, 128, 1.0)):
+        f = sla.sla_workspace_bytes(B, H, N, 128, blk_q, 64, topk, 0)
+        b = sla.sla_backward_workspace_bytes(B, H, N, 128, blk_q, 64, topk)
+        n_qb, n_kb = -(-N // blk_q), -(-N // 64)
+        # at least: row statistics, dH in fp32 and bf16, and G, over the state columns
+        extra = B * H * (3 * N * 4 + n_qb * 16512 * 6 + n_kb * 16512 * 4)
+        assert b >= f + extra, (B, H, N, blk_q, topk)
+    assert sla.sla_backward_workspace_bytes(1, 2, 2048, 64, 64, 64, 0.1) == 0     # d != 128
+    assert sla.sla_backward_workspace_bytes(1, 2, 2048, 128, 96, 64, 0.1) == 0    # blk_q
+    assert sla.sla_backward_workspace_bytes(1, 2, 2048, 128, 64, 64, 1.5) == 0    # topk
+
+
 def test_block_mask_and_quant_host_validation():
     assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, 0.1, None, None, FAKE, 1 << 40, None) == 1
     assert L.sla_block_mask(FAKE, FAKE, 1, 2, 2048, 128, 64, 64, 0.1, FAKE + 2, None, FAKE, 1 << 40, None) == 1
