@@ -420,7 +420,9 @@ def main():
                 "peak_source": f"{peak_kind} bf16 {peaks['bf16_tflops']} TFLOP/s (burst); int8/fp8 = 2x, tf32 = 0.5x",
                 "ops_per_launch": {{0: "qk_bf16", 1: "qk_int8", 2: "qk_fp8"}[a.quant]: ops_qk, "pv_bf16": ops_pv,
                                    "linear_tf32": ops_lin},
-                "launch_ms": stage_ms["attention"]}
+                "launch_ms": stage_ms["attention"],
+                # the same ideal tensor time over the whole call (every stage of the step)
+                "whole_call_frac": ideal / (ms * 1e-3)}
 
     # ---- W8A8 INT8 linear layer (+ FusedNorm) at the DiT projection shape of this workload:
     #      the N tokens of one sample x hidden 5120 -> 5120 (the 14B model's width)
