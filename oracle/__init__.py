@@ -78,6 +78,8 @@ def load(path: Optional[str] = None):
     lib.orc_forward.restype = i32
     lib.orc_backward.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, P, P, P, P]
     lib.orc_backward.restype = i32
+    lib.orc_backward_dq_rows.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, P, P, i64, P]
+    lib.orc_backward_dq_rows.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -237,6 +239,25 @@ def backward(q, k, v, dout, blk_q: int, blk_k: int, topk: float, phi: int = 0,
     if rc != 0:
         raise MemoryError("oracle backward failed (out of memory)")
     return dq, dk, dv
+
+
+def backward_dq_rows(q, k, v, dout, blk_q: int, blk_k: int, topk: float, rows, phi: int = 0,
+                     idx: Optional[np.ndarray] = None, lib=None) -> np.ndarray:
+    """fp64 dq of the rows ``rows`` (int64 [n, 2] of (bh, i)) only: the same
+    steps as ``backward``'s dq, evaluable at sizes where the full backward is too
+    slow.  Returns ``[n, d]``."""
+    lib = lib or load()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    BH, N, d = _shape(q)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    out = np.zeros((rows.shape[0], d), dtype=np.float64)
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    rc = lib.orc_backward_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), BH, N, d, blk_q, blk_k, float(topk),
+                                  int(phi), _ptr(idx), _ptr(rows), rows.shape[0], _ptr(out))
+    if rc != 0:
+        raise MemoryError("oracle backward_dq_rows failed (out of memory or bad row index)")
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -706,6 +706,123 @@ int orc_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const 
     return fail ? -1 : 0;
 }
 
+/* dq of a list of rows only (rows: [nrows][2] pairs (bh, i); dq_out [nrows][d]):
+ * the same steps as the backward's dq, which needs only row i, its selected
+ * blocks and its query block's unselected state, so that it can be evaluated
+ * at sizes where the full backward is too slow.  idx_in as in orc_backward.
+ * Returns 0, or -1 when memory runs out or a row is out of range. */
+int orc_backward_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int BH,
+                         int N, int d, int blk_q, int blk_k, double topk, int phi, const int32_t *idx_in,
+                         const int64_t *rows, int64_t nrows, double *dq_out)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int k_sel = orc_topk_count(n_kb, topk);
+    const double rsd_ = 1.0 / sqrt((double)d);
+    size_t hd = (size_t)N * d, dd = (size_t)d * d;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[2 * r] < 0 || rows[2 * r] >= BH || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= N) return -1;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : fail)
+    for (int bh = 0; bh < BH; ++bh) {
+        int any = 0;
+        for (int64_t r = 0; r < nrows; ++r) any |= rows[2 * r] == bh;
+        if (!any) continue;
+        const uint16_t *qh = q + bh * hd, *kh = k + bh * hd, *vh = v + bh * hd, *dh = dout + bh * hd;
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * ((size_t)n_qb * k_sel + 1));
+        double *h = (double *)malloc(sizeof(double) * (size_t)n_kb * dd);
+        double *z = (double *)malloc(sizeof(double) * (size_t)n_kb * d);
+        double *HI = (double *)malloc(sizeof(double) * dd);
+        double *ZI = (double *)malloc(sizeof(double) * (size_t)d);
+        double *p = (double *)malloc(sizeof(double) * ((size_t)k_sel * blk_k + 1));
+        double *vec = (double *)malloc(sizeof(double) * 8 * (size_t)d);
+        if (!idx || !h || !z || !HI || !ZI || !p || !vec) {
+            free(idx); free(h); free(z); free(HI); free(ZI); free(p); free(vec);
+            fail |= 1;
+            continue;
+        }
+        if (idx_in)
+            memcpy(idx, idx_in + (size_t)bh * n_qb * k_sel, sizeof(int32_t) * (size_t)n_qb * k_sel);
+        else
+            mask_head(qh, kh, N, d, blk_q, blk_k, k_sel, idx, NULL, NULL);
+        states_head(kh, vh, N, d, blk_k, phi, h, z);
+        double *qi = vec, *doi = vec + d, *os = vec + 2 * d, *f = vec + 3 * d, *a = vec + 4 * d, *da = vec + 6 * d;
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (rows[2 * r] != bh) continue;
+            int i = (int)rows[2 * r + 1], I = i / blk_q;
+            const int32_t *sel = idx + (size_t)I * k_sel;
+            double *out = dq_out + (size_t)r * d;
+            for (int c = 0; c < d; ++c) {
+                qi[c] = bf(qh[(size_t)i * d + c]);
+                doi[c] = bf(dh[(size_t)i * d + c]);
+                out[c] = 0.0;
+            }
+            /* sparse branch */
+            int nk = 0;
+            double mx = -INFINITY;
+            for (int s_ = 0; s_ < k_sel; ++s_) {
+                int J = sel[s_], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                for (int j = t0; j < t1; ++j) {
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += qi[c] * bf(kh[(size_t)j * d + c]);
+                    p[nk] = s * rsd_;
+                    if (p[nk] > mx) mx = p[nk];
+                    ++nk;
+                }
+            }
+            if (nk > 0) {
+                double den = 0.0;
+                for (int n = 0; n < nk; ++n) {
+                    p[n] = exp(p[n] - mx);
+                    den += p[n];
+                }
+                for (int n = 0; n < nk; ++n) p[n] /= den;
+                for (int e = 0; e < d; ++e) os[e] = 0.0;
+                int n = 0;
+                for (int s_ = 0; s_ < k_sel; ++s_) {
+                    int J = sel[s_], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                    for (int j = t0; j < t1; ++j, ++n)
+                        for (int e = 0; e < d; ++e) os[e] += p[n] * bf(vh[(size_t)j * d + e]);
+                }
+                double D = 0.0;
+                for (int e = 0; e < d; ++e) D += doi[e] * os[e];
+                n = 0;
+                for (int s_ = 0; s_ < k_sel; ++s_) {
+                    int J = sel[s_], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+                    for (int j = t0; j < t1; ++j, ++n) {
+                        double dp = 0.0;
+                        for (int e = 0; e < d; ++e) dp += doi[e] * bf(vh[(size_t)j * d + e]);
+                        double ds = (dp - D) * p[n]; /* same product as the full backward */
+                        for (int c = 0; c < d; ++c) out[c] += ds * bf(kh[(size_t)j * d + c]) * rsd_;
+                    }
+                }
+            }
+            /* linear branch */
+            unselected_state(sel, k_sel, n_kb, d, h, z, HI, ZI);
+            double b = 0.0;
+            for (int c = 0; c < d; ++c) {
+                f[c] = phi_f(qi[c], phi);
+                b += f[c] * ZI[c];
+            }
+            if (b == 0.0) continue;
+            double dol = 0.0;
+            for (int e = 0; e < d; ++e) {
+                a[e] = 0.0;
+                for (int c = 0; c < d; ++c) a[e] += f[c] * HI[(size_t)c * d + e];
+                dol += doi[e] * (a[e] / b);
+                da[e] = doi[e] / b;
+            }
+            double db = -(dol / b);
+            for (int c = 0; c < d; ++c) {
+                double df = ZI[c] * db;
+                for (int e = 0; e < d; ++e) df += HI[(size_t)c * d + e] * da[e];
+                out[c] += df * dphi_f(qi[c], phi);
+            }
+        }
+        free(idx); free(h); free(z); free(HI); free(ZI); free(p); free(vec);
+    }
+    return fail ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------------
  * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架":
  * W8A8 quantises the weights and activations of the linear layers to 8-bit

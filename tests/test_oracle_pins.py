@@ -36,7 +36,7 @@ of the oracle) and raises AssertionError on a mismatch.  What pins what:
   checked against ``forward``; topk = 1 against autograd of torch's
   scaled_dot_product_attention; topk = 0 against autograd of closed-form
   linear attention; ragged blocks, both phi, and ReLU rows with a zero
-  denominator.
+  denominator; the row-sampled dq equals the full backward's.
 """
 from __future__ import annotations
 
@@ -589,11 +589,24 @@ def pin_backward_linear_limit(lib):
             assert _rel(mine[0, 0], r) < 1e-11, (ph, _rel(mine[0, 0], r))
 
 
+def pin_backward_rows(lib):
+    """The row-sampled dq equals the full backward's dq, row for row."""
+    q, k, v = _qkv((3, 10, 7), d=32, H=3, seed=44)
+    dout = _qkv((3, 10, 7), d=32, H=3, seed=45)[0]
+    for ph, topk, bq in ((0, 0.3, 64), (1, 0.7, 32)):
+        dq, _, _ = oracle.backward(q, k, v, dout, bq, 32, topk, phi=ph, lib=lib)
+        rows = np.array([[2, 209], [0, 0], [1, 64], [2, 3], [0, 150], [1, 65]], dtype=np.int64)
+        part = oracle.backward_dq_rows(q, k, v, dout, bq, 32, topk, rows, phi=ph, lib=lib)
+        full = dq.reshape(-1, 210, 32)
+        for r, (bh, i) in enumerate(rows):
+            assert np.array_equal(part[r], full[bh, i]), (ph, topk, bh, i)
+
+
 PINS = [pin_topk_count, pin_mask_exhaustive, pin_mask_invariances, pin_mask_degenerate,
         pin_quant_exact_block, pin_quant_bounds, pin_quant_smoothing, pin_forward_dense_limit,
         pin_forward_linear_limit, pin_forward_bruteforce, pin_forward_constant_v, pin_forward_hull,
         pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward, pin_w8a8_rowquant, pin_w8a8_linear,
-        pin_backward_autograd, pin_backward_dense_limit, pin_backward_linear_limit]
+        pin_backward_autograd, pin_backward_dense_limit, pin_backward_linear_limit, pin_backward_rows]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
