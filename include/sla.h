@@ -1,5 +1,6 @@
 /*
- * sla.h -- C ABI of libsla.so: the SageSLA attention forward on B200 (sm_100a).
+ * sla.h -- C ABI of libsla.so: the SageSLA attention forward (and its backward)
+ * on B200 (sm_100a).
  *
  * SageSLA is Sparse-Linear Attention (SLA) with a SageAttention-style sparse
  * part, the attention used by TurboDiffusion's video DiT
@@ -35,6 +36,12 @@
  *      Z_I = sum_{J unselected} (column sums of phi(K_J)); phi acts on the raw
  *      Q and K; a zero denominator gives a zero linear output;
  *   6. out = sparse + linear, rounded to bf16.
+ *
+ * Beside the forward and its steps, the library exports the backward of the
+ * unquantised forward (sla_backward: dq, dk, dv, for SLA fine-tuning), the
+ * W8A8 INT8 linear layer with FusedNorm (sla_w8a8_*) and the block
+ * permutations around a Ulysses all-to-all (sla_ulysses_permute); each is
+ * described where it is declared.
  *
  * Layout: q, k, v, out are contiguous bf16 [B, H, N, d] (token index t-major).
  * Only d = 128, blk_k = 64 and blk_q in {64, 128} are supported.
