@@ -7,7 +7,7 @@
  * ("TurboDiffusion技术架构解析：稀疏线性注意力应用实战" §2.1: standard
  * attention softmax(QK^T/sqrt(d))V, linear attention phi(Q)(phi(K)^T V) with
  * phi = ReLU or elu+1, and SLA keeping the top-k% most important key-value
- * pairs; "TurboDiffusion" GitHub summary, 使用方式与安装: SageSLA is the
+ * pairs; "TurboDiffusion" summary page, 使用方式与安装: SageSLA is the
  * SageAttention-based fast SLA forward; "清华开源TurboDiffusion加速框架",
  * SageAttention与稀疏计算: INT8 low-bit attention on the tensor cores, about
  * 10% of the attention connections kept).
@@ -23,8 +23,9 @@
  *      Q and the smoothed K quantised with one fp32 scale per block: INT8 with
  *      quant = 1 (scale = amax/127, code = clamp(rint_even(x/scale), +-127)),
  *      FP8 e4m3 with quant = 2 (scale = amax/448, code = the e4m3 value
- *      nearest to x/scale, ties to even, saturating at +-448; the same section
- *      names FP8 beside INT8); every step in IEEE fp32;
+ *      nearest to x/scale, ties to even, saturating at +-448; no page names
+ *      FP8 -- the SageAttention section speaks of INT8/INT4 -- so quant = 2 is
+ *      an added mode on the same per-block scaling); every step in IEEE fp32;
  *   4. sparse branch: per query row, exact softmax attention over the tokens of
  *      the selected key blocks; logits (qhat.khat)*s_q*s_k/sqrt(d) with
  *      quant = 1 or 2 (INT8 MMA with int32 sums, or FP8 MMA with fp32 sums),
@@ -153,12 +154,16 @@ SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void
  * file-scope device array of sla_block_mask_noalloc_limit() bytes (16 MiB),
  * which every GPU that loads the library holds until the process exits.
  * Problems whose scratch would exceed it return SLA_ERR_WORKSPACE before any
- * launch (about B*H*n_qb*(8*n_kb + 8*ceil(n_kb/64)) + 1 KiB*B*H*(n_qb + n_kb)
- * bytes are needed).  It allocates nothing.
+ * launch.  The scratch is the sum of these regions, each rounded up to a
+ * multiple of 256 bytes: 1024*B*H*n_qb and 1024*B*H*n_kb (fp64 block means),
+ * 8*B*H*n_qb*n_kb (fp64 scores), 8*B*H*n_qb*ceil(n_kb/64) (mask rows), and
+ * 4*B*H*n_qb only when k_sel == 0.  It allocates nothing.
  *
  * The first call on a device resolves the array's device address for that
  * device (cudaGetSymbolAddress, device current); make that first call before
- * any stream capture.  All calls share the one array: calls whose work
+ * any stream capture.  The address is kept for the life of the process: it
+ * does not survive cudaDeviceReset of that device, so do not call this entry
+ * point on a device after resetting it.  All calls share the one array: calls whose work
  * overlaps on the GPU (different streams, or different host threads without
  * ordering) race on it and must be serialised by the caller.  Nothing in the
  * array needs to start at zero: every value a call reads it wrote first. */
@@ -180,9 +185,10 @@ SLA_API sla_status sla_forward_profile(const void *q, const void *k, const void 
                                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                                        size_t ws_bytes, void *stream, float *stage_ms);
 
-/* ---- Backward, for SLA fine-tuning ("清华开源TurboDiffusion加速框架", 方法论:
- * full attention is replaced by SLA and the pretrained model fine-tuned for the
- * sparsity; "TurboDiffusion" summary page, 主要特点: SLA white-box training).
+/* ---- Backward, for SLA fine-tuning (the jiqiren.org.cn TurboDiffusion article,
+ * 方法论: full attention is replaced by SLA and the pretrained model fine-tuned
+ * for the sparsity; "TurboDiffusion" summary page, 主要能力: SLA white-box
+ * training).
  *
  * Gradients of the unquantised forward (sla_forward with quant = 0) with
  * respect to q, k and v for the output gradient dout:
@@ -206,9 +212,10 @@ SLA_API sla_status sla_backward(const void *q_bf16, const void *k_bf16, const vo
                                 float topk, int phi, void *ws, size_t ws_bytes, void *stream);
 
 /* ---- W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架",
- * W8A8 section; "TurboDiffusion" GitHub summary, 主要特点 3: the linear layers'
- * weights and activations quantised to 8-bit integers on the INT8 units, with
- * a FusedNorm operator).  This is not part of the attention forward. */
+ * W8A8 INT8量化: the linear layers' weights and activations quantised to 8-bit
+ * integers on the INT8 units; "TurboDiffusion：让可视化视频生成效率提升200倍的
+ * 加速引擎" §1: W8A8 with a FusedNorm operator).  This is not part of the
+ * attention forward. */
 
 /* Per-row symmetric INT8 quantisation of a bf16 matrix x [rows, cols]
  * (row-major): one fp32 scale per row, scale = amax / 127, code =
@@ -236,8 +243,8 @@ SLA_API sla_status sla_w8a8_linear(const int8_t *qx, const float *sx, const int8
                            const float *bias, int M, int N, int K, void *out_bf16, void *ws, size_t ws_bytes,
                            void *stream);
 
-/* ---- Ulysses context parallelism (the "TurboDiffusion" GitHub summary,
- * 主要特点: the training code supports Ulysses CP).  Each of P ranks holds
+/* ---- Ulysses context parallelism (the "TurboDiffusion" summary page,
+ * 主要能力: the training code supports Ulysses CP).  Each of P ranks holds
  * n_local = N / P consecutive tokens of every head; an all-to-all regroups them
  * into every token of H / P heads, the attention runs per head, and a second
  * all-to-all restores the token sharding.  This call does the block
@@ -252,6 +259,20 @@ SLA_API sla_status sla_w8a8_linear(const int8_t *qx, const float *sx, const int8
  * SLA_ERR_UNSUPPORTED); src, dst 16-byte aligned and distinct. */
 SLA_API sla_status sla_ulysses_permute(const void *src, void *dst, int B, int H, int P, int n_local, int d,
                                int elem_bytes, int mode, void *stream);
+
+/* Diagnostics: sets, on the current device, the clock-cycle budget after which
+ * every bounded wait in the library's kernels gives up (cycles > 0), or
+ * restores the default of 10^9 cycles, about 0.5 s (cycles = 0).  A wait that
+ * runs out records SLA_ERR_TIMEOUT in the call's status word and the kernel
+ * unwinds: it stops issuing work, lets the copies and tensor-core operations
+ * it already issued retire (those drain waits always keep the default budget),
+ * releases its tensor memory and returns.  A budget of a few cycles therefore
+ * makes any call whose kernels wait at all fail cleanly, which is how the
+ * failure path is tested.  Process-wide per device and not ordered with
+ * launches on other host threads: set it while no other call is being
+ * enqueued.  Returns SLA_ERR_INVALID_ARG for cycles < 0, SLA_ERR_CUDA if the
+ * setting could not be copied to the device.  The pages have no counterpart. */
+SLA_API sla_status sla_set_wait_budget(long long cycles);
 
 /* Synchronises `stream` and returns the device-side status word of `ws`
  * (SLA_OK, or SLA_ERR_TIMEOUT when a bounded wait ran out), or SLA_ERR_CUDA

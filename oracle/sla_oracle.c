@@ -23,8 +23,9 @@
  *     K is smoothed by its per-channel mean over all N tokens; per block
  *     scale = amax / 127 in fp32; code = clamp(rint_even(x / scale), -127,
  *     127), every step in IEEE fp32 so that a GPU can reproduce it exactly.
- *     FP8 variant (quant = 2; the same section names FP8 beside INT8): scale =
- *     amax / 448 and code = the fp8 e4m3 value nearest to x / scale (ties to
+ *     FP8 variant (quant = 2): no page names FP8 -- that section speaks of
+ *     INT8/INT4 only -- so this mode is an addition on the same per-block
+ *     scaling, for the e4m3 tensor-core path: scale = amax / 448 and code = the fp8 e4m3 value nearest to x / scale (ties to
  *     even, saturating at +-448; e4m3: 4 exponent bits with bias 7, 3
  *     mantissa bits, subnormals down to 2^-9, no infinities).
  *  5. Sparse branch: for every query row, exact softmax attention
@@ -514,9 +515,9 @@ int orc_forward(const uint16_t *q, const uint16_t *k, const uint16_t *v, int BH,
 /* ------------------------------------------------------------------------
  * Backward: gradients of the unquantised forward (steps 1-3, 5-7 with
  * quant = 0) with respect to q, k and v, for SLA fine-tuning
- * ("清华开源TurboDiffusion加速框架", 方法论: full attention is replaced by SLA
- * and the pretrained model is fine-tuned for the sparsity; the "TurboDiffusion"
- * summary page, 主要特点: SLA white-box training).  The block selection is a
+ * (the jiqiren.org.cn TurboDiffusion article, 方法论: full attention is
+ * replaced by SLA and the pretrained model is fine-tuned for the sparsity; the
+ * "TurboDiffusion" summary page, 主要能力: SLA white-box training).  The block selection is a
  * piecewise-constant function of (q, k), so it is held fixed; everything else
  * is differentiated exactly (chain rule, fp64).  With do = dL/dO:
  *
@@ -824,11 +825,12 @@ int orc_backward_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v
 }
 
 /* ------------------------------------------------------------------------
- * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架":
- * W8A8 quantises the weights and activations of the linear layers to 8-bit
- * integers and runs them on the INT8 units, with a FusedNorm operator; the
- * "TurboDiffusion" GitHub summary, 主要特点 3: W8A8 accelerates the linear
- * layers).  Granularity, rounding and the norm are not stated; the readings:
+ * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架",
+ * W8A8 INT8量化: the weights and activations of the linear layers quantised
+ * to 8-bit integers for the INT8 units; the jiqiren.org.cn TurboDiffusion
+ * article, 方法论 item 4: W8A8 accelerates the linear layers; "TurboDiffusion：
+ * 让可视化视频生成效率提升200倍的加速引擎" §1: W8A8 together with a FusedNorm
+ * operator).  Granularity, rounding and the norm are not stated; the readings:
  *   - activations: one symmetric scale per token (row), weights: one per
  *     output channel (row of W [N, K]); scale = amax / 127 and code =
  *     clamp(rint_even(y / scale), +-127) in IEEE fp32, the SageSLA rule;

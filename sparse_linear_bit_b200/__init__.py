@@ -10,7 +10,8 @@ and streams.  The functions carry the C names:
 * ``sla_quantize_qk(q, k, blk_q, blk_k, q_i8, k_i8, q_scale, k_scale, k_mean, ws)``
 * ``sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws)``
 * ``sla_forward_profile(...)`` (per-stage device times), ``sla_check(ws)``,
-  ``sla_status_string(code)``, ``sla_workspace_layout(...)``
+  ``sla_status_string(code)``, ``sla_workspace_layout(...)``,
+  ``sla_set_wait_budget(cycles)`` (diagnostics: the bounded waits' budget)
 
 Tensors are CUDA tensors laid out as the header states ([B, H, N, d] bf16 for
 q/k/v/out).  Calls enqueue on torch's current stream (or ``stream=``).  A
@@ -28,7 +29,7 @@ __all__ = [
     "sla_workspace_layout", "sla_block_mask", "sla_quantize_qk", "sla_quantize_qk_fp8", "sla_forward", "sla_check", "workspace",
     "LAYOUT_REGIONS", "LIB_PATH", "sla_forward_profile", "PROFILE_STAGES", "sla_block_mask_noalloc",
     "sla_block_mask_noalloc_limit", "head_shard", "shard_heads", "sla_w8a8_quantize", "sla_w8a8_linear",
-    "w8a8_workspace", "sla_backward_workspace_bytes", "sla_backward", "backward_workspace",
+    "w8a8_workspace", "sla_backward_workspace_bytes", "sla_backward", "backward_workspace", "sla_set_wait_budget",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsla.so")
@@ -76,6 +77,8 @@ lib.sla_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
 lib.sla_backward.restype = _I
 lib.sla_check.argtypes = [_P, _P]
 lib.sla_check.restype = _I
+lib.sla_set_wait_budget.argtypes = [ctypes.c_longlong]
+lib.sla_set_wait_budget.restype = _I
 
 
 class SlaError(RuntimeError):
@@ -230,6 +233,12 @@ def sla_forward_profile(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream
                                 int(phi), int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream),
                                 arr), "sla_forward_profile")
     return {name: float(arr[i]) for i, name in enumerate(PROFILE_STAGES)}
+
+
+def sla_set_wait_budget(cycles: int) -> None:
+    """Clock-cycle budget of every bounded wait in the kernels on the current device
+    (0 restores the default, about 0.5 s): a diagnostic for the failure path."""
+    _ok(lib.sla_set_wait_budget(int(cycles)), "sla_set_wait_budget")
 
 
 def sla_check(ws, stream=None) -> None:

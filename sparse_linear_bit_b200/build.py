@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     objs = []
     for src in SOURCES:
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-dc" if False else "-c",
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c",
                os.path.join(CSRC, src), "-o", obj]
         if ptxas_verbose:
             cmd += ["-Xptxas", "-v"]

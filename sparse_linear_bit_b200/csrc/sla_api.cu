@@ -106,6 +106,18 @@ namespace {
 
 bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
 
+char *ws_at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
+
+#define SLA_TRY(expr)                                                    \
+    do {                                                                 \
+        cudaError_t _e = (expr);                                         \
+        if (_e != cudaSuccess) return SLA_ERR_CUDA;                      \
+    } while (0)
+
+}  // namespace
+
+namespace sla {
+
 // shared validation of (B, H, N, d, blk_q, blk_k, topk)
 sla_status check_shape(int B, int H, int N, int d, int blk_q, int blk_k, float topk)
 {
@@ -119,17 +131,6 @@ sla_status check_shape(int B, int H, int N, int d, int blk_q, int blk_k, float t
     return SLA_OK;
 }
 
-char *ws_at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
-
-#define SLA_TRY(expr)                                                    \
-    do {                                                                 \
-        cudaError_t _e = (expr);                                         \
-        if (_e != cudaSuccess) return SLA_ERR_CUDA;                      \
-    } while (0)
-
-}  // namespace
-
-namespace sla {
 sla_status quantize_qk(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k, int fp8,
                            int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale, float *k_mean, void *ws,
                            size_t ws_bytes, void *stream)
@@ -358,6 +359,15 @@ sla_status sla_forward_profile(const void *q, const void *k, const void *v, void
     }
     for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
     return st;
+}
+
+sla_status sla_set_wait_budget(long long cycles)
+{
+    if (cycles < 0) return SLA_ERR_INVALID_ARG;
+    if (set_wait_budget_attention(cycles) != cudaSuccess || set_wait_budget_linear(cycles) != cudaSuccess ||
+        set_wait_budget_w8a8(cycles) != cudaSuccess)
+        return SLA_ERR_CUDA;
+    return SLA_OK;
 }
 
 sla_status sla_check(void *ws, void *stream)

@@ -301,11 +301,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             for (int s = 0; s < NS; ++s) {
                 int tl = -1;
                 for (int t = s; t < issued; t += NS) tl = t;
-                if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / NS) & 1);
+                if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / NS) & 1, status);
             }
         } else {
-            mbar_wait_quiet(&sm.bar_h, 0);
-            mbar_wait_quiet(&sm.bar_qr, 0);
+            mbar_wait_quiet(&sm.bar_h, 0, status);
+            mbar_wait_quiet(&sm.bar_qr, 0, status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ linear-branch MMA
@@ -328,7 +328,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         }
         if (elect_one()) {
             mma_commit(&sm.drain[0]);
-            mbar_wait_quiet(&sm.drain[0], 0);  // this thread's MMAs retired before TMEM is released
+            mbar_wait_quiet(&sm.drain[0], 0, status);  // this thread's MMAs retired before TMEM is released
         }
         __syncwarp();
     } else if (warp >= 10) {
@@ -393,7 +393,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         }
         if (elect_one()) {
             mma_commit(&sm.drain[1 + g]);
-            mbar_wait_quiet(&sm.drain[1 + g], 0);
+            mbar_wait_quiet(&sm.drain[1 + g], 0, status);
         }
         __syncwarp();
     } else {
@@ -656,5 +656,7 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
     if (g.quant == 1) return launch_attn_t<1>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
     return launch_attn_t<0>(q, k, v, q8, k8, qscale, kscale, idx, hq, g, phi, out, status, s);
 }
+
+cudaError_t set_wait_budget_attention(long long cycles) { return set_tu_wait_budget(cycles); }
 
 }  // namespace sla

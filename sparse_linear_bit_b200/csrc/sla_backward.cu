@@ -1,8 +1,8 @@
 // sla_backward.cu -- gradients of the unquantised SageSLA forward with respect
-// to q, k and v, for SLA fine-tuning ("清华开源TurboDiffusion加速框架", 方法论:
-// full attention is replaced by SLA and the pretrained model is fine-tuned for
-// the sparsity; the "TurboDiffusion" summary page, 主要特点: SLA white-box
-// training).  The block selection is piecewise constant in (q, k) and is held
+// to q, k and v, for SLA fine-tuning (the jiqiren.org.cn TurboDiffusion
+// article, 方法论: full attention is replaced by SLA and the pretrained model is
+// fine-tuned for the sparsity; the "TurboDiffusion" summary page, 主要能力: SLA
+// white-box training).  The block selection is piecewise constant in (q, k) and is held
 // fixed; every other step is the exact chain rule of the forward:
 //
 //   sparse branch (row i, selected tokens j, s = q.k / sqrt(d), p = softmax(s),

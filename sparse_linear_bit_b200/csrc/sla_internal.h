@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "../../include/sla.h"
+
 namespace sla {
 
 constexpr int kD = 128;                  // head dimension supported
@@ -25,6 +27,8 @@ struct Layout {
     size_t total;
 };
 
+// argument checks shared by every entry point that takes (B, H, N, d, blk_q, blk_k, topk)
+sla_status check_shape(int B, int H, int N, int d, int blk_q, int blk_k, float topk);
 Geometry make_geometry(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant);
 Layout make_layout(const Geometry &g);
 int topk_count(int n_kb, float topk);
@@ -65,6 +69,11 @@ cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const f
                             float *scale, cudaStream_t s);
 cudaError_t launch_w8a8_gemm(const int8_t *qx, const float *sx, const int8_t *qw, const float *sw, const float *bias,
                              int M, int N, int K, void *out, int *status, cudaStream_t s);
+// run-time override of the bounded waits' budget, one setter per translation unit with waiting
+// kernels (cycles; 0 = default), on the current device
+cudaError_t set_wait_budget_attention(long long cycles);
+cudaError_t set_wait_budget_linear(long long cycles);
+cudaError_t set_wait_budget_w8a8(long long cycles);
 bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const uint64_t *dims,
                  const uint64_t *strides_bytes /* rank-1 entries */, const uint32_t *box);
 

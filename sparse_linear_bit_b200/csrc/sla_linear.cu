@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kStatesThreads, 1) states_kernel(const __grid_
                 for (int s = 0; s < kStStages; ++s) {
                     int jl = -1;
                     for (int x = s; x < j; x += kStStages) jl = x;
-                    if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kStStages) & 1);
+                    if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kStStages) & 1, status);
                 }
             }
         }
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kStatesThreads, 1) states_kernel(const __grid_
                 }
             }
             mma_commit(&sm.drain);
-            mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
+            mbar_wait_quiet(&sm.drain, 0, status);  // MMAs retired before TMEM is freed
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const uint32_t *
             for (int s = 0; s < kRedBStages; ++s) {
                 int jl = -1;
                 for (int j = s; j < kc; j += kRedBStages) jl = j;
-                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedBStages) & 1);
+                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kRedBStages) & 1, status);
             }
         }
     } else if (warp == 1 && lane == 0) {
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const uint32_t *
             mma_commit(&sm.acc_full[buf]);
         }
         mma_commit(&sm.drain);
-        mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
+        mbar_wait_quiet(&sm.drain, 0, status);  // MMAs retired before TMEM is freed
     } else if (warp >= 6) {
         // ------------------------------------------------------------ A builders
         // Thread = one query block (TMEM lane); column c of a k-step holds the mask of key
@@ -680,5 +680,7 @@ cudaError_t launch_state_reduce(const uint32_t *amask, const uint16_t *states, c
                                                                          n_tiles, g.subtract ? 1 : 0, htot, status);
     return cudaGetLastError();
 }
+
+cudaError_t set_wait_budget_linear(long long cycles) { return set_tu_wait_budget(cycles); }
 
 }  // namespace sla

@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double
 // even) is rint(t) in two's complement.
 //
 // FP8 (e4m3) codes: s = amax / 448 and code = e4m3(fl(x / s)), round to nearest
-// even with saturation (SageAttention's FP8 option beside INT8).  The same
+// even with saturation (an added mode: the pages name INT8/INT4 only).  The same
 // reciprocal product is used; |t - fl(x/s)| < 2^-22 |t|, so when t (1 - 2^-20)
 // and t (1 + 2^-20) convert to the same code it is the quotient's code.
 // ---------------------------------------------------------------------------

@@ -52,29 +52,35 @@ size_t sla_block_mask_noalloc_limit(void) { return kStaticScratchBytes; }
 sla_status sla_block_mask_noalloc(const void *q, const void *k, int B, int H, int N, int d, int blk_q, int blk_k,
                                   float topk, int32_t *idx_out, uint32_t *bitmap_out, void *stream)
 {
-    // same arguments and checks as sla_block_mask, minus the workspace
-    if (B < 1 || H < 1 || N < 1 || d < 1 || blk_q < 1 || blk_k < 1) return SLA_ERR_INVALID_ARG;
-    if (!(topk >= 0.0f && topk <= 1.0f)) return SLA_ERR_INVALID_ARG;
-    if (d != sla::kD || blk_k != sla::kBlkK || (blk_q != 64 && blk_q != 128)) return SLA_ERR_UNSUPPORTED;
-    if ((long long)B * H > (1LL << 24) || (long long)N > (1LL << 24)) return SLA_ERR_UNSUPPORTED;
-    // the scratch the mask path uses is the prefix of the forward's workspace layout, up to the mask rows
+    // the checks of sla_block_mask, in the same order, minus the workspace
+    sla_status st = sla::check_shape(B, H, N, d, blk_q, blk_k, topk);
+    if (st != SLA_OK) return st;
     const sla::Geometry g = sla::make_geometry(B, H, N, d, blk_q, blk_k, topk, 0);
-    const sla::Layout L = sla::make_layout(g);
-    const size_t need = L.amask + (size_t)g.BH * g.n_qb * g.n_aw * sizeof(uint32_t);
-    if (need > kStaticScratchBytes) return SLA_ERR_WORKSPACE;  // problem too large for the static scratch
     auto misaligned = [](const void *p, uintptr_t a) { return p == nullptr || ((uintptr_t)p & (a - 1)) != 0; };
     if (misaligned(q, 16) || misaligned(k, 16)) return SLA_ERR_INVALID_ARG;
     if (g.k_sel > 0 && misaligned(idx_out, 4)) return SLA_ERR_INVALID_ARG;
     if (bitmap_out && ((uintptr_t)bitmap_out & 3u)) return SLA_ERR_INVALID_ARG;
+    // scratch regions of the mask path only, each rounded up to 256 bytes: fp64 block means of
+    // Q and K, fp64 scores, the mask rows the top-k kernel also writes, and (k_sel == 0 only)
+    // a stand-in for the empty index lists
+    const size_t BH = (size_t)g.BH;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) / 256 * 256; return o; };
+    const size_t o_qbar = take(BH * g.n_qb * sla::kD * sizeof(double));
+    const size_t o_kbar = take(BH * g.n_kb * sla::kD * sizeof(double));
+    const size_t o_scores = take(BH * g.n_qb * g.n_kb * sizeof(double));
+    const size_t o_amask = take(BH * g.n_qb * (size_t)g.n_aw * sizeof(uint32_t));
+    const size_t o_idx = g.k_sel > 0 ? 0 : take(BH * g.n_qb * sizeof(int32_t));
+    if (off > kStaticScratchBytes) return SLA_ERR_WORKSPACE;  // problem too large for the static scratch
     char *scratch = static_cast<char *>(scratch_for_current_device());
     if (!scratch) return SLA_ERR_CUDA;
     // the mask stages of the forward, with their scratch in the static array
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    double *qbar = reinterpret_cast<double *>(scratch + L.qbar);
-    double *kbar = reinterpret_cast<double *>(scratch + L.kbar);
-    double *scores = reinterpret_cast<double *>(scratch + L.scores);
-    int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(scratch + L.idx);
-    uint32_t *amask = reinterpret_cast<uint32_t *>(scratch + L.amask);
+    double *qbar = reinterpret_cast<double *>(scratch + o_qbar);
+    double *kbar = reinterpret_cast<double *>(scratch + o_kbar);
+    double *scores = reinterpret_cast<double *>(scratch + o_scores);
+    int32_t *idx = g.k_sel > 0 ? idx_out : reinterpret_cast<int32_t *>(scratch + o_idx);
+    uint32_t *amask = reinterpret_cast<uint32_t *>(scratch + o_amask);
     if (sla::launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla::launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, nullptr, s) != cudaSuccess) return SLA_ERR_CUDA;
     if (sla::launch_scores(qbar, kbar, g, scores, s) != cudaSuccess) return SLA_ERR_CUDA;

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_runtime.h>
 
 #define SLA_DEV __device__ __forceinline__
 
@@ -21,6 +22,25 @@ namespace sla {
 constexpr int kStatusTimeout = 5;
 // ~0.5 s at 2 GHz: far above any legitimate wait in these kernels.
 constexpr long long kWaitBudgetCycles = 1000000000LL;
+
+// Run-time override of the budget of the bounded waits (clock cycles; 0 = the
+// default above), one copy per translation unit (internal linkage), set from
+// the host by set_tu_wait_budget.  A diagnostic knob: a short budget makes a
+// wait that is still pending run out, which exercises the failure path.  The
+// drain waits of that path (mbar_wait_quiet) always keep the full default.
+static __device__ long long g_wait_budget_override = 0;
+
+SLA_DEV long long wait_budget()
+{
+    const long long b = g_wait_budget_override;
+    return b > 0 ? b : kWaitBudgetCycles;
+}
+
+// sets this translation unit's override on the current device (blocking copy)
+static inline cudaError_t set_tu_wait_budget(long long cycles)
+{
+    return cudaMemcpyToSymbol(g_wait_budget_override, &cycles, sizeof(cycles));
+}
 
 SLA_DEV void record_error(int *status, int code) { atomicCAS(status, 0, code); }
 
@@ -68,17 +88,17 @@ SLA_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 SLA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, int *status, volatile int *abort_flag)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    long long t0 = clock64();
+    const long long t0 = clock64(), budget = wait_budget();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (clock64() - t0 > budget) {
+            record_error(status, kStatusTimeout);
+            if (abort_flag) *abort_flag = 1;
+            return false;
+        }
+        if ((it & 63u) == 0) {  // the flags live in memory: polled at a lower rate
             if (abort_flag && *abort_flag) return false;
             if (global_failed(status)) {
-                if (abort_flag) *abort_flag = 1;
-                return false;
-            }
-            if (clock64() - t0 > kWaitBudgetCycles) {
-                record_error(status, kStatusTimeout);
                 if (abort_flag) *abort_flag = 1;
                 return false;
             }
@@ -124,14 +144,21 @@ SLA_DEV bool elect_one()
     return pred != 0;
 }
 
-// Bounded wait used only on failure paths, to let copies or MMAs already in
-// flight retire before a CTA releases its shared memory / TMEM.  Ignores the
-// abort flags; gives up after ~50 ms.
-SLA_DEV bool mbar_wait_quiet(uint64_t *bar, uint32_t parity)
+// Bounded wait used on exit paths, to let copies or MMAs already in flight
+// retire before a CTA releases its shared memory / TMEM.  Ignores the abort
+// flags and the run-time override: it always allows the full default budget
+// (~0.5 s), far beyond the latency of any copy or MMA.  If even that runs out
+// the status word records SLA_ERR_TIMEOUT (the call's results are void) and
+// the CTA still releases its TMEM: a CTA that exited holding TMEM would stall
+// every later CTA's allocation on that SM.
+SLA_DEV bool mbar_wait_quiet(uint64_t *bar, uint32_t parity, int *status = nullptr)
 {
-    long long t0 = clock64();
+    const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitBudgetCycles / 10) return false;
+        if (clock64() - t0 > kWaitBudgetCycles) {
+            if (status) record_error(status, kStatusTimeout);
+            return false;
+        }
     return true;
 }
 

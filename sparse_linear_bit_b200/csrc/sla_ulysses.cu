@@ -1,6 +1,6 @@
 // sla_ulysses.cu -- layout permutations around the Ulysses all-to-all.
 //
-// Ulysses context parallelism (the "TurboDiffusion" GitHub summary, 主要特点:
+// Ulysses context parallelism (the "TurboDiffusion" summary page, 主要能力:
 // the training code supports Ulysses CP) keeps, on each of P ranks, a
 // contiguous range of n_local = N / P tokens of every head.  Attention needs
 // every token of a head, so one all-to-all turns [B, H, n_local, d] (tokens of

@@ -1,8 +1,9 @@
 // sla_w8a8.cu -- W8A8 INT8 linear layer with FusedNorm on tcgen05 tensor cores.
 //
-// "清华开源TurboDiffusion加速框架" (W8A8 section) and the "TurboDiffusion" GitHub
-// summary (主要特点 3): the linear layers' weights and activations are quantised
-// to 8-bit integers and run on the INT8 units, with a FusedNorm operator.  The
+// "清华开源TurboDiffusion加速框架" (W8A8 INT8量化) and "TurboDiffusion：让可视化视频
+// 生成效率提升200倍的加速引擎" (§1): the linear layers' weights and activations
+// are quantised to 8-bit integers and run on the INT8 units, with a FusedNorm
+// operator.  The
 // granularity, rounding and norm are not stated; what is implemented:
 //
 //  rowquant_kernel  per row of a bf16 matrix [rows, cols]: optionally the RMS
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(kGmThreads, 1) w8a8_gemm_kernel(const __grid_c
             for (int s = 0; s < kGmStages; ++s) {
                 int jl = -1;
                 for (int j = s; j < kc; j += kGmStages) jl = j;
-                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kGmStages) & 1);
+                if (jl >= 0) mbar_wait_quiet(&sm.full[s], (jl / kGmStages) & 1, status);
             }
         }
         __syncwarp();
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(kGmThreads, 1) w8a8_gemm_kernel(const __grid_c
         }
         if (elect_one()) {
             mma_commit(&sm.drain);
-            mbar_wait_quiet(&sm.drain, 0);  // MMAs retired before TMEM is freed
+            mbar_wait_quiet(&sm.drain, 0, status);  // MMAs retired before TMEM is freed
         }
         __syncwarp();
     } else {
@@ -390,6 +391,10 @@ cudaError_t launch_w8a8_gemm(const int8_t *qx, const float *sx, const int8_t *qw
 namespace {
 bool al(const void *p, uintptr_t a) { return p != nullptr && ((uintptr_t)p & (a - 1)) == 0; }
 }  // namespace
+
+namespace sla {
+cudaError_t set_wait_budget_w8a8(long long cycles) { return set_tu_wait_budget(cycles); }
+}  // namespace sla
 
 extern "C" {
 

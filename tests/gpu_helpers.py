@@ -49,3 +49,21 @@ def mask_mismatches(idx_gpu: np.ndarray, idx_orc: np.ndarray, scores: np.ndarray
         ok = all(abs(row[J] - thr) <= max(rel * max(abs(row[J]), abs(thr)), floor) for J in (a ^ b))
         (exempt if ok else real).append(r)
     return exempt, real
+
+
+_INPUT_CACHE: dict = {}
+
+
+def workload_qkv(name: str, adversarial=(), seed_offset: int = 0):
+    """(q, k, v) of a named workload from synth.WORKLOADS (bf16 bits), generated once per
+    test process and shared by the test modules; at most the two most recent input sets
+    are kept (a 720P set is 2.3 GB of host memory)."""
+    import synth
+
+    key = (name, tuple(adversarial), seed_offset)
+    if key not in _INPUT_CACHE:
+        while len(_INPUT_CACHE) >= 2:
+            _INPUT_CACHE.pop(next(iter(_INPUT_CACHE)))
+        w = synth.WORKLOADS[name]
+        _INPUT_CACHE[key] = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed + seed_offset, adversarial=adversarial)
+    return _INPUT_CACHE[key]

@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_helpers import rel_l2, to_dev
+from gpu_helpers import rel_l2, to_dev, workload_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -80,8 +80,8 @@ def test_backward_full_size_scaling():
     doubling dout doubles every fp32 operation exactly, so the results must be
     exactly twice those for dout; all finite."""
     w = synth.WORKLOADS["wan14b-720p"]
-    q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
-    dout = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed + 1)[0]
+    q, k, v = workload_qkv("wan14b-720p")
+    dout = workload_qkv("wan14b-720p", seed_offset=1)[0]
     qd, kd, vd, dod = (to_dev(x, torch) for x in (q, k, v, dout))
     del q, k, v, dout
     B, H, N, d = qd.shape
@@ -103,8 +103,8 @@ def test_backward_full_size_sampled_dq():
     of 3 heads against the oracle, which computes them row by row.  An fp64 emulation of the
     kernel's bf16 roundings (dS, and P inside D = do.os) on such rows predicts about 2.2e-3."""
     w = synth.WORKLOADS["wan14b-720p"]
-    q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
-    dout = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed + 1)[0]
+    q, k, v = workload_qkv("wan14b-720p")
+    dout = workload_qkv("wan14b-720p", seed_offset=1)[0]
     dq, dk, dv = run_backward(q, k, v, dout, w.blk_q, 0.1, 0)
     del dk, dv
     rows = synth.sample_rows(w.B, w.H, w.N, n_heads=3, rows_per_head=48)

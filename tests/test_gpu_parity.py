@@ -6,8 +6,8 @@
 * INT8 quantisation: codes, scales and the smoothing mean bit-exact;
 * forward: cosine >= 0.999 and relative L2 <= 2e-2 with quantisation on,
   relative L2 <= 2e-3 with it off, over small workloads that span several
-  tiles with ragged tails, phi in {elu+1, relu}, topk in {0, 0.1, ..., 1},
-  and on sampled rows of the full-size 720P workload;
+  tiles with ragged tails, phi in {elu+1, relu}, topk in {0, 0.1, ..., 1}
+  (the workloads at their full sizes are in test_gpu_configs.py);
 * determinism: two calls give identical bytes.
 """
 from __future__ import annotations
@@ -283,19 +283,3 @@ def test_state_reduction_mask_bits(name):
     expect = sel if 2 * ks <= n_kb else 1 - sel
     assert np.array_equal(bits[..., :n_kb], expect)
     assert not bits[..., n_kb:].any()
-
-
-@pytest.mark.parametrize("topk", [0.1])
-def test_forward_full_size_sampled(topk):
-    """14B-720P shape (B=1, H=40, N=75600) in the benchmark's launch
-    configuration; sampled rows of 3 heads checked against the oracle."""
-    w = synth.WORKLOADS["wan14b-720p"]
-    q, k, v = synth.make_qkv(w.B, w.H, w.grid, seed=w.seed)
-    out, _ = run_forward(q, k, v, w.blk_q, w.blk_k, topk, 0, 1)
-    rows = synth.sample_rows(w.B, w.H, w.N, n_heads=3, rows_per_head=48)
-    got_all = bf16_to_f64(out).reshape(w.B * w.H, w.N, 128)
-    got = got_all[rows[:, 0], rows[:, 1]]
-    ref = oracle.forward(q, k, v, w.blk_q, w.blk_k, f32(topk), phi=0, quant=1, rows=rows)
-    r, c = rel_l2(got, ref), cosine(got, ref)
-    assert r <= QUANT_TOL["rel"] and c >= QUANT_TOL["cos"], (r, c)
-    assert np.isfinite(got_all).all()
