@@ -1,5 +1,5 @@
 // sla_attention.cu -- fused block-sparse attention + linear epilogue of the
-// SageSLA forward (one CTA per (batch*head, query block)).
+// SageSLA forward: one CTA per (batch*head, query block), two CTAs per SM.
 //
 // Sparse branch: exact softmax attention softmax(q k^T / sqrt(d)) v
 // ("TurboDiffusion技术架构解析" §2.1, standard attention formula) over the tokens
@@ -11,39 +11,37 @@
 // quantisation off, Q.K^T runs in bf16 and P.V in fp16 (P and an fp16 copy of
 // V, 8x finer rounding than bf16), both with fp32 accumulation.
 //
-// Linear branch epilogue: phi(Q_I) H_I as a tf32 MMA into its own TMEM
-// accumulator, normalised by phi(q) . Z_I on the CUDA cores; output =
-// sparse + linear, rounded to bf16.
+// Linear branch ("TurboDiffusion技术架构解析" §2.1, linear attention
+// phi(Q)(phi(K)^T V)): after the sparse loop the row's normaliser phi(q) . Z_I
+// is computed on the CUDA cores, and A = phi(q) * l / (phi(q) . Z_I) (l: the
+// row's softmax sum) is written to tensor memory in tf32, so that one tf32 MMA
+// O += A H_I leaves O / l = O_sparse + O_linear in the same accumulator.
 //
-// Tiling.  Key blocks are processed in selection order, loaded two per ring
-// stage.  Two softmax warpgroups take one block each (warpgroup g: blocks
-// 2t+g) with their own S (one M=128, N=64 Q.K^T chain per block), P, O
-// accumulator and running (max, sum), merged in the epilogue; the groups share
-// nothing but Q, the ring and the exponential token, so one group's Q.K^T is
-// issued while the other group is still reading its logits.  The two
-// warps that share an SM sub-partition (same query rows, one per group) pass a
-// token so that their exponential phases alternate: the MUFU unit is the
-// scarcest resource, and one group's exponentials overlap the other group's
-// TMEM loads, row maxima and stores.
+// Tiling.  One softmax warpgroup takes the query block's selected key blocks
+// in selection order, one M=128, N=64 Q.K^T per block, with its S, P, O and
+// running (max, sum) in tensor memory and registers.  Two such CTAs share an
+// SM (256 TMEM columns and ~99 KB of shared memory each), so one CTA's
+// prologue (Q codes, first K/V tiles) and epilogue (linear branch, output
+// store) overlap the other CTA's main loop, and their exponential phases
+// interleave on the MUFU units.
 //
 // Issue.  tcgen05 and mbarrier operations cost tens of cycles each on the
-// issuing thread, so each softmax group has its own issuing thread for its
-// Q.K^T and P.V.  Dependencies go through mbarriers only: S of a group is
-// rewritten once that group has read it; P of a group is rewritten once that
-// group's previous P.V has completed.
+// issuing thread, so a dedicated warp issues the Q.K^T and P.V MMAs.
+// Dependencies go through mbarriers only: S is rewritten once it has been
+// read; P is rewritten once the previous P.V has completed.
 //
 // Shared-memory bandwidth (128 B/clk, shared by TMA writes and tensor-core
-// operand reads): both A operands live in tensor memory -- Q (written once per
-// CTA from registers) and P (packed two 16-bit values per 32-bit column) -- so
-// per key block only K and V cross shared memory, through a ring of four
-// pair-stages.  The linear branch runs at the end, reusing the ring for its
-// operands and the S columns for its accumulator.
+// operand reads): the A operands of the quantised modes live in tensor memory
+// -- Q (written once per CTA from registers) and P (two 16-bit values per
+// 32-bit column) -- so per key block only K and V cross shared memory, through
+// a ring of four stages (two without quantisation, whose bf16 Q tile stays in
+// shared memory as the Q.K^T A operand).  The linear branch runs at the end,
+// reusing the ring for H_I and the raw Q rows.
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 linear-branch issuer and
-// TMEM owner, warps 2-5 / 6-9 softmax groups 0 / 1 (one query row per thread,
-// one TMEM lane quarter per warp), warps 10 / 11 Q.K^T + P.V issuers of groups
-// 0 / 1.  TMEM columns: S of group g at 64g (L over both at the end), P of
-// group g at 128 + 32g, Q at 192, O of group g at 256 + 128g.
+// Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 2-5 softmax and epilogue (one query row per thread, one TMEM lane
+// quarter per warp).  TMEM columns: S at 0, P at 64, Q codes at 96, O at 128;
+// the linear branch's A operand takes columns 0-127 at the end.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -57,32 +55,31 @@
 namespace sla {
 namespace {
 
-constexpr int kAttnThreads = 384;
+constexpr int kAttnThreads = 192;
+constexpr uint32_t kAttnTmemCols = 256;
 constexpr uint32_t kBox = 64 * 128;          // [64 rows x 128 B]
 constexpr uint32_t kQRowsBox = 128 * 128;    // [128 rows x 128 B]
+constexpr uint32_t kRegion = 6 * kQRowsBox;  // 96 KB: the K/V ring, then H_I (64 KB) + raw Q rows (32 KB)
+constexpr uint32_t kQRawOff = 4 * kQRowsBox; // raw Q rows (and the bf16 Q tile without quantisation)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: P may grow to 2^8 before O is rescaled
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1 / sqrt(128)
 
 template <bool QUANT>  // QUANT: 8-bit Q/K codes (INT8 or FP8)
 struct AttnCfg {
-    static constexpr uint32_t kKBytes = QUANT ? 2 * kBox : 4 * kBox;        // K of a pair of key blocks
-    static constexpr uint32_t kVBytes = 4 * kBox;                           // V of a pair of key blocks
+    static constexpr uint32_t kKBytes = QUANT ? kBox : 2 * kBox;  // K of one key block (int8, or two bf16 boxes)
+    static constexpr uint32_t kVBytes = 2 * kBox;                 // V of one key block: dims 0-63, 64-127
     static constexpr uint32_t kStageBytes = kKBytes + kVBytes;
-    static constexpr int kStages = QUANT ? 4 : 3;
-    static constexpr uint32_t kLinBytes = 10 * kQRowsBox;  // H_I 64 KB + phi(Q) 64 KB + raw Q 32 KB
-    static constexpr uint32_t kRegion = (kStages * kStageBytes > kLinBytes) ? kStages * kStageBytes : kLinBytes;
+    static constexpr int kStages = QUANT ? 4 : 2;
+    // quantised: the ring fills the region; otherwise it ends where the bf16 Q tile begins
+    static_assert(kStages * kStageBytes <= (QUANT ? kRegion : kQRawOff), "ring fits");
 };
 
-template <bool QUANT>
 struct AttnSmem {
-    alignas(1024) uint8_t region[AttnCfg<QUANT>::kRegion];  // K/V ring, then the linear operands
+    alignas(1024) uint8_t region[kRegion];
     float z[kD];
-    float fin[2][3][128];   // epilogue exchange: [group][max, sum, den]
-    uint64_t bar_q, bar_h, bar_qr, bar_phiq, bar_lin, drain[3];
-    uint64_t full[AttnCfg<QUANT>::kStages], empty[AttnCfg<QUANT>::kStages];
-    uint64_t bar_s[2], bar_sfree[2], bar_p[2], bar_pv[2];
-    uint64_t tok[2][4];     // exponential-phase token per group and lane quarter
+    uint64_t full[4], empty[4];
+    uint64_t bar_q, bar_s, bar_sfree, bar_p, bar_pv, bar_h, bar_qr, bar_phiq, bar_lin, drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -92,15 +89,6 @@ SLA_DEV float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// phi of one Q element, rounded to tf32 for the linear branch's MMA.  exp(x) for
-// x <= 0 is ex2(x log2 e) on the MUFU unit (the result is rounded to 10 mantissa
-// bits next).
-SLA_DEV float phi_tf32(float x, int phi)
-{
-    const float e = ex2(fminf(x, 0.0f) * kLog2e);  // unconditional, so both cases are a select
-    return to_tf32(phi == 1 ? fmaxf(x, 0.0f) : (x > 0.0f ? x + 1.0f : e));
 }
 
 SLA_DEV void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -182,16 +170,39 @@ SLA_DEV void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, ui
         : "memory");
 }
 
+
 // descriptor + byte offset (the start-address field is the low 14 bits, in 16 B units)
 SLA_DEV uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
+// tf32 MMA with A in tensor memory (rows = lanes, one 32-bit K element per column)
+SLA_DEV void mma_tf32_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc_, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc_), "r"(accumulate)
+        : "memory");
+}
+
+// phi of the 8 bf16 channels of one 16-byte unit of a raw Q row (fp32, not rounded)
+SLA_DEV void phi8(const uint4 &w, int phi, float (&f)[8])
+{
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float lo = __uint_as_float(ww[e] << 16), hi = __uint_as_float(ww[e] & 0xFFFF0000u);
+        const float elo = ex2(fminf(lo, 0.0f) * kLog2e), ehi = ex2(fminf(hi, 0.0f) * kLog2e);
+        f[2 * e] = phi == 1 ? fmaxf(lo, 0.0f) : (lo > 0.0f ? lo + 1.0f : elo);
+        f[2 * e + 1] = phi == 1 ? fmaxf(hi, 0.0f) : (hi > 0.0f ? hi + 1.0f : ehi);
+    }
+}
 
 // MODE 0: bf16 Q.K^T, fp16 P.V; 1: INT8 Q.K^T (int32 logits); 2: FP8 e4m3 Q.K^T (fp32
 // logits); P.V in bf16 for both quantised modes.
 template <int MODE>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kAttnThreads, 2)
 attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
             const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_qr,
-            const uint16_t *__restrict__ qraw,
             const int8_t *__restrict__ q8, const float *__restrict__ qscale, const float *__restrict__ kscale,
             const int32_t *__restrict__ idx, const float *__restrict__ hq, int N, int blk_q, int n_qb, int n_kb,
             int k_sel, int phi, uint16_t *__restrict__ out, int *status)
@@ -200,54 +211,48 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     using Cfg = AttnCfg<QUANT>;
     constexpr int NS = Cfg::kStages;
     extern __shared__ uint8_t smem_raw[];
-    AttnSmem<QUANT> &sm =
-        *reinterpret_cast<AttnSmem<QUANT> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    AttnSmem &sm = *reinterpret_cast<AttnSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int I = blockIdx.x, bh = blockIdx.y;
     const int32_t *sel = idx + ((size_t)bh * n_qb + I) * k_sel;
-    const int n_tiles = (k_sel + 1) >> 1;
-    auto n_blk = [&](int g) { return (k_sel + 1 - g) >> 1; };  // blocks of softmax group g
     volatile int *abort_flag = &sm.abort_flag;
     if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
     __syncthreads();
     if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
 
     if (tid == 0) {
-        mbar_init(&sm.bar_q, 256);
+        mbar_init(&sm.bar_q, QUANT ? 128 : 1);  // codes stored by the 128 softmax threads / the Q tile's TMA
+        mbar_init(&sm.bar_s, 1);
+        mbar_init(&sm.bar_sfree, 128);
+        mbar_init(&sm.bar_p, 128);
+        mbar_init(&sm.bar_pv, 1);
         mbar_init(&sm.bar_h, 1);
         mbar_init(&sm.bar_qr, 1);
-        mbar_init(&sm.bar_phiq, 256);
+        mbar_init(&sm.bar_phiq, 128);
         mbar_init(&sm.bar_lin, 1);
-        for (int d = 0; d < 3; ++d) mbar_init(&sm.drain[d], 1);
+        mbar_init(&sm.drain, 1);
         for (int s = 0; s < NS; ++s) {
             mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 2);  // one commit from each P.V issuer per tile
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.bar_s[b], 1);
-            mbar_init(&sm.bar_sfree[b], 128);
-            mbar_init(&sm.bar_p[b], 128);
-            mbar_init(&sm.bar_pv[b], 1);
-            for (int q = 0; q < 4; ++q) mbar_init(&sm.tok[b][q], 1);
+            mbar_init(&sm.empty[s], 1);
         }
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, 512);
+        tmem_alloc(&sm.tmem_base, kAttnTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t t_s = tmem, t_p = tmem + 128, t_q = tmem + 192, t_o = tmem + 256, t_l = tmem;
-    uint8_t *h_s = sm.region;                       // end: 4 x [128 dims x 32 fp32]
-    uint8_t *phiq_s = sm.region + 4 * kQRowsBox;    // end: 4 x [128 rows x 32 fp32]
-    uint8_t *qraw_s = sm.region + 8 * kQRowsBox;    // end: 2 x [128 rows x 64 bf16] (raw Q for phi)
+    // S at 0 (64 columns), P at 64 (32), Q codes at 96 (32), O at 128 (128); at the end the
+    // linear branch's A operand (128 tf32 columns) replaces S, P and Q
+    const uint32_t t_s = tmem, t_p = tmem + 64, t_q = tmem + 96, t_a = tmem, t_o = tmem + 128;
+    uint8_t *h_s = sm.region;                       // end: H_I, 4 x [128 dims x 32 fp32]
+    uint8_t *qraw_s = sm.region + kQRawOff;         // raw Q rows, 2 x [128 rows x 64 bf16]
 
-    // Issuing warps (producer, linear branch, Q.K^T + P.V of each group) run their
-    // loops with all 32 lanes, so that stage offsets and descriptors are
-    // warp-uniform, and elect one lane for each TMA / tcgen05 instruction.
+    // Issuing warps (producer, MMA issuer) run their loops with all 32 lanes, so that stage
+    // offsets and descriptors are warp-uniform, and elect one lane for each TMA / tcgen05 instruction.
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (elect_one()) {
@@ -255,49 +260,53 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_h);
             tma_prefetch_desc(&tm_qr);
-            // the linear epilogue's operands (H_I, raw Q rows) into L2 now, so that their loads
-            // at the end of the CTA do not wait on HBM
+            // the linear epilogue's operands into L2 now, so that their loads at the end do not wait on HBM
             for (int c = 0; c < 4; ++c) tma_prefetch_l2_3d(&tm_h, 32 * c, 0, bh * n_qb + I);
-            for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_qr, 64 * c, I * blk_q, bh);
+            if (QUANT) {
+                for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_qr, 64 * c, I * blk_q, bh);
+            } else {  // the bf16 Q tile: A operand of Q.K^T, and the raw Q of phi at the end
+                mbar_expect_tx(&sm.bar_q, 2 * kQRowsBox);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_q, 64 * c, I * blk_q, bh);
+            }
         }
+        __syncwarp();
         int issued = 0;
         bool ok = true;
-        for (int t = 0; ok && t < n_tiles; ++t) {
+        for (int t = 0; ok && t < k_sel; ++t) {
             const int s = t % NS, u = t / NS;
             if (u > 0 && !(ok = mbar_wait_warp(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
-            const int nb = min(2, k_sel - 2 * t);
             uint8_t *st = sm.region + s * Cfg::kStageBytes;
-            const int J0 = __ldg(sel + 2 * t), J1 = nb > 1 ? __ldg(sel + 2 * t + 1) : 0;
+            const int J = __ldg(sel + t);
             if (elect_one()) {
-                mbar_expect_tx(&sm.full[s], (uint32_t)nb * Cfg::kStageBytes / 2);
-                for (int x = 0; x < nb; ++x) {
-                    const int J = x ? J1 : J0;
-                    // K: rows 64x..64x+63 of the pair (one 128-channel int8 box, or two 64-channel bf16 boxes)
-                    tma_load_3d(st + x * kBox, &tm_k, &sm.full[s], 0, J * 64, bh);
-                    if (!QUANT) tma_load_3d(st + 2 * kBox + x * kBox, &tm_k, &sm.full[s], 64, J * 64, bh);
-                    // V: dims 0-63 then dims 64-127, each [128 keys x 128 B] for the pair
-                    tma_load_3d(st + Cfg::kKBytes + x * kBox, &tm_v, &sm.full[s], 0, J * 64, bh);
-                    tma_load_3d(st + Cfg::kKBytes + 2 * kBox + x * kBox, &tm_v, &sm.full[s], 64, J * 64, bh);
-                }
+                mbar_expect_tx(&sm.full[s], Cfg::kStageBytes);
+                // K: one 128-channel int8 box, or two 64-channel bf16 boxes; V: dims 0-63, then 64-127
+                tma_load_3d(st, &tm_k, &sm.full[s], 0, J * 64, bh);
+                if (!QUANT) tma_load_3d(st + kBox, &tm_k, &sm.full[s], 64, J * 64, bh);
+                tma_load_3d(st + Cfg::kKBytes, &tm_v, &sm.full[s], 0, J * 64, bh);
+                tma_load_3d(st + Cfg::kKBytes + kBox, &tm_v, &sm.full[s], 64, J * 64, bh);
             }
             __syncwarp();
             issued = t + 1;
         }
-        // H_I and the raw Q rows into the region once every stage is retired
+        // H_I (and, quantised, the raw Q rows) into the ring once every stage is retired
         for (int s = 0; ok && s < NS; ++s) {
             int tl = -1;
-            for (int t = s; t < n_tiles; t += NS) tl = t;
+            for (int t = s; t < k_sel; t += NS) tl = t;
             if (tl >= 0) ok = mbar_wait_warp(&sm.empty[s], (tl / NS) & 1, status, abort_flag);
         }
         if (ok && elect_one()) {
             mbar_expect_tx(&sm.bar_h, 4 * kQRowsBox);
             for (int c = 0; c < 4; ++c) tma_load_3d(h_s + c * kQRowsBox, &tm_h, &sm.bar_h, 32 * c, 0, bh * n_qb + I);
-            mbar_expect_tx(&sm.bar_qr, 2 * kQRowsBox);
-            for (int c = 0; c < 2; ++c)
-                tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_qr, 64 * c, I * blk_q, bh);
+            if (QUANT) {
+                mbar_expect_tx(&sm.bar_qr, 2 * kQRowsBox);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_qr, 64 * c, I * blk_q, bh);
+            }
         }
         __syncwarp();
-        if (!ok) {  // failure: let loads in flight land before shared memory is released
+        // before shared memory is released: every load issued has landed
+        if (!ok) {
             for (int s = 0; s < NS; ++s) {
                 int tl = -1;
                 for (int t = s; t < issued; t += NS) tl = t;
@@ -305,100 +314,88 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             }
         } else {
             mbar_wait_quiet(&sm.bar_h, 0, status);
-            mbar_wait_quiet(&sm.bar_qr, 0, status);
+            if (QUANT) mbar_wait_quiet(&sm.bar_qr, 0, status);
         }
+        if (!QUANT) mbar_wait_quiet(&sm.bar_q, 0, status);
     } else if (warp == 1) {
-        // ------------------------------------------------------------ linear-branch MMA
-        // L = phi(Q_I) H_I (tf32) into the S columns, after the softmax groups are done
-        bool ok = mbar_wait_warp(&sm.bar_h, 0, status, abort_flag);
-        if (ok) ok = mbar_wait_warp(&sm.bar_phiq, 0, status, abort_flag);
-        if (ok) {
-            tc_fence_after();
-            constexpr uint32_t id_lin = idesc(1, 2, 2, 0, 0, 128, 128);  // f32 <- tf32 x tf32, K-major
-            const uint64_t pd = sdesc_sw128(smem_u32(phiq_s), 16, 1024), hd = sdesc_sw128(smem_u32(h_s), 16, 1024);
-            if (elect_one()) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const uint32_t off = (k >> 2) * kQRowsBox + (k & 3) * 32;
-                    mma_tf32(t_l, dadd(pd, off), dadd(hd, off), id_lin, k > 0 ? 1u : 0u);
-                }
-                mma_commit(&sm.bar_lin);
-            }
-            __syncwarp();
-        }
-        if (elect_one()) {
-            mma_commit(&sm.drain[0]);
-            mbar_wait_quiet(&sm.drain[0], 0, status);  // this thread's MMAs retired before TMEM is released
-        }
-        __syncwarp();
-    } else if (warp >= 10) {
-        // ------------------------------------------------------------ Q.K^T + P.V issuer of group g
-        const int g = warp - 10;
+        // ------------------------------------------------------------ MMA issuer
         // S32 <- s8 x s8 (INT8), F32 <- e4m3 x e4m3 (FP8), F32 <- bf16 x bf16
         constexpr uint32_t id_qk = MODE == 1   ? idesc(2, 1, 1, 0, 0, 128, 64)
                                    : MODE == 2 ? idesc(1, 0, 0, 0, 0, 128, 64)
                                                : idesc(1, 1, 1, 0, 0, 128, 64);
         constexpr uint32_t id_pv = QUANT ? idesc(1, 1, 1, 0, 1, 128, 128) : idesc(1, 0, 0, 0, 1, 128, 128);
+        constexpr uint32_t id_lin = idesc(1, 2, 2, 0, 0, 128, 128);  // f32 <- tf32 x tf32, K-major
         const uint64_t kd0 = sdesc_sw128(smem_u32(sm.region), 16, 1024);
-        const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), 2 * kBox, 1024);
-        const uint32_t s_g = t_s + 64 * g, o_g = t_o + 128 * g, p_g = t_p + 32 * g;
-        const int nb = n_blk(g);
+        const uint64_t vd0 = sdesc_sw128(smem_u32(sm.region + Cfg::kKBytes), kBox, 1024);
+        const uint64_t qd0 = sdesc_sw128(smem_u32(qraw_s), 16, 1024);  // the bf16 Q tile (quantisation off)
         bool ok = true;
-        // S_g = Q K_j^T for this group's block of tile t (K rows of block g of the pair)
+        // S = Q K_J^T for key block t of the selection
         auto issue_qk = [&](int t) {
             if (!(ok = mbar_wait_warp(&sm.full[t % NS], (t / NS) & 1, status, abort_flag))) return;
-            if (t > 0 && !(ok = mbar_wait_warp(&sm.bar_sfree[g], (t - 1) & 1, status, abort_flag))) return;
+            if (t > 0 && !(ok = mbar_wait_warp(&sm.bar_sfree, (t - 1) & 1, status, abort_flag))) return;
             tc_fence_after();
-            const uint64_t kd = dadd(kd0, (t % NS) * Cfg::kStageBytes + g * kBox);
+            const uint64_t kd = dadd(kd0, (t % NS) * Cfg::kStageBytes);
             if (elect_one()) {
                 if (MODE == 1) {  // K-step of 32 int8 = 8 TMEM columns of Q
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(s_g, t_q + 8 * k, kd + 2 * k, id_qk, k > 0 ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k) mma_i8_tmem_a(t_s, t_q + 8 * k, dadd(kd, 32 * k), id_qk, k > 0 ? 1u : 0u);
                 } else if (MODE == 2) {  // K-step of 32 e4m3 = 8 TMEM columns of Q
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_f8_tmem_a(s_g, t_q + 8 * k, kd + 2 * k, id_qk, k > 0 ? 1u : 0u);
-                } else {  // K-step of 16 bf16 = 8 TMEM columns of Q
+                    for (int k = 0; k < 4; ++k) mma_f8_tmem_a(t_s, t_q + 8 * k, dadd(kd, 32 * k), id_qk, k > 0 ? 1u : 0u);
+                } else {  // K-step of 16 bf16: 32 bytes of a 64-channel box
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_f16_tmem_a(s_g, t_q + 8 * k, kd + (k >> 2) * (2 * kBox >> 4) + 2 * (k & 3), id_qk,
-                                       k > 0 ? 1u : 0u);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * kQRowsBox + (k & 3) * 32, koff = (k >> 2) * kBox + (k & 3) * 32;
+                        mma_bf16(t_s, dadd(qd0, off), dadd(kd, koff), id_qk, k > 0 ? 1u : 0u);
+                    }
                 }
-                mma_commit(&sm.bar_s[g]);
+                mma_commit(&sm.bar_s);
             }
             __syncwarp();
         };
-        if (nb > 0) {
+        if (k_sel > 0) {
             ok = mbar_wait_warp(&sm.bar_q, 0, status, abort_flag);
             if (ok) issue_qk(0);
         }
-        for (int t = 0; ok && t < n_tiles; ++t) {
-            if (t < nb) {
-                if (t + 1 < nb) {  // next logits as soon as this group has read S
-                    issue_qk(t + 1);
-                    if (!ok) break;
-                }
-                if (!(ok = mbar_wait_warp(&sm.bar_p[g], t & 1, status, abort_flag))) break;
-                tc_fence_after();
-                const uint64_t vd = dadd(vd0, (t % NS) * Cfg::kStageBytes + g * kBox);  // this block's rows
-                if (elect_one()) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_f16_tmem_a(o_g, p_g + 8 * k, vd + 128 * k, id_pv, (t > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&sm.bar_pv[g]);
-                }
-                __syncwarp();
+        for (int t = 0; ok && t < k_sel; ++t) {
+            if (t + 1 < k_sel) {  // next logits as soon as S has been read
+                issue_qk(t + 1);
+                if (!ok) break;
             }
-            if (elect_one()) mma_commit(&sm.empty[t % NS]);  // stage t free once both groups' MMAs retired
+            if (!(ok = mbar_wait_warp(&sm.bar_p, t & 1, status, abort_flag))) break;
+            tc_fence_after();
+            const uint64_t vd = dadd(vd0, (t % NS) * Cfg::kStageBytes);
+            if (elect_one()) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // K-step of 16 keys = 8 TMEM columns of P, 2 KB of V rows
+                    mma_f16_tmem_a(t_o, t_p + 8 * k, dadd(vd, 2048 * k), id_pv, (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_pv);
+                mma_commit(&sm.empty[t % NS]);  // the stage is free once Q.K^T and P.V of block t retired
+            }
+            __syncwarp();
+        }
+        // linear branch: O += A H_I, A = phi(Q) scaled per row (tf32, TMEM columns 0-127)
+        if (ok) ok = mbar_wait_warp(&sm.bar_h, 0, status, abort_flag);
+        if (ok) ok = mbar_wait_warp(&sm.bar_phiq, 0, status, abort_flag);
+        if (ok) {
+            tc_fence_after();
+            const uint64_t hd = sdesc_sw128(smem_u32(h_s), 16, 1024);
+            if (elect_one()) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k)  // K-step of 8 tf32 channels: 32 bytes of a 32-channel box
+                    mma_tf32_tmem_a(t_o, t_a + 8 * k, dadd(hd, (k >> 2) * kQRowsBox + (k & 3) * 32), id_lin,
+                                    (k > 0 || k_sel > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_lin);
+            }
             __syncwarp();
         }
         if (elect_one()) {
-            mma_commit(&sm.drain[1 + g]);
-            mbar_wait_quiet(&sm.drain[1 + g], 0, status);
+            mma_commit(&sm.drain);
+            mbar_wait_quiet(&sm.drain, 0, status);  // this thread's MMAs retired before TMEM is released
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax / epilogue
-        const int g = (warp - 2) >> 2;                  // group: key blocks 2t + g
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;              // query row within the tile (= TMEM lane)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -410,72 +407,57 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const bool w = mbar_wait(bar, par, status, abort_flag);
             return __all_sync(0xffffffffu, w);
         };
-        if (g == 0) sm.z[r] = __ldg(hq + ((size_t)bh * n_qb + I) * kStateCols + kD * kD + r);
-        // Q (INT8 codes, or bf16 without quantisation) into tensor memory: row r -> lane r, four
-        // int8 (two bf16) per 32-bit column; group g writes its half of the columns
-        if (k_sel > 0) {
-            const bool qrow = i < N;  // rows of the next block (blk_q = 64) or past N: anything finite
-            if (QUANT) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(q8 + ((size_t)bh * N + (qrow ? i : 0)) * kD) + 4 * g;
-                uint32_t w[16];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint4 x = qrow ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
-                    w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
-                }
-                tmem_st16(t_q + lane_off + 16 * g, w);
-            } else {
-                const uint4 *src = reinterpret_cast<const uint4 *>(qraw + ((size_t)bh * N + (qrow ? i : 0)) * kD) + 8 * g;
+        sm.z[r] = __ldg(hq + ((size_t)bh * n_qb + I) * kStateCols + kD * kD + r);
+        if (QUANT) {
+            // Q codes into tensor memory: row r -> lane r, four codes per 32-bit column
+            if (k_sel > 0) {
+                const bool qrow = i < N;  // rows of the next block (blk_q = 64) or past N: anything finite
+                const uint4 *src = reinterpret_cast<const uint4 *>(q8 + ((size_t)bh * N + (qrow ? i : 0)) * kD);
                 uint32_t w[32];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const uint4 x = qrow ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
                     w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
                 }
-                tmem_st32(t_q + lane_off + 32 * g, w);
+                tmem_st32(t_q + lane_off, w);
+                tmem_wait_st();
             }
-            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_q);
         }
-        tc_fence_before();
-        mbar_arrive(&sm.bar_q);
-        if (g == 1) {  // group 0 takes the first exponential phase
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.tok[0][quarter]);
-        }
+        named_bar_sync(1, 128);  // z is visible to every softmax thread
 
-        // ---- sparse loop: this group's key blocks j = 2t + g
+        // ---- sparse loop over the selected key blocks, in selection order
         const float sq = QUANT ? __ldg(qscale + (size_t)bh * n_qb + I) : 0.0f;
         const float kscale_log2 = kLog2e * kInvSqrtD;
         constexpr float kBias = 12582912.0f;  // 1.5 * 2^23: int32 d + bias bits read as float 12582912 + d
-        const uint32_t s_own = t_s + 64 * g + lane_off, p_own = t_p + 32 * g + lane_off;
-        const uint32_t o_own = t_o + 128 * g + lane_off;
-        // per-tile block index and key scale, prefetched ahead of use
-        auto blk_of = [&](int t) { return (2 * t + g < k_sel) ? __ldg(sel + 2 * t + g) : -1; };
+        const uint32_t s_own = t_s + lane_off, p_own = t_p + lane_off, o_own = t_o + lane_off;
+        // block index and key scale of the next blocks, prefetched ahead of use
+        auto blk_of = [&](int t) { return t < k_sel ? __ldg(sel + t) : -1; };
         int J_a = blk_of(0), J_b = blk_of(1);
         float ks_a = (QUANT && J_a >= 0) ? __ldg(kscale + (size_t)bh * n_kb + J_a) : 0.0f;
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
-        const int nb = n_blk(g);
         // Phase tests are issued ahead of use (see mbar_test); a negative answer
         // falls back to the bounded wait.
         bool s_ready = false;
-        for (int t = 0; ok && t < nb; ++t) {
+        for (int t = 0; ok && t < k_sel; ++t) {
             const int J = J_a;
             const float c = QUANT ? sq * ks_a * kscale_log2 : kscale_log2;
-            if (t + 1 < nb) {
+            if (t + 1 < k_sel) {
                 J_a = J_b;
                 if (QUANT) ks_a = __ldg(kscale + (size_t)bh * n_kb + J_b);
             }
-            if (t + 2 < nb) J_b = blk_of(t + 2);
-            if (!__all_sync(0xffffffffu, s_ready) && !(ok = wait_all(&sm.bar_s[g], t & 1))) break;
+            if (t + 2 < k_sel) J_b = blk_of(t + 2);
+            if (!__all_sync(0xffffffffu, s_ready) && !(ok = wait_all(&sm.bar_s, t & 1))) break;
             tc_fence_after();
             uint32_t sv[64];
             tmem_ld32(s_own, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
             tmem_ld32(s_own + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&sm.bar_sfree[g]);  // S_g may be rewritten now
-            const bool tok_ready = mbar_test(&sm.tok[g][quarter], t & 1);
+            mbar_arrive(&sm.bar_sfree);  // S may be rewritten now
+            const bool pv_ready = t == 0 || mbar_test(&sm.bar_pv, (t - 1) & 1);
             const int valid = min(64, N - J * 64);
             // the two paths are separate instantiations so the full-tile path carries no masking
             const float tmax = valid == 64 ? tile_max<INT_S, false>(sv, 64, c) : tile_max<INT_S, true>(sv, valid, c);
@@ -487,18 +469,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
                 m_used = m_new;
                 l *= alpha;
             }
-            // exponential phase, alternating with the other group's warp on this sub-partition
-            if (!__all_sync(0xffffffffu, tok_ready) && !(ok = wait_all(&sm.tok[g][quarter], t & 1))) break;
-            const bool pv_ready = t == 0 || mbar_test(&sm.bar_pv[g], (t - 1) & 1);
             uint32_t pk[32];
             const float off = INT_S ? -fmaf(kBias, c, m_used) : -m_used;
             if (valid == 64) l += tile_exp<QUANT, false>(sv, 64, c, off, pk);
             else l += tile_exp<QUANT, true>(sv, valid, c, off, pk);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.tok[g ^ 1][quarter]);
-            // P and O of this group are free/stable once its previous P.V has retired
-            if (!__all_sync(0xffffffffu, pv_ready) && !(ok = wait_all(&sm.bar_pv[g], (t - 1) & 1))) break;
-            if (t > 0 && __any_sync(0xffffffffu, need)) {  // rescale O of this group
+            // P and O are free/stable once the previous P.V has retired
+            if (!__all_sync(0xffffffffu, pv_ready) && !(ok = wait_all(&sm.bar_pv, (t - 1) & 1))) break;
+            if (t > 0 && __any_sync(0xffffffffu, need)) {  // rescale O
                 tc_fence_after();
                 uint32_t o[32];
 #pragma unroll 1
@@ -513,76 +490,59 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tmem_st32(p_own, pk);  // P packed to bf16 (fp16 without quantisation)
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&sm.bar_p[g]);
-            if (t + 1 < nb) s_ready = mbar_test(&sm.bar_s[g], (t + 1) & 1);
+            mbar_arrive(&sm.bar_p);
+            if (t + 1 < k_sel) s_ready = mbar_test(&sm.bar_s, (t + 1) & 1);
         }
-        // ---- linear branch operands: wait for every P.V (the ring is then free), then phi(Q) + den
-        if (ok && n_blk(0) > 0) ok = wait_all(&sm.bar_pv[0], (n_blk(0) - 1) & 1);
-        if (ok && n_blk(1) > 0) ok = wait_all(&sm.bar_pv[1], (n_blk(1) - 1) & 1);
-        named_bar_sync(5, 256);  // every group past its P.V waits (z is also visible now)
-        float den = 0.0f;
-        if (ok) ok = wait_all(&sm.bar_qr, 0);  // raw Q rows of this tile (rows past N read as 0)
+
+        // ---- linear branch: A = phi(q) * l / (phi(q) . Z_I) in tf32, so that the MMA O += A H_I
+        // leaves O / l = O_sparse + O_linear
+        if (ok && k_sel > 0) ok = wait_all(&sm.bar_pv, (k_sel - 1) & 1);  // P and S columns are free
+        if (ok) ok = wait_all(QUANT ? &sm.bar_qr : &sm.bar_q, 0);         // raw Q rows (past N: zeros)
+        const float l_eff = k_sel > 0 ? l : 1.0f;  // no sparse blocks: O is the linear MMA's alone
         if (ok) {
+            float den = 0.0f;
 #pragma unroll 2
-            for (int uu = 0; uu < 8; ++uu) {  // group g: channels 64g..64g+63, 8 per iteration
-                const int u = 8 * g + uu;
-                const uint4 w = *reinterpret_cast<const uint4 *>(qraw_s + g * kQRowsBox + sw128_off(r, uu));
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            for (int u = 0; u < 16; ++u) {  // channels 8u..8u+7
+                const uint4 w = *reinterpret_cast<const uint4 *>(qraw_s + (u >> 3) * kQRowsBox + sw128_off(r, u & 7));
                 float f[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    f[2 * e] = row_valid ? phi_tf32(__uint_as_float(ww[e] << 16), phi) : 0.0f;
-                    f[2 * e + 1] = row_valid ? phi_tf32(__uint_as_float(ww[e] & 0xFFFF0000u), phi) : 0.0f;
-                }
+                phi8(w, phi, f);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) den = fmaf(f[e], sm.z[8 * u + e], den);
-                // channels 8u..8u+7 = chunk (u/4), 16-byte units (2u)%8 and (2u+1)%8 of row r
-                uint8_t *base = phiq_s + (u >> 2) * kQRowsBox;
-                *reinterpret_cast<float4 *>(base + sw128_off(r, (2 * u) & 7)) = make_float4(f[0], f[1], f[2], f[3]);
-                *reinterpret_cast<float4 *>(base + sw128_off(r, (2 * u + 1) & 7)) = make_float4(f[4], f[5], f[6], f[7]);
             }
-            fence_async_smem();
+            const float scale = (row_valid && den != 0.0f) ? __fdiv_rn(l_eff, den) : 0.0f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t a[32];
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) {
+                    const int u = (c0 >> 3) + uu;
+                    const uint4 w =
+                        *reinterpret_cast<const uint4 *>(qraw_s + (u >> 3) * kQRowsBox + sw128_off(r, u & 7));
+                    float f[8];
+                    phi8(w, phi, f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a[8 * uu + e] = __float_as_uint(to_tf32(f[e] * scale));
+                }
+                tmem_st32(t_a + lane_off + c0, a);
+            }
+            tmem_wait_st();
         }
+        tc_fence_before();
         mbar_arrive(&sm.bar_phiq);
-        // ---- epilogue: merge the two groups' partial softmax; group g writes output columns 64g..64g+63
-        sm.fin[g][0][r] = m_used;
-        sm.fin[g][1][r] = l;
-        sm.fin[g][2][r] = den;
-        named_bar_sync(5, 256);
         if (ok) ok = wait_all(&sm.bar_lin, 0);
         if (ok) {
             tc_fence_after();
-            const int n0 = n_blk(0), n1 = n_blk(1);
-            const float m0 = sm.fin[0][0][r], l0 = sm.fin[0][1][r], m1 = sm.fin[1][0][r], l1 = sm.fin[1][1][r];
-            const float m = fmaxf(m0, m1);
-            const float s0 = n0 > 0 ? ex2(m0 - m) : 0.0f, s1 = n1 > 0 ? ex2(m1 - m) : 0.0f;
-            const float lt = l0 * s0 + l1 * s1;
-            const float inv_l = lt > 0.0f ? 1.0f / lt : 0.0f;
-            const float w0 = s0 * inv_l, w1 = s1 * inv_l;
-            const float dt = sm.fin[0][2][r] + sm.fin[1][2][r];
-            const float inv_den = dt != 0.0f ? 1.0f / dt : 0.0f;
-            uint16_t *orow = out + ((size_t)bh * N + (row_valid ? i : 0)) * kD + 64 * g;
-            const uint32_t o0 = t_o + lane_off + 64 * g, o1 = t_o + 128 + lane_off + 64 * g;
+            const float inv_l = l_eff > 0.0f ? 1.0f / l_eff : 0.0f;
+            uint16_t *orow = out + ((size_t)bh * N + (row_valid ? i : 0)) * kD;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                uint32_t lr[32], a0[32], a1[32];
-                tmem_ld32(t_l + lane_off + 64 * g + c0, lr);
-                if (n0 > 0) tmem_ld32(o0 + c0, a0);
-                if (n1 > 0) tmem_ld32(o1 + c0, a1);
+            for (int c0 = 0; c0 < kD; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(o_own + c0, o);
                 tmem_wait_ld();
                 uint32_t pkk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float v[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float x = __uint_as_float(lr[2 * e + h]) * inv_den;
-                        if (n0 > 0) x = fmaf(__uint_as_float(a0[2 * e + h]), w0, x);
-                        if (n1 > 0) x = fmaf(__uint_as_float(a1[2 * e + h]), w1, x);
-                        v[h] = x;
-                    }
-                    pkk[e] = pack_bf16x2(v[0], v[1]);
-                }
+                for (int e = 0; e < 16; ++e)
+                    pkk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
                 if (row_valid) {
                     uint4 *o4 = reinterpret_cast<uint4 *>(orow + c0);
 #pragma unroll
@@ -597,7 +557,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
     __syncwarp();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kAttnTmemCols);
     }
 }
 
@@ -631,18 +591,18 @@ cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int
         if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, hd, st, bh)) return cudaErrorInvalidValue;
     }
     {
-        // raw Q rows of a query block for phi(Q): [BH, N, 128] bf16, boxes of 64 channels x 128 rows
+        // raw Q rows of a query block: [BH, N, 128] bf16, boxes of 64 channels x 128 rows
         const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
         const uint32_t bq[3] = {64, 128, 1};
         if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, st, bq)) return cudaErrorInvalidValue;
     }
-    const size_t smem = sizeof(AttnSmem<QUANT>) + 1024;
+    const size_t smem = sizeof(AttnSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(g.n_qb, g.BH);
-    attn_kernel<MODE><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, tq, static_cast<const uint16_t *>(q), q8, qscale,
-                                                        kscale, idx, hq, g.N, g.blk_q, g.n_qb, g.n_kb, g.k_sel, phi,
-                                                        static_cast<uint16_t *>(out), status);
+    attn_kernel<MODE><<<grid, kAttnThreads, smem, s>>>(tk, tv, th, tq, q8, qscale, kscale, idx, hq, g.N, g.blk_q,
+                                                        g.n_qb, g.n_kb, g.k_sel, phi, static_cast<uint16_t *>(out),
+                                                        status);
     return cudaGetLastError();
 }
 
