@@ -20,6 +20,8 @@ Parity status of each function (what pins it is in tests/test_oracle_pins.py):
   library routine; topk=0 equals closed-form linear attention; an independent
   attention-form brute force with a dense token mask; constant-V identity;
   convex-hull bounds; a hand-worked golden case).
+* ``backward_dq_rows``, ``backward_dkdv_blocks`` -- pinned (equal, bit for bit,
+  to the corresponding rows of ``backward``).
 * ``backward``  -- pinned (float64 autograd of an independent PyTorch
   statement of the unquantised forward, whose values are checked against
   ``forward``; topk=1 against the gradient of a library attention routine;
@@ -80,6 +82,8 @@ def load(path: Optional[str] = None):
     lib.orc_backward.restype = i32
     lib.orc_backward_dq_rows.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, P, P, i64, P]
     lib.orc_backward_dq_rows.restype = i32
+    lib.orc_backward_dkdv_blocks.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, P, P, i64, P, P]
+    lib.orc_backward_dkdv_blocks.restype = i32
     if path is None:
         _lib = lib
     return lib
@@ -258,6 +262,26 @@ def backward_dq_rows(q, k, v, dout, blk_q: int, blk_k: int, topk: float, rows, p
     if rc != 0:
         raise MemoryError("oracle backward_dq_rows failed (out of memory or bad row index)")
     return out
+
+
+def backward_dkdv_blocks(q, k, v, dout, blk_q: int, blk_k: int, topk: float, blocks, phi: int = 0,
+                         idx: Optional[np.ndarray] = None, lib=None):
+    """fp64 dk and dv of the key blocks ``blocks`` (int64 [n, 2] of (bh, J)) only: the
+    same steps, in the same order, as ``backward`` restricted to those blocks.
+    Returns ``(dk, dv)``, each ``[n, blk_k, d]`` (rows past N are zero)."""
+    lib = lib or load()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    BH, N, d = _shape(q)
+    blocks = np.ascontiguousarray(blocks, dtype=np.int64).reshape(-1, 2)
+    dk = np.zeros((blocks.shape[0], blk_k, d), dtype=np.float64)
+    dv = np.zeros((blocks.shape[0], blk_k, d), dtype=np.float64)
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    rc = lib.orc_backward_dkdv_blocks(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), BH, N, d, blk_q, blk_k, float(topk),
+                                      int(phi), _ptr(idx), _ptr(blocks), blocks.shape[0], _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise MemoryError("oracle backward_dkdv_blocks failed (out of memory or bad block index)")
+    return dk, dv
 
 
 # --------------------------------------------------------------------------

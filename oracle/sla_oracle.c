@@ -824,6 +824,201 @@ int orc_backward_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return fail ? -1 : 0;
 }
 
+/* dk and dv of a list of key blocks only (blocks: [nblk][2] pairs (bh, J);
+ * dk_out, dv_out: [nblk][blk_k][d], rows past N left zero): the same steps,
+ * in the same order, as the full backward restricted to those key blocks, so
+ * that they can be evaluated at sizes where the full backward is too slow.
+ * A key block's gradient needs (a) the linear branch's state gradients dH_I,
+ * dZ_I of every query block that did not select it, and (b) for every row of
+ * every query block that did select it, the row's softmax over all its
+ * selected tokens and D = do.os.  Each contribution is added to dk, dv in the
+ * order the full backward adds it (query blocks ascending, rows ascending,
+ * then the linear key side), so the results equal orc_backward's rows bit for
+ * bit.  idx_in as in orc_backward.  Returns 0, or -1 when memory runs out or a
+ * block is out of range. */
+int orc_backward_dkdv_blocks(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                             int BH, int N, int d, int blk_q, int blk_k, double topk, int phi,
+                             const int32_t *idx_in, const int64_t *blocks, int64_t nblk, double *dk_out,
+                             double *dv_out)
+{
+    int n_qb = (N + blk_q - 1) / blk_q, n_kb = (N + blk_k - 1) / blk_k;
+    int k_sel = orc_topk_count(n_kb, topk);
+    const double rsd = 1.0 / sqrt((double)d);
+    size_t hd = (size_t)N * d, dd = (size_t)d * d;
+    for (int64_t b = 0; b < nblk; ++b)
+        if (blocks[2 * b] < 0 || blocks[2 * b] >= BH || blocks[2 * b + 1] < 0 || blocks[2 * b + 1] >= n_kb) return -1;
+    memset(dk_out, 0, sizeof(double) * (size_t)nblk * blk_k * d);
+    memset(dv_out, 0, sizeof(double) * (size_t)nblk * blk_k * d);
+    int fail = 0;
+    for (int bh = 0; bh < BH && !fail; ++bh) {
+        int any = 0;
+        for (int64_t b = 0; b < nblk; ++b) any |= blocks[2 * b] == bh;
+        if (!any) continue;
+        const uint16_t *qh = q + bh * hd, *kh = k + bh * hd, *vh = v + bh * hd, *dh = dout + bh * hd;
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * ((size_t)n_qb * k_sel + 1));
+        double *h = (double *)malloc(sizeof(double) * (size_t)n_kb * dd);
+        double *z = (double *)malloc(sizeof(double) * (size_t)n_kb * d);
+        double *dH = (double *)calloc((size_t)n_qb * dd, sizeof(double));
+        double *dZ = (double *)calloc((size_t)n_qb * d, sizeof(double));
+        double *G = (double *)malloc(sizeof(double) * dd);
+        double *gz = (double *)malloc(sizeof(double) * (size_t)d);
+        unsigned char *selected = (unsigned char *)calloc((size_t)n_qb * n_kb + 1, 1);
+        /* per selecting row: p_ij and ds_ij of the block's keys (blk_k each) */
+        double *pr = (double *)malloc(sizeof(double) * ((size_t)n_qb * blk_q * blk_k + 1));
+        double *dsr = (double *)malloc(sizeof(double) * ((size_t)n_qb * blk_q * blk_k + 1));
+        if (!idx || !h || !z || !dH || !dZ || !G || !gz || !selected || !pr || !dsr) {
+            free(idx); free(h); free(z); free(dH); free(dZ); free(G); free(gz); free(selected); free(pr); free(dsr);
+            fail = 1;
+            break;
+        }
+        if (idx_in)
+            memcpy(idx, idx_in + (size_t)bh * n_qb * k_sel, sizeof(int32_t) * (size_t)n_qb * k_sel);
+        else
+            mask_head(qh, kh, N, d, blk_q, blk_k, k_sel, idx, NULL, NULL);
+        states_head(kh, vh, N, d, blk_k, phi, h, z);
+        for (int I = 0; I < n_qb; ++I)
+            for (int r = 0; r < k_sel; ++r) selected[(size_t)I * n_kb + idx[(size_t)I * k_sel + r]] = 1;
+        /* (a) the linear branch's state gradients of every query block, as in the full backward */
+#pragma omp parallel
+        {
+            double *HI = (double *)malloc(sizeof(double) * dd);
+            double *ZI = (double *)malloc(sizeof(double) * (size_t)d);
+            double *vec = (double *)malloc(sizeof(double) * 8 * (size_t)d);
+#pragma omp for schedule(dynamic)
+            for (int I = 0; I < n_qb; ++I) {
+                if (!HI || !ZI || !vec) continue;
+                unselected_state(idx + (size_t)I * k_sel, k_sel, n_kb, d, h, z, HI, ZI);
+                double *dHI = dH + (size_t)I * dd, *dZI = dZ + (size_t)I * d;
+                double *qi = vec, *doi = vec + d, *f = vec + 3 * d, *a = vec + 4 * d, *ol = vec + 5 * d,
+                       *da = vec + 6 * d;
+                int i1 = (I + 1) * blk_q < N ? (I + 1) * blk_q : N;
+                for (int i = I * blk_q; i < i1; ++i) {
+                    for (int c = 0; c < d; ++c) {
+                        qi[c] = bf(qh[(size_t)i * d + c]);
+                        doi[c] = bf(dh[(size_t)i * d + c]);
+                    }
+                    double b = 0.0;
+                    for (int c = 0; c < d; ++c) {
+                        f[c] = phi_f(qi[c], phi);
+                        b += f[c] * ZI[c];
+                    }
+                    if (b == 0.0) continue;
+                    for (int e = 0; e < d; ++e) {
+                        a[e] = 0.0;
+                        for (int c = 0; c < d; ++c) a[e] += f[c] * HI[(size_t)c * d + e];
+                        ol[e] = a[e] / b;
+                    }
+                    double dol = 0.0;
+                    for (int e = 0; e < d; ++e) dol += doi[e] * ol[e];
+                    double db = -dol / b;
+                    for (int e = 0; e < d; ++e) da[e] = doi[e] / b;
+                    for (int c = 0; c < d; ++c) {
+                        for (int e = 0; e < d; ++e) dHI[(size_t)c * d + e] += f[c] * da[e];
+                        dZI[c] += f[c] * db;
+                    }
+                }
+            }
+            free(HI); free(ZI); free(vec);
+        }
+        for (int64_t bb = 0; bb < nblk; ++bb) {
+            if (blocks[2 * bb] != bh) continue;
+            int J = (int)blocks[2 * bb + 1], t0 = J * blk_k, t1 = t0 + blk_k < N ? t0 + blk_k : N;
+            double *dkb = dk_out + (size_t)bb * blk_k * d, *dvb = dv_out + (size_t)bb * blk_k * d;
+            /* (b) the softmax branch: every row of every query block that selected J, p and ds of
+             * J's keys (rows evaluated in parallel, added in order below) */
+#pragma omp parallel
+            {
+                double *p = (double *)malloc(sizeof(double) * ((size_t)k_sel * blk_k + 1));
+                double *vec = (double *)malloc(sizeof(double) * 3 * (size_t)d);
+#pragma omp for schedule(dynamic)
+                for (int I = 0; I < n_qb; ++I) {
+                    if (!p || !vec || !selected[(size_t)I * n_kb + J]) continue;
+                    const int32_t *sel = idx + (size_t)I * k_sel;
+                    double *qi = vec, *doi = vec + d, *os = vec + 2 * d;
+                    int i1 = (I + 1) * blk_q < N ? (I + 1) * blk_q : N;
+                    for (int i = I * blk_q; i < i1; ++i) {
+                        for (int c = 0; c < d; ++c) {
+                            qi[c] = bf(qh[(size_t)i * d + c]);
+                            doi[c] = bf(dh[(size_t)i * d + c]);
+                        }
+                        int nk = 0, at = -1;
+                        double mx = -INFINITY;
+                        for (int r = 0; r < k_sel; ++r) {
+                            int Jr = sel[r], u0 = Jr * blk_k, u1 = u0 + blk_k < N ? u0 + blk_k : N;
+                            if (Jr == J) at = nk;
+                            for (int j = u0; j < u1; ++j) {
+                                double sc = 0.0;
+                                for (int c = 0; c < d; ++c) sc += qi[c] * bf(kh[(size_t)j * d + c]);
+                                p[nk] = sc * rsd;
+                                if (p[nk] > mx) mx = p[nk];
+                                ++nk;
+                            }
+                        }
+                        double den = 0.0;
+                        for (int n = 0; n < nk; ++n) {
+                            p[n] = exp(p[n] - mx);
+                            den += p[n];
+                        }
+                        for (int n = 0; n < nk; ++n) p[n] /= den;
+                        for (int e = 0; e < d; ++e) os[e] = 0.0;
+                        int n = 0;
+                        for (int r = 0; r < k_sel; ++r) {
+                            int Jr = sel[r], u0 = Jr * blk_k, u1 = u0 + blk_k < N ? u0 + blk_k : N;
+                            for (int j = u0; j < u1; ++j, ++n)
+                                for (int e = 0; e < d; ++e) os[e] += p[n] * bf(vh[(size_t)j * d + e]);
+                        }
+                        double D = 0.0;
+                        for (int e = 0; e < d; ++e) D += doi[e] * os[e];
+                        double *prow = pr + ((size_t)I * blk_q + (i - I * blk_q)) * blk_k;
+                        double *dsrow = dsr + ((size_t)I * blk_q + (i - I * blk_q)) * blk_k;
+                        for (int j = t0; j < t1; ++j) {
+                            double dp = 0.0;
+                            for (int e = 0; e < d; ++e) dp += doi[e] * bf(vh[(size_t)j * d + e]);
+                            prow[j - t0] = p[at + (j - t0)];
+                            dsrow[j - t0] = p[at + (j - t0)] * (dp - D);
+                        }
+                    }
+                }
+                free(p); free(vec);
+            }
+            for (int I = 0; I < n_qb; ++I) {
+                if (!selected[(size_t)I * n_kb + J]) continue;
+                int i1 = (I + 1) * blk_q < N ? (I + 1) * blk_q : N;
+                for (int i = I * blk_q; i < i1; ++i) {
+                    const double *prow = pr + ((size_t)I * blk_q + (i - I * blk_q)) * blk_k;
+                    const double *dsrow = dsr + ((size_t)I * blk_q + (i - I * blk_q)) * blk_k;
+                    for (int j = t0; j < t1; ++j)
+                        for (int c = 0; c < d; ++c) {
+                            dkb[(size_t)(j - t0) * d + c] += dsrow[j - t0] * bf(qh[(size_t)i * d + c]) * rsd;
+                            dvb[(size_t)(j - t0) * d + c] += prow[j - t0] * bf(dh[(size_t)i * d + c]);
+                        }
+                }
+            }
+            /* the linear key side */
+            memset(G, 0, sizeof(double) * dd);
+            memset(gz, 0, sizeof(double) * (size_t)d);
+            for (int I = 0; I < n_qb; ++I) {
+                if (selected[(size_t)I * n_kb + J]) continue;
+                for (size_t e = 0; e < dd; ++e) G[e] += dH[(size_t)I * dd + e];
+                for (int c = 0; c < d; ++c) gz[c] += dZ[(size_t)I * d + c];
+            }
+            for (int j = t0; j < t1; ++j) {
+                for (int c = 0; c < d; ++c) {
+                    double kc = bf(kh[(size_t)j * d + c]), fk = phi_f(kc, phi);
+                    double dfk = gz[c];
+                    for (int e = 0; e < d; ++e) {
+                        dfk += G[(size_t)c * d + e] * bf(vh[(size_t)j * d + e]);
+                        dvb[(size_t)(j - t0) * d + e] += G[(size_t)c * d + e] * fk;
+                    }
+                    dkb[(size_t)(j - t0) * d + c] += dfk * dphi_f(kc, phi);
+                }
+            }
+        }
+        free(idx); free(h); free(z); free(dH); free(dZ); free(G); free(gz); free(selected); free(pr); free(dsr);
+    }
+    return fail ? -1 : 0;
+}
+
 /* ------------------------------------------------------------------------
  * W8A8 INT8 linear layer with FusedNorm ("清华开源TurboDiffusion加速框架",
  * W8A8 INT8量化: the weights and activations of the linear layers quantised

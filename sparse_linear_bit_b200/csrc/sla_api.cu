@@ -365,7 +365,7 @@ sla_status sla_set_wait_budget(long long cycles)
 {
     if (cycles < 0) return SLA_ERR_INVALID_ARG;
     if (set_wait_budget_attention(cycles) != cudaSuccess || set_wait_budget_linear(cycles) != cudaSuccess ||
-        set_wait_budget_w8a8(cycles) != cudaSuccess)
+        set_wait_budget_w8a8(cycles) != cudaSuccess || set_wait_budget_bwd(cycles) != cudaSuccess)
         return SLA_ERR_CUDA;
     return SLA_OK;
 }

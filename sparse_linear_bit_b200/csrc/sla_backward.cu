@@ -18,23 +18,23 @@
 // Launch sequence (all on one stream):
 //   1. the forward's block means, scores, top-k, key-block states and
 //      per-query-block states H_I, Z_I (the forward's own kernels, quantisation
-//      off);
-//   2. bwd_query_kernel, one CTA per (head, query block): online-softmax
-//      recompute of p and os over the selected blocks, the row statistics
-//      (max, sum, D = do.os) for step 5, dq of both branches, and dH_I, dZ_I
-//      (fp32 and a bf16 copy);
-//   3. the column sum of dH_I over the query blocks (for the subtract form) and
+//      off), and the head's mean key mu (for the dq of the softmax branch);
+//   2. the softmax branch's query side on the tensor cores (bwdq_kernel,
+//      sla_bwd_sparse.cu): the row statistics (max, sum, D = do.os) and its dq;
+//   3. bwd_qlin_kernel, one CTA per (head, query block): the linear branch's
+//      dq (added), and dH_I, dZ_I (fp32 and a bf16 copy);
+//   4. the column sum of dH_I over the query blocks (for the subtract form) and
 //      the transposed selection bits (key block J -> query blocks I);
-//   4. G = A^T dH on the tensor cores: the forward's state-reduction kernel on
+//   5. G = A^T dH on the tensor cores: the forward's state-reduction kernel on
 //      the transposed mask (same subtract / complement rule);
-//   5. bwd_key_kernel, one CTA per (head, key block): the linear key side from
-//      G_J, then dk, dv of the sparse branch over the query blocks that
-//      selected J (no atomics: each CTA owns its key block's rows).
+//   6. bwd_klin_kernel, one CTA per (head, key block): the linear key side from
+//      G_J, written to dk, dv;
+//   7. the softmax branch's key side on the tensor cores (bwdk_kernel): its dk,
+//      dv over the query blocks that selected the key block, added.
 //
-// The per-tile products of the sparse branch (Q.K^T, P.V, dO.V^T, dS.K,
-// P^T dO, dS^T Q) run on the tensor cores as warp-level bf16 MMAs with fp32
-// accumulation; P and dS enter them rounded to bf16.  The linear branch's
-// d x d products run in fp32 on the CUDA cores.  Results are fp32.
+// The softmax branch's per-tile products run as tcgen05 MMAs with bf16
+// operands (P and dS rounded to bf16) and fp32 accumulation; the linear
+// branch's d x d products run in fp32 on the CUDA cores.  Results are fp32.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,7 +50,6 @@ namespace {
 
 constexpr int kBwdThreads = 256;
 constexpr int kRS = 68;          // 32-bit words per shared row of 128 bf16 (16-byte rows, conflict-free fragments)
-constexpr int kRS64 = 36;        // 32-bit words per shared row of 64 bf16
 constexpr int kGW = 129;         // floats per shared row of a 128 x 128 state tile
 constexpr float kRsd = 0.08838834764831845f;  // 1 / sqrt(128)
 
@@ -102,67 +101,6 @@ __device__ __forceinline__ void load_tile(uint32_t *t, uint32_t *tt, int rs_t, c
     }
 }
 
-// ---- warp-level bf16 tensor-core products (mma.sync m16n8k16, fp32 accumulation).  Fragments are
-// read from "k-major" shared tiles (row = the M or N index, two consecutive K elements per word).
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// A fragment: rows m0..m0+15, K columns k0..k0+15
-__device__ __forceinline__ void frag_a(const uint32_t *t, int rs, int m0, int k0, uint32_t (&a)[4])
-{
-    const int lane = threadIdx.x & 31;
-    const uint32_t *p = t + (m0 + (lane >> 2)) * rs + (k0 >> 1) + (lane & 3);
-    a[0] = p[0];
-    a[1] = p[8 * rs];
-    a[2] = p[4];
-    a[3] = p[8 * rs + 4];
-}
-
-// acc[nt] (n-tile nt: N columns n0 + 8 nt ..) += A(m0.., 0..K) * B(0..K, n0 + 8 nt ..), B stored [n][k]
-template <int NT>
-__device__ __forceinline__ void warp_gemm(float (&acc)[NT][4], const uint32_t *ta, int rsa, int m0,
-                                          const uint32_t *tb, int rsb, int n0, int K)
-{
-    const int lane = threadIdx.x & 31;
-    const uint32_t *pb = tb + (n0 + (lane >> 2)) * rsb + (lane & 3);
-    for (int k0 = 0; k0 < K; k0 += 16) {
-        uint32_t a[4];
-        frag_a(ta, rsa, m0, k0, a);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint32_t *q = pb + 8 * nt * rsb + (k0 >> 1);
-            mma16816(acc[nt], a, q[0], q[4]);
-        }
-    }
-}
-
-// acc[nt] += P * B for P held as the fp32 accumulators of an m16 x n64 product (8 n-tiles), used as the
-// A operand over K = 64 (the accumulator layout of two n-tiles is the A layout of one k-step)
-template <int NT>
-__device__ __forceinline__ void warp_gemm_regs(float (&acc)[NT][4], const float (&p)[8][4], const uint32_t *tb,
-                                               int rsb, int n0)
-{
-    const int lane = threadIdx.x & 31;
-    const uint32_t *pb = tb + (n0 + (lane >> 2)) * rsb + (lane & 3);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t a[4] = {pack_bf16(p[2 * kk][0], p[2 * kk][1]), pack_bf16(p[2 * kk][2], p[2 * kk][3]),
-                               pack_bf16(p[2 * kk + 1][0], p[2 * kk + 1][1]),
-                               pack_bf16(p[2 * kk + 1][2], p[2 * kk + 1][3])};
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint32_t *q = pb + 8 * nt * rsb + 8 * kk;
-            mma16816(acc[nt], a, q[0], q[4]);
-        }
-    }
-}
-
 // acc[i][j] += sum_k A(ty + 16 i, k) * B(k, tx + 16 j) over k < K, with ty = tid / 16, tx = tid % 16
 // (fp32 on the CUDA cores: the linear branch's d x d products)
 template <int TM, int TN, class FA, class FB>
@@ -183,174 +121,43 @@ __device__ __forceinline__ void gemm_acc(float (&acc)[TM][TN], int K, FA A, FB B
     }
 }
 
-// reductions over the 16 threads (tx) that share a row group (a half warp), and over a quad
+// sum over the 16 threads (tx) that share a row group (a half warp)
 __device__ __forceinline__ float hw_sum(float x)
 {
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
     return x;
 }
-__device__ __forceinline__ float quad_max(float x)
-{
-    x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
-    return fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
-}
-__device__ __forceinline__ float quad_sum(float x)
-{
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    return x + __shfl_xor_sync(0xffffffffu, x, 2);
-}
 
-struct QuerySmem {
+struct QlinSmem {
     uint32_t q[128 * kRS];    // Q rows of the query block
     uint32_t dO[128 * kRS];   // dO rows
-    // key-block tiles; the linear part reuses this region for H_I^T (128 x kGW floats)
-    uint32_t k[64 * kRS];     // K rows (B of Q.K^T)
-    uint32_t kt[128 * kRS64]; // K^T (B of dS.K)
-    uint32_t v[64 * kRS];     // V rows (B of dO.V^T)
-    uint32_t vt[128 * kRS64]; // V^T (B of P.V)
+    float ht[128 * kGW];      // H_I^T
     float z[128], binv[128], db[128];
 };
-static_assert(sizeof(uint32_t) * (2 * 64 * kRS + 2 * 128 * kRS64) >= sizeof(float) * 128 * kGW,
-              "H_I^T fits in the key-block region");
 
 // ---------------------------------------------------------------------------
-// step 2: one CTA per (head, query block); warp w owns query rows 16w..16w+15 of the
-// sparse products (rows g and g+8 of each fragment: r0, r1)
+// step 3: the linear branch's query side, one CTA per (head, query block): dq += (H_I da + Z_I db)
+// phi'(q) (dq holds the softmax branch's part), and dH_I, dZ_I for the key side
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBwdThreads, 1)
-bwd_query_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
-                 const uint16_t *__restrict__ dout, const int32_t *__restrict__ idx, const float *__restrict__ hq,
-                 int N, int blk_q, int n_qb, int k_sel, int phi, float *__restrict__ dq, float *__restrict__ st_m,
-                 float *__restrict__ st_l, float *__restrict__ st_D, float *__restrict__ dh32,
-                 uint16_t *__restrict__ dh16)
+bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dout, const float *__restrict__ hq,
+                int N, int blk_q, int n_qb, int phi, float *__restrict__ dq, float *__restrict__ dh32,
+                uint16_t *__restrict__ dh16)
 {
     extern __shared__ uint8_t smem_raw[];
-    QuerySmem &sm = *reinterpret_cast<QuerySmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+    QlinSmem &sm = *reinterpret_cast<QlinSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    const int warp = tid >> 5, lane = tid & 31, tq = lane & 3;
-    const int r0 = 16 * warp + (lane >> 2), r1 = r0 + 8;
     const int I = blockIdx.x, bh = blockIdx.y;
     const int i0 = I * blk_q, rows = min(blk_q, N - i0);  // valid rows of this query block
     const size_t head = (size_t)bh * N * 128;
-    const int32_t *sel = idx + ((size_t)bh * n_qb + I) * k_sel;
-
     load_tile(sm.q, nullptr, 0, q + head, i0, rows, 128);
     load_tile(sm.dO, nullptr, 0, dout + head, i0, rows, 128);
-
-    // ---- sparse branch, pass 1: online softmax, os = sum p v, row statistics
-    float O[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.0f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
-    for (int r = 0; r < k_sel; ++r) {
-        const int t0 = __ldg(sel + r) * 64, kv = min(64, N - t0);
-        __syncthreads();
-        load_tile(sm.k, nullptr, 0, k + head, t0, kv, 64);
-        load_tile(sm.v, sm.vt, kRS64, v + head, t0, kv, 64);
-        __syncthreads();
-        float s[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
-        warp_gemm<8>(s, sm.q, kRS, 16 * warp, sm.k, kRS, 0, 128);
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const bool ok = 8 * n + 2 * tq + h < kv;
-                s[n][h] = ok ? s[n][h] * kRsd : -INFINITY;
-                s[n][2 + h] = ok ? s[n][2 + h] * kRsd : -INFINITY;
-                mx0 = fmaxf(mx0, s[n][h]);
-                mx1 = fmaxf(mx1, s[n][2 + h]);
-            }
-        const float mn0 = fmaxf(m0, quad_max(mx0)), mn1 = fmaxf(m1, quad_max(mx1));
-        const float al0 = __expf(m0 - mn0), al1 = __expf(m1 - mn1);  // 0 while m = -inf
-        float sum0 = 0.0f, sum1 = 0.0f;
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                s[n][h] = __expf(s[n][h] - mn0);
-                s[n][2 + h] = __expf(s[n][2 + h] - mn1);
-                sum0 += s[n][h];
-                sum1 += s[n][2 + h];
-            }
-        l0 = l0 * al0 + quad_sum(sum0);
-        l1 = l1 * al1 + quad_sum(sum1);
-        m0 = mn0;
-        m1 = mn1;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            O[n][0] *= al0; O[n][1] *= al0;
-            O[n][2] *= al1; O[n][3] *= al1;
-        }
-        warp_gemm_regs<16>(O, s, sm.vt, kRS64, 0);  // O += P V
-    }
-    const float il0 = l0 > 0.0f ? 1.0f / l0 : 0.0f, il1 = l1 > 0.0f ? 1.0f / l1 : 0.0f;
-    float D0 = 0.0f, D1 = 0.0f;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const uint32_t w0 = sm.dO[r0 * kRS + 4 * n + tq], w1 = sm.dO[r1 * kRS + 4 * n + tq];
-        D0 += bf_lo(w0) * O[n][0] + bf_hi(w0) * O[n][1];
-        D1 += bf_lo(w1) * O[n][2] + bf_hi(w1) * O[n][3];
-    }
-    D0 = quad_sum(D0) * il0;
-    D1 = quad_sum(D1) * il1;
-    if (tq == 0) {
-        if (r0 < rows) {
-            st_m[(size_t)bh * N + i0 + r0] = m0;
-            st_l[(size_t)bh * N + i0 + r0] = il0;
-            st_D[(size_t)bh * N + i0 + r0] = D0;
-        }
-        if (r1 < rows) {
-            st_m[(size_t)bh * N + i0 + r1] = m1;
-            st_l[(size_t)bh * N + i0 + r1] = il1;
-            st_D[(size_t)bh * N + i0 + r1] = D1;
-        }
-    }
-
-    // ---- sparse branch, pass 2: dq = sum_j p (do.v_j - D) k_j / sqrt(d)
-    float dQ[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) dQ[n][0] = dQ[n][1] = dQ[n][2] = dQ[n][3] = 0.0f;
-    for (int r = 0; r < k_sel; ++r) {
-        const int t0 = __ldg(sel + r) * 64, kv = min(64, N - t0);
-        __syncthreads();
-        load_tile(sm.k, sm.kt, kRS64, k + head, t0, kv, 64);
-        load_tile(sm.v, nullptr, 0, v + head, t0, kv, 64);
-        __syncthreads();
-        float s[8][4], dp[8][4];
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.0f;
-        warp_gemm<8>(s, sm.q, kRS, 16 * warp, sm.k, kRS, 0, 128);
-        warp_gemm<8>(dp, sm.dO, kRS, 16 * warp, sm.v, kRS, 0, 128);
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const bool ok = 8 * n + 2 * tq + h < kv;
-                const float p0 = ok ? __expf(s[n][h] * kRsd - m0) * il0 : 0.0f;
-                const float p1 = ok ? __expf(s[n][2 + h] * kRsd - m1) * il1 : 0.0f;
-                s[n][h] = p0 * (dp[n][h] - D0) * kRsd;
-                s[n][2 + h] = p1 * (dp[n][2 + h] - D1) * kRsd;
-            }
-        warp_gemm_regs<16>(dQ, s, sm.kt, kRS64, 0);  // dq += dS K
-    }
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int c = 8 * n + 2 * tq;
-        if (r0 < rows) *reinterpret_cast<float2 *>(dq + head + (size_t)(i0 + r0) * 128 + c) = make_float2(dQ[n][0], dQ[n][1]);
-        if (r1 < rows) *reinterpret_cast<float2 *>(dq + head + (size_t)(i0 + r1) * 128 + c) = make_float2(dQ[n][2], dQ[n][3]);
-    }
-    __syncthreads();  // the sparse dq rows are written; the key-block region is free
 
     // ---- linear branch: H_I^T (stored [dim e][channel c]) and Z_I of this query block
     auto Qa = [&](int r, int c) { return tile_bf(sm.q, r, c); };
     auto dOa = [&](int r, int c) { return tile_bf(sm.dO, r, c); };
-    float *ht = reinterpret_cast<float *>(sm.k);
+    float *ht = sm.ht;
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
     for (int w = tid; w < 128 * 128; w += kBwdThreads) ht[(w >> 7) * kGW + (w & 127)] = __ldg(hrow + w);
     if (tid < 128) sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
@@ -429,42 +236,30 @@ bwd_query_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k,
     }
 }
 
-struct KeySmem {
-    uint32_t k[64 * kRS];      // K rows (B of Q.K^T)
-    uint32_t v[64 * kRS];      // V rows (B of dO.V^T)
-    uint32_t pt[64 * kRS];     // P^T: row j holds P[.][j] over the query rows (A of P^T dO)
-    uint32_t dst[64 * kRS];    // dS^T (A of dS^T Q)
-    // query-block tiles; the linear key side uses this region first for G_J^T (128 x kGW floats)
-    uint32_t q[128 * kRS];     // Q rows (A of Q.K^T)
-    uint32_t qt[128 * kRS];    // Q^T (B of dS^T Q)
-    uint32_t dO[128 * kRS];    // dO rows (A of dO.V^T)
-    uint32_t dOt[128 * kRS];   // dO^T (B of P^T dO)
-    float g[128], m[128], l[128], D[128];
+struct KlinSmem {
+    uint32_t k[64 * kRS];   // K rows of the key block
+    uint32_t v[64 * kRS];   // V rows
+    float gt[128 * kGW];    // G_J^T
+    float g[128];
 };
-static_assert(sizeof(uint32_t) * 4 * 128 * kRS >= sizeof(float) * 128 * kGW, "G_J^T fits in the query region");
 
 // ---------------------------------------------------------------------------
-// step 5: one CTA per (head, key block).  Q.K^T and dO.V^T: warp w owns query rows 16w..;
-// P^T dO and dS^T Q: warp w owns key rows 16 (w % 4).. and dims / channels 64 (w / 4)..
+// step 6: the linear branch's key side, one CTA per (head, key block)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBwdThreads, 1)
-bwd_key_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, const uint16_t *__restrict__ v,
-               const uint16_t *__restrict__ dout, const uint32_t *__restrict__ selT, int n_awT,
-               const float *__restrict__ G, const float *__restrict__ st_m, const float *__restrict__ st_l,
-               const float *__restrict__ st_D, int N, int blk_q, int n_qb, int n_kb, int phi,
-               float *__restrict__ dk, float *__restrict__ dv)
+bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, const float *__restrict__ G, int N,
+                int n_kb, int phi, float *__restrict__ dk, float *__restrict__ dv)
 {
     extern __shared__ uint8_t smem_raw[];
-    KeySmem &sm = *reinterpret_cast<KeySmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+    KlinSmem &sm = *reinterpret_cast<KlinSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
     const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-    const int warp = tid >> 5, lane = tid & 31, tq = lane & 3;
     const int J = blockIdx.x, bh = blockIdx.y;
     const int t0 = J * 64, kv = min(64, N - t0);
     const size_t head = (size_t)bh * N * 128;
 
     load_tile(sm.k, nullptr, 0, k + head, t0, kv, 64);
     load_tile(sm.v, nullptr, 0, v + head, t0, kv, 64);
-    float *gt = reinterpret_cast<float *>(sm.q);
+    float *gt = sm.gt;
     const float *grow = G + ((size_t)bh * n_kb + J) * kStateCols;
     for (int w = tid; w < 128 * 128; w += kBwdThreads) gt[(w >> 7) * kGW + (w & 127)] = __ldg(grow + w);
     if (tid < 128) sm.g[tid] = __ldg(grow + 128 * 128 + tid);
@@ -476,7 +271,7 @@ bwd_key_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, c
     auto GTt = [&](int c, int e) { return gt[e * kGW + c]; };  // B(c, e) = G[c][e]
 
     // ---- linear key side (fp32): dk = (G_J v_j + g_J) phi'(k_j); dv = G_J^T phi(k_j), written
-    //      first and completed by the sparse part below
+    //      here and completed by the softmax branch's key side
     {
         float T[4][8], L[4][8];
 #pragma unroll
@@ -495,82 +290,6 @@ bwd_key_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, c
                 dk[head + (size_t)(t0 + jj) * 128 + c] = (T[i][j] + sm.g[c]) * dphi_f(Ka(jj, c), phi);
                 dv[head + (size_t)(t0 + jj) * 128 + c] = L[i][j];
             }
-        }
-    }
-
-    // ---- sparse branch over the query blocks that selected J
-    const int r0 = 16 * warp + (lane >> 2), r1 = r0 + 8;  // query rows of this thread's S fragments
-    const int jm = 16 * (warp & 3), nh = 64 * (warp >> 2);  // key rows / column half of P^T dO, dS^T Q
-    float dV[8][4], dK[8][4];
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dV[n][e] = dK[n][e] = 0.0f;
-    uint16_t *pt16 = reinterpret_cast<uint16_t *>(sm.pt), *dst16 = reinterpret_cast<uint16_t *>(sm.dst);
-    const uint32_t *bits = selT + ((size_t)bh * n_kb + J) * n_awT;
-    const int words = (n_qb + 31) / 32;
-    for (int w = 0; w < words; ++w) {
-        uint32_t b = __ldg(bits + w);
-        while (b) {
-            const int I = 32 * w + __ffs(b) - 1;
-            b &= b - 1;
-            const int i0 = I * blk_q, rows = min(blk_q, N - i0);
-            __syncthreads();
-            load_tile(sm.q, sm.qt, kRS, q + head, i0, rows, 128);
-            load_tile(sm.dO, sm.dOt, kRS, dout + head, i0, rows, 128);
-            if (tid < 128) {
-                const bool ok = tid < rows;
-                sm.m[tid] = ok ? __ldg(st_m + (size_t)bh * N + i0 + tid) : 0.0f;
-                sm.l[tid] = ok ? __ldg(st_l + (size_t)bh * N + i0 + tid) : 0.0f;
-                sm.D[tid] = ok ? __ldg(st_D + (size_t)bh * N + i0 + tid) : 0.0f;
-            }
-            __syncthreads();
-            float s[8][4], dp[8][4];
-#pragma unroll
-            for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) s[n][e] = dp[n][e] = 0.0f;
-            warp_gemm<8>(s, sm.q, kRS, 16 * warp, sm.k, kRS, 0, 128);
-            warp_gemm<8>(dp, sm.dO, kRS, 16 * warp, sm.v, kRS, 0, 128);
-            const float mq0 = sm.m[r0], lq0 = sm.l[r0], Dq0 = sm.D[r0];
-            const float mq1 = sm.m[r1], lq1 = sm.l[r1], Dq1 = sm.D[r1];
-            const bool v0 = r0 < rows, v1 = r1 < rows;
-#pragma unroll
-            for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = 8 * n + 2 * tq + h;
-                    const float p0 = (v0 && j < kv) ? __expf(s[n][h] * kRsd - mq0) * lq0 : 0.0f;
-                    const float p1 = (v1 && j < kv) ? __expf(s[n][2 + h] * kRsd - mq1) * lq1 : 0.0f;
-                    pt16[j * 2 * kRS + r0] = __bfloat16_as_ushort(__float2bfloat16_rn(p0));
-                    pt16[j * 2 * kRS + r1] = __bfloat16_as_ushort(__float2bfloat16_rn(p1));
-                    dst16[j * 2 * kRS + r0] = __bfloat16_as_ushort(__float2bfloat16_rn(p0 * (dp[n][h] - Dq0) * kRsd));
-                    dst16[j * 2 * kRS + r1] =
-                        __bfloat16_as_ushort(__float2bfloat16_rn(p1 * (dp[n][2 + h] - Dq1) * kRsd));
-                }
-            __syncthreads();
-            warp_gemm<8>(dV, sm.pt, kRS, jm, sm.dOt, kRS, nh, 128);  // dv += P^T dO
-            warp_gemm<8>(dK, sm.dst, kRS, jm, sm.qt, kRS, nh, 128);  // dk += dS^T q / sqrt(d)
-        }
-    }
-    __syncthreads();  // the linear part's dk, dv rows are written
-    const int j0 = jm + (lane >> 2), j1 = j0 + 8;
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-        const int c = nh + 8 * n + 2 * tq;
-        if (j0 < kv) {
-            float2 *pk = reinterpret_cast<float2 *>(dk + head + (size_t)(t0 + j0) * 128 + c);
-            float2 *pv = reinterpret_cast<float2 *>(dv + head + (size_t)(t0 + j0) * 128 + c);
-            const float2 ok_ = *pk, ov_ = *pv;
-            *pk = make_float2(ok_.x + dK[n][0], ok_.y + dK[n][1]);
-            *pv = make_float2(ov_.x + dV[n][0], ov_.y + dV[n][1]);
-        }
-        if (j1 < kv) {
-            float2 *pk = reinterpret_cast<float2 *>(dk + head + (size_t)(t0 + j1) * 128 + c);
-            float2 *pv = reinterpret_cast<float2 *>(dv + head + (size_t)(t0 + j1) * 128 + c);
-            const float2 ok_ = *pk, ov_ = *pv;
-            *pk = make_float2(ok_.x + dK[n][2], ok_.y + dK[n][3]);
-            *pv = make_float2(ov_.x + dV[n][2], ov_.y + dV[n][3]);
         }
     }
 }
@@ -639,6 +358,8 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
     int *status = static_cast<int *>(at(ws, F.status));
     double *qbar = static_cast<double *>(at(ws, F.qbar));
     double *kbar = static_cast<double *>(at(ws, F.kbar));
+    double *kpart = static_cast<double *>(at(ws, F.kpart));
+    float *kmean = static_cast<float *>(at(ws, F.kmean));
     double *scores = static_cast<double *>(at(ws, F.scores));
     int32_t *idx = static_cast<int32_t *>(at(ws, F.idx));
     uint32_t *amask = static_cast<uint32_t *>(at(ws, F.amask));
@@ -658,26 +379,28 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
     cudaError_t e;
 #define BWD_TRY(x) do { if ((e = (x)) != cudaSuccess) return e; } while (0)
     BWD_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-    // 1. the forward's selection and states (quantisation off)
+    // 1. the forward's selection and states (quantisation off), and the head's mean key
     BWD_TRY(launch_pool(q, g.BH, g.N, g.blk_q, g.n_qb, qbar, nullptr, s));
-    BWD_TRY(launch_pool(k, g.BH, g.N, g.blk_k, g.n_kb, kbar, nullptr, s));
+    BWD_TRY(launch_pool(k, g.BH, g.N, g.blk_k, g.n_kb, kbar, kpart, s));
+    BWD_TRY(launch_kmean(kpart, g.BH, g.N, pool_parts(g.n_kb), kmean, s));
     BWD_TRY(launch_states(k, v, g, phi, states, partials, nullptr, status, s));
     BWD_TRY(launch_htot(partials, g, htot, s));
     BWD_TRY(launch_scores(qbar, kbar, g, scores, s));
     BWD_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
     BWD_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));
-    // 2. query side
+    // 2. softmax branch, query side: row statistics and dq
     const int ks = g.k_sel;
+    BWD_TRY(launch_bwd_query_sparse(q, k, v, dout, idx, kmean, g, dq, st_m, st_l, st_D, status, s));
+    // 3. linear branch, query side: dq (added), dH_I, dZ_I
     {
-        const size_t smem = sizeof(QuerySmem) + 16;
-        BWD_TRY(cudaFuncSetAttribute(bwd_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        bwd_query_kernel<<<dim3(g.n_qb, g.BH), kBwdThreads, smem, s>>>(
-            static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v),
-            static_cast<const uint16_t *>(dout), idx, hq, g.N, g.blk_q, g.n_qb, ks, phi, dq, st_m, st_l, st_D, dh32,
-            dh16);
+        const size_t smem = sizeof(QlinSmem) + 16;
+        BWD_TRY(cudaFuncSetAttribute(bwd_qlin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        bwd_qlin_kernel<<<dim3(g.n_qb, g.BH), kBwdThreads, smem, s>>>(
+            static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(dout), hq, g.N, g.blk_q, g.n_qb, phi, dq,
+            dh32, dh16);
         BWD_TRY(cudaGetLastError());
     }
-    // 3. column sum of dH over the query blocks; transposed selection bits
+    // 4. column sum of dH over the query blocks; transposed selection bits
     {
         Geometry gh = g;
         gh.n_chunks = g.n_qb;
@@ -695,7 +418,7 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
             BWD_TRY(cudaGetLastError());
         }
     }
-    // 4. G = A^T dH (the state reduction on the transposed mask)
+    // 5. G = A^T dH (the state reduction on the transposed mask)
     {
         Geometry gt = g;
         gt.n_qb = g.n_kb;
@@ -703,16 +426,16 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const v
         gt.n_aw = L.n_awT;
         BWD_TRY(launch_state_reduce(amaskT, dh16, dhtot, gt, G, status, s));
     }
-    // 5. key side
+    // 6. linear branch, key side: dk, dv written
     {
-        const size_t smem = sizeof(KeySmem) + 16;
-        BWD_TRY(cudaFuncSetAttribute(bwd_key_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        bwd_key_kernel<<<dim3(g.n_kb, g.BH), kBwdThreads, smem, s>>>(
-            static_cast<const uint16_t *>(q), static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v),
-            static_cast<const uint16_t *>(dout), selT, L.n_awT, G, st_m, st_l, st_D, g.N, g.blk_q, g.n_qb, g.n_kb,
-            phi, dk, dv);
+        const size_t smem = sizeof(KlinSmem) + 16;
+        BWD_TRY(cudaFuncSetAttribute(bwd_klin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        bwd_klin_kernel<<<dim3(g.n_kb, g.BH), kBwdThreads, smem, s>>>(
+            static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), G, g.N, g.n_kb, phi, dk, dv);
         BWD_TRY(cudaGetLastError());
     }
+    // 7. softmax branch, key side: dk, dv added
+    BWD_TRY(launch_bwd_key_sparse(q, k, v, dout, selT, L.n_awT, st_m, st_l, st_D, g, dk, dv, status, s));
 #undef BWD_TRY
     return cudaSuccess;
 }

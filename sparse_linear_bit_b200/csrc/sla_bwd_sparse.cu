@@ -1,0 +1,645 @@
+// sla_bwd_sparse.cu -- the softmax branch of the SageSLA backward on tcgen05
+// tensor cores (SLA fine-tuning: the jiqiren.org.cn TurboDiffusion article,
+// 方法论; the "TurboDiffusion" summary page, 主要能力: SLA white-box training).
+//
+// For row i of query block I and the tokens j of the key blocks I selected,
+// with s = q.k / sqrt(d), p = softmax_j(s), dP = do.v, D_i = sum_j p_ij dP_ij:
+//   dS_ij = p_ij (dP_ij - D_i) / sqrt(d);  dq_i = sum_j dS_ij k_j;
+//   dv_j = sum_i p_ij do_i;                 dk_j = sum_i dS_ij q_i.
+//
+// bwdq_kernel, one CTA per (head, query block), two passes over the selected
+// key blocks (K and V tiles stream through a TMA ring twice):
+//   pass 1: S = Q K^T and dP = dO V^T into tensor memory; per row the online
+//           max m, sum l and D (the softmax-weighted sum of dP), written out
+//           for the key side;
+//   pass 2: S and dP again; dS from them in fp32, rounded to bf16 into shared
+//           memory, and dQ += dS K accumulated in tensor memory.  Since
+//           sum_j dS_ij = 0, dq_i = sum_j dS_ij (k_j - mu) for any vector mu;
+//           with mu = the head's mean key, the bf16 rounding of dS is not
+//           multiplied by the keys' common component: the kernel sums, in
+//           fp32, sigma_i = sum_j of the rounded dS_ij and writes
+//           dq_i = (dS K)_i - sigma_i mu.
+// bwdk_kernel, one CTA per (head, key block), over the query blocks that
+//   selected it: S and dP as above, P and dS (from the row statistics of
+//   pass 1) rounded to bf16 into shared memory, and dV^T += dO^T P,
+//   dK^T += Q^T dS accumulated in tensor memory (M = 128 dims, N = 64 keys);
+//   the results are added to dk, dv, which the linear branch's key side has
+//   written before.
+//
+// Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 2-5 one row per thread (query rows; in bwdk's epilogue, dims).  All
+// products take bf16 operands with fp32 accumulation.  Every wait is bounded
+// (see sla_ptx.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "sla_internal.h"
+#include "sla_ptx.cuh"
+
+namespace sla {
+namespace {
+
+constexpr int kBwThreads = 192;
+constexpr uint32_t kBox = 64 * 128;    // [64 rows x 128 B]
+constexpr uint32_t kTile = 128 * 128;  // [128 rows x 128 B]
+constexpr int kBqStages = 3;
+constexpr int kBkStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRsd = 0.08838834764831845f;  // 1 / sqrt(128)
+
+SLA_DEV uint64_t dadd(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
+SLA_DEV float ex2f(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+SLA_DEV void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// 64 fp32 columns of this thread's TMEM lane
+SLA_DEV void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
+{
+    tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+}
+
+// row r (64 bf16 = 128 B, packed in 32 words) of a [128 rows x 128 B] tile with the 128-byte swizzle
+SLA_DEV void store_row_sw128(uint8_t *tile, int r, const uint32_t (&w)[32])
+{
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4 *>(tile + sw128_off(r, u)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+}
+
+// S and dP of one (query block, key block) tile: M = 128 query rows, N = 64 keys, K = 128 in
+// 8 steps of 16 bf16.  A tiles (Q, dO) are [128 rows x 128 B] boxes, B tiles (K, V) [64 rows x 128 B]
+// boxes, both K-major with the 128-byte swizzle, channels 0-63 then 64-127.
+SLA_DEV void issue_s_dp(uint32_t t_s, uint32_t t_dp, uint64_t qd, uint64_t dod, uint64_t kd, uint64_t vd)
+{
+    constexpr uint32_t id = idesc(1, 1, 1, 0, 0, 128, 64);  // f32 <- bf16 x bf16
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_bf16(t_s, dadd(qd, (k >> 2) * kTile + (k & 3) * 32), dadd(kd, (k >> 2) * kBox + (k & 3) * 32), id,
+                 k > 0 ? 1u : 0u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_bf16(t_dp, dadd(dod, (k >> 2) * kTile + (k & 3) * 32), dadd(vd, (k >> 2) * kBox + (k & 3) * 32), id,
+                 k > 0 ? 1u : 0u);
+}
+
+// ---------------------------------------------------------------------------
+// query side
+// ---------------------------------------------------------------------------
+struct BqSmem {
+    alignas(1024) uint8_t q[2 * kTile];              // Q_I: channels 0-63 | 64-127
+    alignas(1024) uint8_t dO[2 * kTile];             // dO_I: dims 0-63 | 64-127
+    alignas(1024) uint8_t kv[kBqStages][4][kBox];    // per stage: K_J ch 0-63 | 64-127, V_J dims 0-63 | 64-127
+    alignas(1024) uint8_t ds[2][kTile];              // dS tiles: [128 rows x 64 keys] bf16
+    float mu[128];
+    uint64_t full[kBqStages], empty[kBqStages];
+    uint64_t bar_qdo, bar_sd[2], bar_sdfree[2], bar_ds[2], bar_dsfree[2], bar_dq, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+            const int32_t *__restrict__ idx, const float *__restrict__ kmean, int N, int blk_q, int n_qb, int k_sel,
+            float *__restrict__ dq, float *__restrict__ st_m, float *__restrict__ st_l, float *__restrict__ st_D,
+            int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    BqSmem &sm = *reinterpret_cast<BqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int I = blockIdx.x, bh = blockIdx.y;
+    const int32_t *sel = idx + ((size_t)bh * n_qb + I) * k_sel;
+    const int nT = 2 * k_sel;  // tiles: pass 1 (T < k_sel), then pass 2
+    volatile int *abort_flag = &sm.abort_flag;
+    if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
+    __syncthreads();
+    if (sm.abort_flag) return;  // another CTA already failed: CTA-uniform early exit
+
+    if (tid == 0) {
+        for (int s = 0; s < kBqStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.bar_qdo, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_sd[b], 1);
+            mbar_init(&sm.bar_sdfree[b], 128);
+            mbar_init(&sm.bar_ds[b], 128);
+            mbar_init(&sm.bar_dsfree[b], 1);
+        }
+        mbar_init(&sm.bar_dq, 1);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;  // S / dP of buffer b at 128 b / 128 b + 64; dQ at 256
+    const uint32_t t_dq = tmem + 256;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_do);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_expect_tx(&sm.bar_qdo, 4 * kTile);
+            for (int c = 0; c < 2; ++c) {
+                tma_load_3d(sm.q + c * kTile, &tm_q, &sm.bar_qdo, 64 * c, I * blk_q, bh);
+                tma_load_3d(sm.dO + c * kTile, &tm_do, &sm.bar_qdo, 64 * c, I * blk_q, bh);
+            }
+        }
+        __syncwarp();
+        int issued = 0;
+        bool ok = true;
+        for (int T = 0; ok && T < nT; ++T) {
+            const int s = T % kBqStages, u = T / kBqStages;
+            if (u > 0 && !(ok = mbar_wait_warp(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+            const int J = __ldg(sel + (T < k_sel ? T : T - k_sel));
+            if (elect_one()) {
+                mbar_expect_tx(&sm.full[s], 4 * kBox);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_3d(sm.kv[s][c], &tm_k, &sm.full[s], 64 * c, J * 64, bh);
+                    tma_load_3d(sm.kv[s][2 + c], &tm_v, &sm.full[s], 64 * c, J * 64, bh);
+                }
+            }
+            __syncwarp();
+            issued = T + 1;
+        }
+        // every load issued has landed before shared memory is released
+        for (int s = 0; s < kBqStages; ++s) {
+            int tl = -1;
+            for (int T = s; T < issued; T += kBqStages) tl = T;
+            if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / kBqStages) & 1, status);
+        }
+        mbar_wait_quiet(&sm.bar_qdo, 0, status);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t id_dq = idesc(1, 1, 1, 0, 1, 128, 128);  // A = dS K-major, B = K MN-major
+        const uint64_t qd = sdesc_sw128(smem_u32(sm.q), 16, 1024), dod = sdesc_sw128(smem_u32(sm.dO), 16, 1024);
+        bool ok = k_sel == 0 || mbar_wait_warp(&sm.bar_qdo, 0, status, abort_flag);
+        auto issue_sd = [&](int T) {
+            const int s = T % kBqStages, b = T & 1;
+            if (!(ok = mbar_wait_warp(&sm.full[s], (T / kBqStages) & 1, status, abort_flag))) return;
+            if (T >= 2 && !(ok = mbar_wait_warp(&sm.bar_sdfree[b], ((T >> 1) - 1) & 1, status, abort_flag))) return;
+            tc_fence_after();
+            if (elect_one()) {
+                issue_s_dp(tmem + 128 * b, tmem + 128 * b + 64, qd, dod, sdesc_sw128(smem_u32(sm.kv[s][0]), 16, 1024),
+                           sdesc_sw128(smem_u32(sm.kv[s][2]), 16, 1024));
+                mma_commit(&sm.bar_sd[b]);
+                if (T < k_sel) mma_commit(&sm.empty[s]);  // pass 1: the stage is free after S and dP
+            }
+            __syncwarp();
+        };
+        auto issue_dq = [&](int t) {  // pass-2 tile t
+            const int T = k_sel + t, s = T % kBqStages, b = t & 1;
+            if (!(ok = mbar_wait_warp(&sm.bar_ds[b], (t >> 1) & 1, status, abort_flag))) return;
+            tc_fence_after();
+            if (elect_one()) {
+                const uint64_t dsd = sdesc_sw128(smem_u32(sm.ds[b]), 16, 1024);
+                const uint64_t kmn = sdesc_sw128(smem_u32(sm.kv[s][0]), kBox, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)  // K-step of 16 keys: 32 B of a dS row, 2 KB of K rows
+                    mma_bf16(t_dq, dadd(dsd, 32 * k), dadd(kmn, 2048 * k), id_dq, (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_dsfree[b]);
+                mma_commit(&sm.empty[s]);
+                if (t == k_sel - 1) mma_commit(&sm.bar_dq);
+            }
+            __syncwarp();
+        };
+        for (int T = 0; ok && T < nT; ++T) {
+            issue_sd(T);
+            if (ok && T - 1 >= k_sel) issue_dq(T - 1 - k_sel);
+        }
+        if (ok && k_sel > 0) issue_dq(k_sel - 1);
+        if (elect_one()) {
+            mma_commit(&sm.drain);
+            mbar_wait_quiet(&sm.drain, 0, status);  // this thread's MMAs retired before TMEM is released
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ rows
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int i = I * blk_q + r;
+        const bool row_valid = r < blk_q && i < N;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            const bool w = mbar_wait(bar, par, status, abort_flag);
+            return __all_sync(0xffffffffu, w);
+        };
+        sm.mu[r] = __ldg(kmean + (size_t)bh * 128 + r);
+        named_bar_sync(1, 128);
+        const float c = kLog2e * kRsd;
+        bool ok = true;
+        // ---- pass 1: row max m, sum l and D = sum p dP (online, in log2 units)
+        float m = -INFINITY, l = 0.0f, Dt = 0.0f;
+        for (int t = 0; ok && t < k_sel; ++t) {
+            const int T = t, b = T & 1;
+            const int J = __ldg(sel + t), valid = min(64, N - J * 64);
+            if (!(ok = wait_all(&sm.bar_sd[b], (T >> 1) & 1))) break;
+            tc_fence_after();
+            uint32_t sv[64], dv[64];
+            tmem_ld64(tmem + 128 * b + lane_off, sv);
+            tmem_ld64(tmem + 128 * b + 64 + lane_off, dv);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_sdfree[b]);
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < valid) tmax = fmaxf(tmax, __uint_as_float(sv[j]) * c);
+            const float mn = fmaxf(m, tmax);
+            const float alpha = ex2f(m - mn);  // 0 while m = -inf
+            l *= alpha;
+            Dt *= alpha;
+            m = mn;
+            float ls = 0.0f, ds = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float p = j < valid ? ex2f(__uint_as_float(sv[j]) * c - m) : 0.0f;
+                ls += p;
+                ds = fmaf(p, __uint_as_float(dv[j]), ds);
+            }
+            l += ls;
+            Dt += ds;
+        }
+        const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
+        const float D = Dt * inv_l;
+        if (ok && row_valid) {
+            st_m[(size_t)bh * N + i] = m;
+            st_l[(size_t)bh * N + i] = inv_l;
+            st_D[(size_t)bh * N + i] = D;
+        }
+        // ---- pass 2: dS (bf16) into shared memory for dQ += dS K
+        float sigma = 0.0f;  // fp32 sum of the rounded dS of this row
+        for (int t = 0; ok && t < k_sel; ++t) {
+            const int T = k_sel + t, b = T & 1, bd = t & 1;
+            const int J = __ldg(sel + t), valid = row_valid ? min(64, N - J * 64) : 0;
+            if (!(ok = wait_all(&sm.bar_sd[b], (T >> 1) & 1))) break;
+            tc_fence_after();
+            uint32_t sv[64], dv[64];
+            tmem_ld64(tmem + 128 * b + lane_off, sv);
+            tmem_ld64(tmem + 128 * b + 64 + lane_off, dv);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_sdfree[b]);
+            uint32_t w[32];
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+                float g[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float p = (j + h) < valid ? ex2f(__uint_as_float(sv[j + h]) * c - m) * inv_l : 0.0f;
+                    g[h] = p * (__uint_as_float(dv[j + h]) - D) * kRsd;
+                }
+                w[j >> 1] = pack_bf16x2(g[0], g[1]);
+                sigma += __uint_as_float(w[j >> 1] << 16) + __uint_as_float(w[j >> 1] & 0xFFFF0000u);
+            }
+            if (t >= 2 && !(ok = wait_all(&sm.bar_dsfree[bd], ((t >> 1) - 1) & 1))) break;
+            store_row_sw128(sm.ds[bd], r, w);
+            fence_async_smem();
+            mbar_arrive(&sm.bar_ds[bd]);
+        }
+        // ---- dq = dS K - sigma mu (zero without selected blocks)
+        if (ok && k_sel > 0) ok = wait_all(&sm.bar_dq, 0);
+        if (ok) {
+            tc_fence_after();
+            float *drow = dq + ((size_t)bh * N + (row_valid ? i : 0)) * 128;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t a[32];
+                if (k_sel > 0) {
+                    tmem_ld32(t_dq + lane_off + c0, a);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) a[e] = 0u;
+                }
+                if (row_valid) {
+                    float4 *o = reinterpret_cast<float4 *>(drow + c0);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = make_float4(fmaf(-sigma, sm.mu[c0 + 4 * e], __uint_as_float(a[4 * e])),
+                                           fmaf(-sigma, sm.mu[c0 + 4 * e + 1], __uint_as_float(a[4 * e + 1])),
+                                           fmaf(-sigma, sm.mu[c0 + 4 * e + 2], __uint_as_float(a[4 * e + 2])),
+                                           fmaf(-sigma, sm.mu[c0 + 4 * e + 3], __uint_as_float(a[4 * e + 3])));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// key side
+// ---------------------------------------------------------------------------
+struct BkSmem {
+    alignas(1024) uint8_t k[2 * kBox];               // K_J: ch 0-63 | 64-127
+    alignas(1024) uint8_t v[2 * kBox];               // V_J: dims 0-63 | 64-127
+    alignas(1024) uint8_t qd[kBkStages][4 * kTile];  // per stage: Q_I ch 0-63 | 64-127, dO_I dims 0-63 | 64-127
+    alignas(1024) uint8_t p[2][kTile];               // P tiles: [128 query rows x 64 keys] bf16
+    alignas(1024) uint8_t ds[2][kTile];              // dS tiles
+    uint64_t full[kBkStages], empty[kBkStages];
+    uint64_t bar_kv, bar_sd[2], bar_sdfree[2], bar_pd[2], bar_pdfree[2], bar_acc, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// walks the set bits of a selection row (query blocks that selected a key block), in order
+struct BitWalk {
+    const uint32_t *bits;
+    int words, w;
+    uint32_t cur;
+    SLA_DEV BitWalk(const uint32_t *b, int nw) : bits(b), words(nw), w(0), cur(nw > 0 ? __ldg(b) : 0u) {}
+    SLA_DEV int next()
+    {
+        while (cur == 0u) {
+            if (++w >= words) return -1;
+            cur = __ldg(bits + w);
+        }
+        const int I = 32 * w + __ffs(cur) - 1;
+        cur &= cur - 1u;
+        return I;
+    }
+};
+
+__global__ void __launch_bounds__(kBwThreads, 1)
+bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+            const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+            const uint32_t *__restrict__ selT, int n_awT, const float *__restrict__ st_m,
+            const float *__restrict__ st_l, const float *__restrict__ st_D, int N, int blk_q, int n_qb, int n_kb,
+            float *__restrict__ dk, float *__restrict__ dv, int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    BkSmem &sm = *reinterpret_cast<BkSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int J = blockIdx.x, bh = blockIdx.y;
+    const int t0 = J * 64, kv = min(64, N - t0);
+    const uint32_t *bits = selT + ((size_t)bh * n_kb + J) * n_awT;
+    const int words = (n_qb + 31) / 32;
+    int n_sel = 0;
+    for (int w = 0; w < words; ++w) n_sel += __popc(__ldg(bits + w));
+    volatile int *abort_flag = &sm.abort_flag;
+    if (tid == 0) sm.abort_flag = global_failed(status) ? 1 : 0;
+    __syncthreads();
+    // no query block selected this key block (dk, dv hold the linear part alone), or another CTA
+    // failed: CTA-uniform early exit
+    if (sm.abort_flag || n_sel == 0) return;
+
+    if (tid == 0) {
+        for (int s = 0; s < kBkStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.bar_kv, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.bar_sd[b], 1);
+            mbar_init(&sm.bar_sdfree[b], 128);
+            mbar_init(&sm.bar_pd[b], 128);
+            mbar_init(&sm.bar_pdfree[b], 1);
+        }
+        mbar_init(&sm.bar_acc, 1);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;  // S / dP of buffer b at 128 b / 128 b + 64; dV^T at 256, dK^T at 320
+    const uint32_t t_dv = tmem + 256, t_dk = tmem + 320;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_do);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_expect_tx(&sm.bar_kv, 4 * kBox);
+            for (int c = 0; c < 2; ++c) {
+                tma_load_3d(sm.k + c * kBox, &tm_k, &sm.bar_kv, 64 * c, t0, bh);
+                tma_load_3d(sm.v + c * kBox, &tm_v, &sm.bar_kv, 64 * c, t0, bh);
+            }
+        }
+        __syncwarp();
+        BitWalk walk(bits, words);
+        int issued = 0;
+        bool ok = true;
+        for (int t = 0; ok && t < n_sel; ++t) {
+            const int I = walk.next();
+            const int s = t % kBkStages, u = t / kBkStages;
+            if (u > 0 && !(ok = mbar_wait_warp(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
+            if (elect_one()) {
+                mbar_expect_tx(&sm.full[s], 4 * kTile);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_3d(sm.qd[s] + c * kTile, &tm_q, &sm.full[s], 64 * c, I * blk_q, bh);
+                    tma_load_3d(sm.qd[s] + (2 + c) * kTile, &tm_do, &sm.full[s], 64 * c, I * blk_q, bh);
+                }
+            }
+            __syncwarp();
+            issued = t + 1;
+        }
+        for (int s = 0; s < kBkStages; ++s) {
+            int tl = -1;
+            for (int t = s; t < issued; t += kBkStages) tl = t;
+            if (tl >= 0) mbar_wait_quiet(&sm.full[s], (tl / kBkStages) & 1, status);
+        }
+        mbar_wait_quiet(&sm.bar_kv, 0, status);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // dV^T += dO^T P and dK^T += Q^T dS: M = 128 dims / channels, N = 64 keys, K = 128 query rows,
+        // A (dO, Q) and B (P, dS) both MN-major
+        constexpr uint32_t id_acc = idesc(1, 1, 1, 1, 1, 128, 64);
+        const uint64_t kd = sdesc_sw128(smem_u32(sm.k), 16, 1024), vd = sdesc_sw128(smem_u32(sm.v), 16, 1024);
+        bool ok = mbar_wait_warp(&sm.bar_kv, 0, status, abort_flag);
+        auto issue_sd = [&](int t) {
+            const int s = t % kBkStages, b = t & 1;
+            if (!(ok = mbar_wait_warp(&sm.full[s], (t / kBkStages) & 1, status, abort_flag))) return;
+            if (t >= 2 && !(ok = mbar_wait_warp(&sm.bar_sdfree[b], ((t >> 1) - 1) & 1, status, abort_flag))) return;
+            tc_fence_after();
+            if (elect_one()) {
+                issue_s_dp(tmem + 128 * b, tmem + 128 * b + 64, sdesc_sw128(smem_u32(sm.qd[s]), 16, 1024),
+                           sdesc_sw128(smem_u32(sm.qd[s] + 2 * kTile), 16, 1024), kd, vd);
+                mma_commit(&sm.bar_sd[b]);
+            }
+            __syncwarp();
+        };
+        auto issue_acc = [&](int t) {
+            const int s = t % kBkStages, b = t & 1;
+            if (!(ok = mbar_wait_warp(&sm.bar_pd[b], (t >> 1) & 1, status, abort_flag))) return;
+            tc_fence_after();
+            if (elect_one()) {
+                const uint64_t qmn = sdesc_sw128(smem_u32(sm.qd[s]), kTile, 1024);
+                const uint64_t domn = sdesc_sw128(smem_u32(sm.qd[s] + 2 * kTile), kTile, 1024);
+                const uint64_t pmn = sdesc_sw128(smem_u32(sm.p[b]), kTile, 1024);
+                const uint64_t dsmn = sdesc_sw128(smem_u32(sm.ds[b]), kTile, 1024);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)  // K-step of 16 query rows: 2 KB of each tile
+                    mma_bf16(t_dv, dadd(domn, 2048 * k), dadd(pmn, 2048 * k), id_acc, (t > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(t_dk, dadd(qmn, 2048 * k), dadd(dsmn, 2048 * k), id_acc, (t > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&sm.bar_pdfree[b]);
+                mma_commit(&sm.empty[s]);  // Q and dO of the stage are no longer read
+                if (t == n_sel - 1) mma_commit(&sm.bar_acc);
+            }
+            __syncwarp();
+        };
+        for (int t = 0; ok && t < n_sel; ++t) {
+            issue_sd(t);
+            if (ok && t >= 1) issue_acc(t - 1);
+        }
+        if (ok) issue_acc(n_sel - 1);
+        if (elect_one()) {
+            mma_commit(&sm.drain);
+            mbar_wait_quiet(&sm.drain, 0, status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ rows (query rows; dims at the end)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        auto wait_all = [&](uint64_t *bar, uint32_t par) {
+            const bool w = mbar_wait(bar, par, status, abort_flag);
+            return __all_sync(0xffffffffu, w);
+        };
+        const float c = kLog2e * kRsd;
+        BitWalk walk(bits, words);
+        bool ok = true;
+        for (int t = 0; ok && t < n_sel; ++t) {
+            const int I = walk.next(), b = t & 1;
+            const int i = I * blk_q + r;
+            const bool row_valid = r < blk_q && i < N;  // rows of the next query block (blk_q = 64) excluded
+            const size_t si = (size_t)bh * N + (row_valid ? i : 0);
+            const float m = row_valid ? __ldg(st_m + si) : 0.0f;
+            const float il = row_valid ? __ldg(st_l + si) : 0.0f;
+            const float D = row_valid ? __ldg(st_D + si) : 0.0f;
+            const int valid = row_valid ? kv : 0;
+            if (!(ok = wait_all(&sm.bar_sd[b], (t >> 1) & 1))) break;
+            tc_fence_after();
+            uint32_t sv[64], dpv[64];
+            tmem_ld64(tmem + 128 * b + lane_off, sv);
+            tmem_ld64(tmem + 128 * b + 64 + lane_off, dpv);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&sm.bar_sdfree[b]);
+            uint32_t wp[32], wd[32];
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+                float p[2], g[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    p[h] = (j + h) < valid ? ex2f(__uint_as_float(sv[j + h]) * c - m) * il : 0.0f;
+                    g[h] = p[h] * (__uint_as_float(dpv[j + h]) - D) * kRsd;
+                }
+                wp[j >> 1] = pack_bf16x2(p[0], p[1]);
+                wd[j >> 1] = pack_bf16x2(g[0], g[1]);
+            }
+            if (t >= 2 && !(ok = wait_all(&sm.bar_pdfree[b], ((t >> 1) - 1) & 1))) break;
+            store_row_sw128(sm.p[b], r, wp);
+            store_row_sw128(sm.ds[b], r, wd);
+            fence_async_smem();
+            mbar_arrive(&sm.bar_pd[b]);
+        }
+        // ---- epilogue: TMEM lane r = dim / channel r; column j = key t0 + j.  Added to the linear part.
+        if (ok) ok = wait_all(&sm.bar_acc, 0);
+        if (ok) {
+            tc_fence_after();
+            uint32_t a[64];
+            tmem_ld64(t_dv + lane_off, a);
+            tmem_wait_ld();
+            float *pv = dv + ((size_t)bh * N + t0) * 128 + r;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < kv) pv[(size_t)j * 128] += __uint_as_float(a[j]);
+            tmem_ld64(t_dk + lane_off, a);
+            tmem_wait_ld();
+            float *pk = dk + ((size_t)bh * N + t0) * 128 + r;
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (j < kv) pk[(size_t)j * 128] += __uint_as_float(a[j]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    __syncwarp();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// 3-D map [BH, N, 128] of a bf16 tensor, boxes of 64 channels x `rows` rows
+bool map_rows(CUtensorMap *m, const void *base, const Geometry &g, uint32_t rows)
+{
+    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
+    const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
+    const uint32_t box[3] = {64, rows, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, st, box);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_query_sparse(const void *q, const void *k, const void *v, const void *dout,
+                                    const int32_t *idx, const float *kmean, const Geometry &g, float *dq,
+                                    float *st_m, float *st_l, float *st_D, int *status, cudaStream_t s)
+{
+    CUtensorMap tq, tdo, tk, tv;
+    if (!map_rows(&tq, q, g, 128) || !map_rows(&tdo, dout, g, 128) || !map_rows(&tk, k, g, 64) ||
+        !map_rows(&tv, v, g, 64))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(BqSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwdq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwdq_kernel<<<dim3(g.n_qb, g.BH), kBwThreads, smem, s>>>(tq, tdo, tk, tv, idx, kmean, g.N, g.blk_q, g.n_qb,
+                                                             g.k_sel, dq, st_m, st_l, st_D, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, const void *dout,
+                                  const uint32_t *selT, int n_awT, const float *st_m, const float *st_l,
+                                  const float *st_D, const Geometry &g, float *dk, float *dv, int *status,
+                                  cudaStream_t s)
+{
+    CUtensorMap tq, tdo, tk, tv;
+    if (!map_rows(&tq, q, g, 128) || !map_rows(&tdo, dout, g, 128) || !map_rows(&tk, k, g, 64) ||
+        !map_rows(&tv, v, g, 64))
+        return cudaErrorInvalidValue;
+    const size_t smem = sizeof(BkSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwdk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwdk_kernel<<<dim3(g.n_kb, g.BH), kBwThreads, smem, s>>>(tq, tdo, tk, tv, selT, n_awT, st_m, st_l, st_D, g.N,
+                                                             g.blk_q, g.n_qb, g.n_kb, dk, dv, status);
+    return cudaGetLastError();
+}
+
+cudaError_t set_wait_budget_bwd(long long cycles) { return set_tu_wait_budget(cycles); }
+
+}  // namespace sla

@@ -63,6 +63,15 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
 size_t backward_workspace_bytes(const Geometry &g);
 cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *dout, float *dq, float *dk,
                             float *dv, const Geometry &g, int phi, void *ws, cudaStream_t s);
+// the softmax branch of the backward on the tensor cores (sla_bwd_sparse.cu): the query side writes
+// dq and the row statistics (max m, 1/l, D); the key side adds to dk, dv
+cudaError_t launch_bwd_query_sparse(const void *q, const void *k, const void *v, const void *dout,
+                                    const int32_t *idx, const float *kmean, const Geometry &g, float *dq,
+                                    float *st_m, float *st_l, float *st_D, int *status, cudaStream_t s);
+cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, const void *dout,
+                                  const uint32_t *selT, int n_awT, const float *st_m, const float *st_l,
+                                  const float *st_D, const Geometry &g, float *dk, float *dv, int *status,
+                                  cudaStream_t s);
 // TMA descriptor encoding (driver entry point fetched once through the runtime)
 // W8A8 linear layer (sla_w8a8.cu)
 cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,
@@ -74,6 +83,7 @@ cudaError_t launch_w8a8_gemm(const int8_t *qx, const float *sx, const int8_t *qw
 cudaError_t set_wait_budget_attention(long long cycles);
 cudaError_t set_wait_budget_linear(long long cycles);
 cudaError_t set_wait_budget_w8a8(long long cycles);
+cudaError_t set_wait_budget_bwd(long long cycles);
 bool encode_tmap(CUtensorMap *map, CUtensorMapDataType dtype, int rank, const void *base, const uint64_t *dims,
                  const uint64_t *strides_bytes /* rank-1 entries */, const uint32_t *box);
 

@@ -10,6 +10,8 @@ tf32 (2^-11), and the state gradients entering G = A^T dH as bf16 (2^-9).  So
 either branch's part of a gradient carries up to ~2 x 2^-9 ~ 4e-3 relative
 error, and the whole gradient less.
 Every element must also be finite, and two calls must give identical bytes.
+At the full 14B-720P size, dq of sampled rows and dk, dv of sampled key blocks are
+compared with the oracle, which evaluates exactly those rows / blocks.
 """
 from __future__ import annotations
 
@@ -63,6 +65,7 @@ def test_backward_parity(name):
     for nm, g_, r_ in zip(("dq", "dk", "dv"), got, ref):
         assert np.isfinite(g_).all(), (name, nm)
         err = rel_l2(g_, r_)
+        print(f"\n{name} {nm}: rel_l2={err:.3e}")
         assert err <= TOL, (name, nm, err)
 
 
@@ -112,4 +115,34 @@ def test_backward_full_size_sampled_dq():
     ref = oracle.backward_dq_rows(q, k, v, dout, w.blk_q, w.blk_k, float(np.float32(0.1)), rows, phi=0)
     assert np.isfinite(got).all()
     err = rel_l2(got, ref)
+    print(f"\nfull-size sampled rows: dq rel_l2={err:.3e}")
     assert err <= TOL, err
+
+
+def test_backward_full_size_sampled_dkdv():
+    """14B-720P shape (B=1, H=40, N=75600), the launch configuration bench.py times: dk and dv of three
+    key blocks of three heads -- the first block, one in the middle and the ragged last block (16 keys)
+    -- against the oracle, which evaluates exactly those blocks (their linear part needs the state
+    gradients of every query block that did not select them, their softmax part every row that did)."""
+    w = synth.WORKLOADS["wan14b-720p"]
+    q, k, v = workload_qkv("wan14b-720p")
+    dout = workload_qkv("wan14b-720p", seed_offset=1)[0]
+    dq, dk, dv = run_backward(q, k, v, dout, w.blk_q, 0.1, 0)
+    del dq
+    n_kb = -(-w.N // w.blk_k)
+    blocks = np.array([[0, 0], [17, n_kb // 2], [39, n_kb - 1]], dtype=np.int64)
+    ref_k, ref_v = oracle.backward_dkdv_blocks(q, k, v, dout, w.blk_q, w.blk_k, float(np.float32(0.1)), blocks,
+                                               phi=0)
+    dk_h, dv_h = dk.view(w.B * w.H, w.N, 128), dv.view(w.B * w.H, w.N, 128)
+    gk, gv, rk, rv = [], [], [], []
+    for b, (bh, J) in enumerate(blocks.tolist()):
+        n = min(64, w.N - 64 * J)
+        gk.append(dk_h[bh, 64 * J:64 * J + n].cpu().numpy().astype(np.float64))
+        gv.append(dv_h[bh, 64 * J:64 * J + n].cpu().numpy().astype(np.float64))
+        rk.append(ref_k[b, :n])
+        rv.append(ref_v[b, :n])
+    gk, gv, rk, rv = (np.concatenate(x) for x in (gk, gv, rk, rv))
+    assert np.isfinite(gk).all() and np.isfinite(gv).all()
+    ek, ev = rel_l2(gk, rk), rel_l2(gv, rv)
+    print(f"\nfull-size sampled key blocks: dk rel_l2={ek:.3e} dv rel_l2={ev:.3e}")
+    assert ek <= TOL and ev <= TOL, (ek, ev)

@@ -602,11 +602,30 @@ def pin_backward_rows(lib):
             assert np.array_equal(part[r], full[bh, i]), (ph, topk, bh, i)
 
 
+def pin_backward_key_blocks(lib):
+    """The key-block-sampled dk, dv equal the full backward's rows of those key blocks, bit for bit:
+    subtract and complement selections, both phi, a ragged last key block (N = 210, blk_k = 32: 18 rows),
+    blocks of several heads given out of order, and topk 0 (linear only) and 1 (softmax only)."""
+    q, k, v = _qkv((3, 10, 7), d=32, H=3, seed=46)
+    dout = _qkv((3, 10, 7), d=32, H=3, seed=47)[0]
+    for ph, topk, bq in ((0, 0.3, 64), (1, 0.7, 32), (0, 0.0, 64), (1, 1.0, 32)):
+        _, dk, dv = oracle.backward(q, k, v, dout, bq, 32, topk, phi=ph, lib=lib)
+        blocks = np.array([[2, 6], [0, 0], [1, 3], [0, 5], [2, 0]], dtype=np.int64)
+        pk, pv = oracle.backward_dkdv_blocks(q, k, v, dout, bq, 32, topk, blocks, phi=ph, lib=lib)
+        fk, fv = dk.reshape(-1, 210, 32), dv.reshape(-1, 210, 32)
+        for b, (bh, J) in enumerate(blocks):
+            n = min(32, 210 - 32 * J)
+            assert np.array_equal(pk[b, :n], fk[bh, 32 * J:32 * J + n]), (ph, topk, bh, J)
+            assert np.array_equal(pv[b, :n], fv[bh, 32 * J:32 * J + n]), (ph, topk, bh, J)
+            assert not pk[b, n:].any() and not pv[b, n:].any()
+
+
 PINS = [pin_topk_count, pin_mask_exhaustive, pin_mask_invariances, pin_mask_degenerate,
         pin_quant_exact_block, pin_quant_bounds, pin_quant_smoothing, pin_forward_dense_limit,
         pin_forward_linear_limit, pin_forward_bruteforce, pin_forward_constant_v, pin_forward_hull,
         pin_forward_relu_zero, pin_forward_rows, pin_fp8_encoder, pin_fp8_quant, pin_fp8_forward, pin_w8a8_rowquant, pin_w8a8_linear,
-        pin_backward_autograd, pin_backward_dense_limit, pin_backward_linear_limit, pin_backward_rows]
+        pin_backward_autograd, pin_backward_dense_limit, pin_backward_linear_limit, pin_backward_rows,
+        pin_backward_key_blocks]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
