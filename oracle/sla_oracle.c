@@ -888,7 +888,7 @@ int orc_backward_dkdv_blocks(const uint16_t *q, const uint16_t *k, const uint16_
             for (int I = 0; I < n_qb; ++I) {
                 if (!HI || !ZI || !vec) continue;
                 unselected_state(idx + (size_t)I * k_sel, k_sel, n_kb, d, h, z, HI, ZI);
-                double *dHI = dH + (size_t)I * dd, *dZI = dZ + (size_t)I * d;
+                double *dH_I = dH + (size_t)I * dd, *dZ_I = dZ + (size_t)I * d;
                 double *qi = vec, *doi = vec + d, *f = vec + 3 * d, *a = vec + 4 * d, *ol = vec + 5 * d,
                        *da = vec + 6 * d;
                 int i1 = (I + 1) * blk_q < N ? (I + 1) * blk_q : N;
@@ -910,11 +910,11 @@ int orc_backward_dkdv_blocks(const uint16_t *q, const uint16_t *k, const uint16_
                     }
                     double dol = 0.0;
                     for (int e = 0; e < d; ++e) dol += doi[e] * ol[e];
-                    double db = -dol / b;
+                    double g_b = -dol / b;
                     for (int e = 0; e < d; ++e) da[e] = doi[e] / b;
                     for (int c = 0; c < d; ++c) {
-                        for (int e = 0; e < d; ++e) dHI[(size_t)c * d + e] += f[c] * da[e];
-                        dZI[c] += f[c] * db;
+                        for (int e = 0; e < d; ++e) dH_I[(size_t)c * d + e] += f[c] * da[e];
+                        dZ_I[c] += f[c] * g_b;
                     }
                 }
             }
@@ -998,19 +998,19 @@ int orc_backward_dkdv_blocks(const uint16_t *q, const uint16_t *k, const uint16_
             memset(G, 0, sizeof(double) * dd);
             memset(gz, 0, sizeof(double) * (size_t)d);
             for (int I = 0; I < n_qb; ++I) {
-                if (selected[(size_t)I * n_kb + J]) continue;
+                if (selected[(size_t)I * n_kb + J] != 0) continue;
                 for (size_t e = 0; e < dd; ++e) G[e] += dH[(size_t)I * dd + e];
                 for (int c = 0; c < d; ++c) gz[c] += dZ[(size_t)I * d + c];
             }
             for (int j = t0; j < t1; ++j) {
                 for (int c = 0; c < d; ++c) {
                     double kc = bf(kh[(size_t)j * d + c]), fk = phi_f(kc, phi);
-                    double dfk = gz[c];
+                    double dkf = gz[c];
                     for (int e = 0; e < d; ++e) {
-                        dfk += G[(size_t)c * d + e] * bf(vh[(size_t)j * d + e]);
+                        dkf += G[(size_t)c * d + e] * bf(vh[(size_t)j * d + e]);
                         dvb[(size_t)(j - t0) * d + e] += G[(size_t)c * d + e] * fk;
                     }
-                    dkb[(size_t)(j - t0) * d + c] += dfk * dphi_f(kc, phi);
+                    dkb[(size_t)(j - t0) * d + c] += dkf * dphi_f(kc, phi);
                 }
             }
         }

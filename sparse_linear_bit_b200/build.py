@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsla.so")
-SOURCES = ["sla_api.cu", "sla_mask_quant.cu", "sla_linear.cu", "sla_attention.cu", "sla_noalloc.cu", "sla_w8a8.cu", "sla_ulysses.cu", "sla_backward.cu", "sla_bwd_sparse.cu"]
+SOURCES = ["sla_api.cu", "sla_mask_quant.cu", "sla_linear.cu", "sla_attention.cu", "sla_noalloc.cu", "sla_w8a8.cu", "sla_ulysses.cu", "sla_backward.cu", "sla_bwd_tc.cu"]
 HEADERS = ["sla_internal.h", "sla_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

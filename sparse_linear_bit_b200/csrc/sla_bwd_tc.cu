@@ -1,4 +1,4 @@
-// sla_bwd_sparse.cu -- the softmax branch of the SageSLA backward on tcgen05
+// sla_bwd_tc.cu -- the softmax branch of the SageSLA backward on tcgen05
 // tensor cores (SLA fine-tuning: the jiqiren.org.cn TurboDiffusion article,
 // 方法论; the "TurboDiffusion" summary page, 主要能力: SLA white-box training).
 //
@@ -533,14 +533,26 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const float c = kLog2e * kRsd;
         BitWalk walk(bits, words);
         bool ok = true;
+        // this row's statistics in query block I (rows of the next query block when blk_q = 64, and
+        // rows past N, take none); loaded one tile ahead of use
+        auto stats = [&](int I, float &m, float &il, float &D) {
+            const int i = I * blk_q + r;
+            const bool rv = I >= 0 && r < blk_q && i < N;
+            const size_t si = (size_t)bh * N + (rv ? i : 0);
+            m = rv ? __ldg(st_m + si) : 0.0f;
+            il = rv ? __ldg(st_l + si) : 0.0f;  // 0 for rows that take no part: P = 0
+            D = rv ? __ldg(st_D + si) : 0.0f;
+        };
+        int I_next = walk.next();
+        float m_n, il_n, D_n;
+        stats(I_next, m_n, il_n, D_n);
         for (int t = 0; ok && t < n_sel; ++t) {
-            const int I = walk.next(), b = t & 1;
+            const int I = I_next, b = t & 1;
+            const float m = m_n, il = il_n, D = D_n;
+            I_next = t + 1 < n_sel ? walk.next() : -1;
+            stats(I_next, m_n, il_n, D_n);
             const int i = I * blk_q + r;
             const bool row_valid = r < blk_q && i < N;  // rows of the next query block (blk_q = 64) excluded
-            const size_t si = (size_t)bh * N + (row_valid ? i : 0);
-            const float m = row_valid ? __ldg(st_m + si) : 0.0f;
-            const float il = row_valid ? __ldg(st_l + si) : 0.0f;
-            const float D = row_valid ? __ldg(st_D + si) : 0.0f;
             const int valid = row_valid ? kv : 0;
             if (!(ok = wait_all(&sm.bar_sd[b], (t >> 1) & 1))) break;
             tc_fence_after();
@@ -596,6 +608,350 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 }
 
+// ---------------------------------------------------------------------------
+// linear branch.  Row i of query block I, f = phi(q_i), b = f . Z_I, a = f H_I,
+// ol = a / b (zero when b = 0), da = do / b, db = -(do . ol) / b:
+//   dq_i += (H_I da + Z_I db) phi'(q_i);  dH_I = sum_i f (outer) da;  dZ_I = sum_i f db;
+// and for key block J, with G_J, g_J the sums of dH_I, dZ_I over the query blocks
+// that did not select J:  dk_j = (G_J v_j + g_J) phi'(k_j);  dv_j = G_J^T phi(k_j).
+// The d x d products run as bf16 tcgen05 MMAs with fp32 accumulation; the operand
+// tiles are written by the threads in the 128-byte-swizzled layout, [rows x 128 B]
+// boxes of 64 bf16 (two boxes per 128 columns).
+// ---------------------------------------------------------------------------
+constexpr int kLinThreads = 128;
+
+SLA_DEV float phi_lin(float x, int phi)
+{
+    if (phi == 1) return fmaxf(x, 0.0f);
+    const float e = ex2f(fminf(x, 0.0f) * kLog2e);
+    return x > 0.0f ? x + 1.0f : e;
+}
+
+SLA_DEV float dphi_lin(float x, int phi)
+{
+    if (phi == 1) return x > 0.0f ? 1.0f : 0.0f;
+    const float e = ex2f(fminf(x, 0.0f) * kLog2e);
+    return x > 0.0f ? 1.0f : e;
+}
+
+// row r of a [rows x 128 bf16] operand (two [rows x 128 B] boxes `box` bytes apart): element c = val(c)
+template <class F>
+SLA_DEV void store_row128(uint8_t *tile, uint32_t box, int r, F val)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = pack_bf16x2(val(64 * h + 2 * e), val(64 * h + 2 * e + 1));
+        store_row_sw128(tile + h * box, r, w);
+    }
+}
+
+// element (r, c) of a [rows x 128 bf16] operand written by store_row128
+SLA_DEV float load_elem128(const uint8_t *tile, uint32_t box, int r, int c)
+{
+    const uint16_t *p = reinterpret_cast<const uint16_t *>(tile + (c >> 6) * box + sw128_off(r, (c & 63) >> 3)) + (c & 7);
+    return __uint_as_float((uint32_t)*p << 16);
+}
+
+struct LqSmem {
+    alignas(1024) uint8_t h[2 * kTile];   // H_I^T as [dim e][channel c] bf16 (K-major B of a = F H; MN-major B of H da)
+    alignas(1024) uint8_t f[2 * kTile];   // F = phi(Q_I) as [row i][channel c] (K-major A of a; MN-major A of dH)
+    alignas(1024) uint8_t da[2 * kTile];  // dA as [row i][dim e] (K-major A of H da; MN-major B of dH)
+    float z[128], db[128];
+    uint64_t bar_a, bar_d;
+    uint32_t tmem_base;
+};
+
+// query side: dq (added to the softmax branch's), dH_I and dZ_I (fp32 and bf16)
+__global__ void __launch_bounds__(kLinThreads, 2)
+bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dout, const float *__restrict__ hq,
+                int N, int blk_q, int n_qb, int phi, float *__restrict__ dq, float *__restrict__ dh32,
+                uint16_t *__restrict__ dh16, int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    LqSmem &sm = *reinterpret_cast<LqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int I = blockIdx.x, bh = blockIdx.y;
+    const int r = tid, i = I * blk_q + r;
+    const bool row_valid = r < blk_q && i < N;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (tid == 0) {
+        mbar_init(&sm.bar_a, 1);
+        mbar_init(&sm.bar_d, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 256);
+        tmem_relinquish();
+    }
+    // H_I^T row e = tid, and Z_I
+    const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
+    store_row128(sm.h, kTile, tid, [&](int c) { return __ldg(hrow + (size_t)tid * 128 + c); });
+    sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
+    // this thread's Q and dO rows (16-byte units re-read from L1/L2 where they are used)
+    const uint4 *qs = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
+    const uint4 *ds = reinterpret_cast<const uint4 *>(dout + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
+    auto unit = [&](const uint4 *src, int u, float (&x)[8]) {  // channels 8u .. 8u+7 (zeros past the rows)
+        const uint4 w = row_valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            x[2 * e] = __uint_as_float(ww[e] << 16);
+            x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+        }
+    };
+    __syncthreads();  // z visible
+    // F row (zero past the block's rows) and b = f . Z_I
+    float b = 0.0f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t w[32];
+#pragma unroll
+        for (int uu = 0; uu < 8; ++uu) {
+            float x[8];
+            unit(qs, 8 * h + uu, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                x[e] = row_valid ? phi_lin(x[e], phi) : 0.0f;
+                b = fmaf(x[e], sm.z[64 * h + 8 * uu + e], b);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w[4 * uu + e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        }
+        store_row_sw128(sm.f + h * kTile, r, w);
+    }
+    const float binv = (row_valid && b != 0.0f) ? 1.0f / b : 0.0f;
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base, t_a = tmem, t_d = tmem + 128;  // a then dH at 0; dF at 128
+    // a = F H_I: M = 128 rows, N = 128 dims, K = 128 channels
+    if (tid == 0) {
+        constexpr uint32_t id = idesc(1, 1, 1, 0, 0, 128, 128);
+        const uint64_t fd = sdesc_sw128(smem_u32(sm.f), 16, 1024), hd = sdesc_sw128(smem_u32(sm.h), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t off = (k >> 2) * kTile + (k & 3) * 32;
+            mma_bf16(t_a, dadd(fd, off), dadd(hd, off), id, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.bar_a);
+    }
+    // ol = a / b, db = -(do . ol) / b, da = do / b
+    bool ok = mbar_wait_quiet(&sm.bar_a, 0, status);
+    ok = __all_sync(0xffffffffu, ok);
+    float db = 0.0f;
+    if (ok) {
+        tc_fence_after();
+        float dot = 0.0f;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t a[32];
+            tmem_ld32(t_a + lane_off + c0, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int uu = 0; uu < 4; ++uu) {
+                float x[8];
+                unit(ds, (c0 >> 3) + uu, x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dot = fmaf(x[e], __uint_as_float(a[8 * uu + e]), dot);
+            }
+        }
+        db = -(dot * binv) * binv;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t w[32];
+#pragma unroll
+            for (int uu = 0; uu < 8; ++uu) {
+                float x[8];
+                unit(ds, 8 * h + uu, x);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[4 * uu + e] = pack_bf16x2(x[2 * e] * binv, x[2 * e + 1] * binv);
+            }
+            store_row_sw128(sm.da + h * kTile, r, w);
+        }
+    }
+    sm.db[tid] = db;
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // dF = dA H_I^T (N = 128 channels: H_I^T as an MN-major B) and dH = F^T dA (M = 128 channels,
+    // N = 128 dims, K = 128 rows: both operands MN-major), into the dF and a columns
+    if (tid == 0 && ok) {
+        constexpr uint32_t id_df = idesc(1, 1, 1, 0, 1, 128, 128), id_dh = idesc(1, 1, 1, 1, 1, 128, 128);
+        const uint64_t dad = sdesc_sw128(smem_u32(sm.da), 16, 1024);
+        const uint64_t hmn = sdesc_sw128(smem_u32(sm.h), kTile, 1024);
+        const uint64_t fmn = sdesc_sw128(smem_u32(sm.f), kTile, 1024), damn = sdesc_sw128(smem_u32(sm.da), kTile, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // K-step of 16 dims: 32 B of a dA row, 16 rows (2 KB) of H_I^T
+            mma_bf16(t_d, dadd(dad, (k >> 2) * kTile + (k & 3) * 32), dadd(hmn, 2048 * k), id_df, k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // K-step of 16 rows
+            mma_bf16(t_a, dadd(fmn, 2048 * k), dadd(damn, 2048 * k), id_dh, k > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_d);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_quiet(&sm.bar_d, 0, status));
+    if (ok) {
+        tc_fence_after();
+        // dq_i += (dF + Z_I db) phi'(q_i); the warp-collective TMEM loads run on every lane
+        float *drow = dq + ((size_t)bh * N + (row_valid ? i : 0)) * 128;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t a[32];
+            tmem_ld32(t_d + lane_off + c0, a);
+            tmem_wait_ld();
+            if (row_valid) {
+                float4 *o = reinterpret_cast<float4 *>(drow + c0);
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) {
+                    float x[8];
+                    unit(qs, (c0 >> 3) + uu, x);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int e = 8 * uu + 4 * hh;
+                        float4 v = o[2 * uu + hh];
+                        v.x += fmaf(sm.z[c0 + e], db, __uint_as_float(a[e])) * dphi_lin(x[4 * hh], phi);
+                        v.y += fmaf(sm.z[c0 + e + 1], db, __uint_as_float(a[e + 1])) * dphi_lin(x[4 * hh + 1], phi);
+                        v.z += fmaf(sm.z[c0 + e + 2], db, __uint_as_float(a[e + 2])) * dphi_lin(x[4 * hh + 2], phi);
+                        v.w += fmaf(sm.z[c0 + e + 3], db, __uint_as_float(a[e + 3])) * dphi_lin(x[4 * hh + 3], phi);
+                        o[2 * uu + hh] = v;
+                    }
+                }
+            }
+        }
+        // dH (TMEM lane = channel c = tid, column = dim e) stored as dH^T [e][c]; dZ_I[c] = sum_i F[i][c] db_i
+        float *d32 = dh32 + ((size_t)bh * n_qb + I) * kStateCols;
+        uint16_t *d16 = dh16 + ((size_t)bh * n_qb + I) * kStateCols;
+        const int c = tid;
+#pragma unroll 1
+        for (int e0 = 0; e0 < 128; e0 += 32) {
+            uint32_t a[32];
+            tmem_ld32(t_a + lane_off + e0, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float x = __uint_as_float(a[e]);
+                d32[(size_t)(e0 + e) * 128 + c] = x;
+                d16[(size_t)(e0 + e) * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+            }
+        }
+        float dz = 0.0f;
+        for (int rr = 0; rr < 128; ++rr) dz = fmaf(load_elem128(sm.f, kTile, rr, c), sm.db[rr], dz);
+        d32[128 * 128 + c] = dz;
+        d16[128 * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(dz));
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+struct LkSmem {
+    alignas(1024) uint8_t g[2 * kTile];   // G_J^T as [dim e][channel c] bf16 (MN-major A of G v; K-major A of G^T phi(k))
+    alignas(1024) uint8_t v[2 * kBox];    // V_J as [key j][dim e] (K-major B of G v)
+    alignas(1024) uint8_t fk[2 * kBox];   // phi(K_J) as [key j][channel c] (K-major B of G^T phi(k))
+    float gz[128];
+    uint64_t bar;
+    uint32_t tmem_base;
+};
+
+// key side: dk, dv of the linear branch, written (the softmax branch's key side adds to them)
+__global__ void __launch_bounds__(kLinThreads, 3)
+bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, const float *__restrict__ G, int N,
+                int n_kb, int phi, float *__restrict__ dk, float *__restrict__ dv, int *status)
+{
+    extern __shared__ uint8_t smem_raw[];
+    LkSmem &sm = *reinterpret_cast<LkSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int J = blockIdx.x, bh = blockIdx.y;
+    const int t0 = J * 64, kv = min(64, N - t0);
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (tid == 0) {
+        mbar_init(&sm.bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 128);
+        tmem_relinquish();
+    }
+    const float *grow = G + ((size_t)bh * n_kb + J) * kStateCols;
+    store_row128(sm.g, kTile, tid, [&](int c) { return __ldg(grow + (size_t)tid * 128 + c); });
+    sm.gz[tid] = __ldg(grow + 128 * 128 + tid);
+    {
+        // thread -> (key row j = tid % 64, half h = tid / 64 of its 128 columns): V and phi(K) rows
+        const int j = tid & 63, h = tid >> 6;
+        const bool ok = j < kv;
+        const uint4 *vs = reinterpret_cast<const uint4 *>(v + ((size_t)bh * N + t0 + (ok ? j : 0)) * 128 + 64 * h);
+        const uint4 *ks = reinterpret_cast<const uint4 *>(k + ((size_t)bh * N + t0 + (ok ? j : 0)) * 128 + 64 * h);
+        uint32_t wv[32], wk[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint4 a = ok ? __ldg(vs + u) : make_uint4(0, 0, 0, 0);
+            const uint4 c = ok ? __ldg(ks + u) : make_uint4(0, 0, 0, 0);
+            wv[4 * u] = a.x; wv[4 * u + 1] = a.y; wv[4 * u + 2] = a.z; wv[4 * u + 3] = a.w;
+            const uint32_t cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = ok ? phi_lin(__uint_as_float(cc[e] << 16), phi) : 0.0f;
+                const float hi = ok ? phi_lin(__uint_as_float(cc[e] & 0xFFFF0000u), phi) : 0.0f;
+                wk[4 * u + e] = pack_bf16x2(lo, hi);
+            }
+        }
+        store_row_sw128(sm.v + h * kBox, j, wv);
+        store_row_sw128(sm.fk + h * kBox, j, wk);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base, t_k = tmem, t_v = tmem + 64;
+    if (tid == 0) {
+        // T^T = G V^T: M = 128 channels, N = 64 keys, K = 128 dims (A = G_J^T tile read MN-major);
+        // dV^T = G^T phi(K)^T: M = 128 dims, N = 64 keys, K = 128 channels (A K-major)
+        constexpr uint32_t id_k = idesc(1, 1, 1, 1, 0, 128, 64), id_v = idesc(1, 1, 1, 0, 0, 128, 64);
+        const uint64_t gmn = sdesc_sw128(smem_u32(sm.g), kTile, 1024), gk = sdesc_sw128(smem_u32(sm.g), 16, 1024);
+        const uint64_t vd = sdesc_sw128(smem_u32(sm.v), 16, 1024), fd = sdesc_sw128(smem_u32(sm.fk), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(t_k, dadd(gmn, 2048 * kk), dadd(vd, (kk >> 2) * kBox + (kk & 3) * 32), id_k, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+            mma_bf16(t_v, dadd(gk, (kk >> 2) * kTile + (kk & 3) * 32), dadd(fd, (kk >> 2) * kBox + (kk & 3) * 32), id_v,
+                     kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar);
+    }
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_quiet(&sm.bar, 0, status));
+    if (ok) {
+        tc_fence_after();
+        const int c = tid;  // TMEM lane: channel c (dk) and dim c (dv)
+        uint32_t a[64];
+        tmem_ld64(t_k + lane_off, a);
+        tmem_wait_ld();
+        const size_t base = ((size_t)bh * N + t0) * 128 + c;
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            if (j < kv) {
+                const float kc = __uint_as_float((uint32_t)k[base + (size_t)j * 128] << 16);
+                dk[base + (size_t)j * 128] = (__uint_as_float(a[j]) + sm.gz[c]) * dphi_lin(kc, phi);
+            }
+        tmem_ld64(t_v + lane_off, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            if (j < kv) dv[base + (size_t)j * 128] = __uint_as_float(a[j]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
 // 3-D map [BH, N, 128] of a bf16 tensor, boxes of 64 channels x `rows` rows
 bool map_rows(CUtensorMap *m, const void *base, const Geometry &g, uint32_t rows)
 {
@@ -637,6 +993,30 @@ cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, c
     if (e != cudaSuccess) return e;
     bwdk_kernel<<<dim3(g.n_kb, g.BH), kBwThreads, smem, s>>>(tq, tdo, tk, tv, selT, n_awT, st_m, st_l, st_D, g.N,
                                                              g.blk_q, g.n_qb, g.n_kb, dk, dv, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_query_linear(const void *q, const void *dout, const float *hq, const Geometry &g, int phi,
+                                    float *dq, float *dh32, uint16_t *dh16, int *status, cudaStream_t s)
+{
+    const size_t smem = sizeof(LqSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_qlin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_qlin_kernel<<<dim3(g.n_qb, g.BH), kLinThreads, smem, s>>>(static_cast<const uint16_t *>(q),
+                                                                  static_cast<const uint16_t *>(dout), hq, g.N,
+                                                                  g.blk_q, g.n_qb, phi, dq, dh32, dh16, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_key_linear(const void *k, const void *v, const float *G, const Geometry &g, int phi, float *dk,
+                                  float *dv, int *status, cudaStream_t s)
+{
+    const size_t smem = sizeof(LkSmem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_klin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_klin_kernel<<<dim3(g.n_kb, g.BH), kLinThreads, smem, s>>>(static_cast<const uint16_t *>(k),
+                                                                  static_cast<const uint16_t *>(v), G, g.N, g.n_kb,
+                                                                  phi, dk, dv, status);
     return cudaGetLastError();
 }
 

@@ -63,7 +63,8 @@ cudaError_t launch_attention(const void *q, const void *k, const void *v, const 
 size_t backward_workspace_bytes(const Geometry &g);
 cudaError_t launch_backward(const void *q, const void *k, const void *v, const void *dout, float *dq, float *dk,
                             float *dv, const Geometry &g, int phi, void *ws, cudaStream_t s);
-// the softmax branch of the backward on the tensor cores (sla_bwd_sparse.cu): the query side writes
+// the softmax branch of the backward on the tensor cores (sla_bwd_tc.cu, as the linear branch's
+// kernels below): the query side writes
 // dq and the row statistics (max m, 1/l, D); the key side adds to dk, dv
 cudaError_t launch_bwd_query_sparse(const void *q, const void *k, const void *v, const void *dout,
                                     const int32_t *idx, const float *kmean, const Geometry &g, float *dq,
@@ -72,6 +73,12 @@ cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, c
                                   const uint32_t *selT, int n_awT, const float *st_m, const float *st_l,
                                   const float *st_D, const Geometry &g, float *dk, float *dv, int *status,
                                   cudaStream_t s);
+// the linear branch of the backward on the tensor cores: the query side adds to dq and writes dH, dZ
+// (fp32 and bf16); the key side writes dk, dv
+cudaError_t launch_bwd_query_linear(const void *q, const void *dout, const float *hq, const Geometry &g, int phi,
+                                    float *dq, float *dh32, uint16_t *dh16, int *status, cudaStream_t s);
+cudaError_t launch_bwd_key_linear(const void *k, const void *v, const float *G, const Geometry &g, int phi, float *dk,
+                                  float *dv, int *status, cudaStream_t s);
 // TMA descriptor encoding (driver entry point fetched once through the runtime)
 // W8A8 linear layer (sla_w8a8.cu)
 cudaError_t launch_rowquant(const void *x, int rows, int cols, int norm, const float *gamma, float eps, int8_t *q,
