@@ -82,14 +82,14 @@ SLA_DEV void store_row_sw128(uint8_t *tile, int r, const uint32_t (&w)[32])
 SLA_DEV void issue_s_dp(uint32_t t_s, uint32_t t_dp, uint64_t qd, uint64_t dod, uint64_t kd, uint64_t vd)
 {
     constexpr uint32_t id = idesc(1, 1, 1, 0, 0, 128, 64);  // f32 <- bf16 x bf16
+    // the two accumulation chains alternate, so that one chain's MMA overlaps the other's
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < 8; ++k) {
         mma_bf16(t_s, dadd(qd, (k >> 2) * kTile + (k & 3) * 32), dadd(kd, (k >> 2) * kBox + (k & 3) * 32), id,
                  k > 0 ? 1u : 0u);
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
         mma_bf16(t_dp, dadd(dod, (k >> 2) * kTile + (k & 3) * 32), dadd(vd, (k >> 2) * kBox + (k & 3) * 32), id,
                  k > 0 ? 1u : 0u);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -500,22 +500,47 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const uint64_t pmn = sdesc_sw128(smem_u32(sm.p[b]), kTile, 1024);
                 const uint64_t dsmn = sdesc_sw128(smem_u32(sm.ds[b]), kTile, 1024);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)  // K-step of 16 query rows: 2 KB of each tile
+                for (int k = 0; k < 8; ++k) {  // K-step of 16 query rows: 2 KB of each tile; the chains alternate
                     mma_bf16(t_dv, dadd(domn, 2048 * k), dadd(pmn, 2048 * k), id_acc, (t > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
                     mma_bf16(t_dk, dadd(qmn, 2048 * k), dadd(dsmn, 2048 * k), id_acc, (t > 0 || k > 0) ? 1u : 0u);
+                }
                 mma_commit(&sm.bar_pdfree[b]);
                 mma_commit(&sm.empty[s]);  // Q and dO of the stage are no longer read
                 if (t == n_sel - 1) mma_commit(&sm.bar_acc);
             }
             __syncwarp();
         };
-        for (int t = 0; ok && t < n_sel; ++t) {
-            issue_sd(t);
-            if (ok && t >= 1) issue_acc(t - 1);
+        // S/dP of tile t may run ahead of the accumulation of tile t-1 by one tile (two S/dP
+        // buffers); between them, whichever is ready first is issued first: the accumulation frees
+        // a Q/dO stage for the producer, S/dP feeds the row threads
+        int n_sd = 0, n_acc = 0;
+        long long t0c = clock64();
+        const long long budget = wait_budget();
+        while (ok && n_acc < n_sel) {
+            const bool can_acc = n_acc < n_sd && mbar_test(&sm.bar_pd[n_acc & 1], (n_acc >> 1) & 1);
+            if (__any_sync(0xffffffffu, can_acc)) {
+                issue_acc(n_acc++);
+                t0c = clock64();
+                continue;
+            }
+            const bool can_sd = n_sd < n_sel && n_sd <= n_acc + 1 &&
+                                mbar_test(&sm.full[n_sd % kBkStages], (n_sd / kBkStages) & 1) &&
+                                (n_sd < 2 || mbar_test(&sm.bar_sdfree[n_sd & 1], ((n_sd >> 1) - 1) & 1));
+            if (__any_sync(0xffffffffu, can_sd)) {
+                issue_sd(n_sd++);
+                t0c = clock64();
+                continue;
+            }
+            if (clock64() - t0c > budget) {  // neither came: the same bounded-wait rule as mbar_wait
+                if (elect_one()) record_error(status, kStatusTimeout);
+                *abort_flag = 1;
+                ok = false;
+            } else if (global_failed(status) || *abort_flag) {
+                *abort_flag = 1;
+                ok = false;
+            }
+            ok = __all_sync(0xffffffffu, ok);
         }
-        if (ok) issue_acc(n_sel - 1);
         if (elect_one()) {
             mma_commit(&sm.drain);
             mbar_wait_quiet(&sm.drain, 0, status);
@@ -617,6 +642,18 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // The d x d products run as bf16 tcgen05 MMAs with fp32 accumulation; the operand
 // tiles are written by the threads in the 128-byte-swizzled layout, [rows x 128 B]
 // boxes of 64 bf16 (two boxes per 128 columns).
+//
+// Centring.  When the values share a common component, H_I da and Z_I db nearly
+// cancel in dq (H_I ~ Z_I (outer) mean value), and so do G_J v_j and g_J in dk; bf16
+// operands would then carry errors relative to the large terms.  Both sides are
+// therefore evaluated with centred operands, which is exact algebra: for any vector
+// mu, with H' = H_I - Z_I (outer) mu, a' = f H', ol = a' / b + mu, and
+//   H_I da + Z_I db = H' da + Z_I db',  db' = -(da . a') / b,  db = db' - da . mu;
+// the kernel takes mu_e = (sum_c Z_c H[c][e]) / (sum_c Z_c^2), the least-squares fit
+// of H_I by Z_I (outer) mu, and rounds H' to bf16 (dZ_I still uses the true db).  On
+// the key side, with nu the key block's mean value row,
+//   G_J v_j + g_J = G_J (v_j - nu) + (g_J + G_J nu),
+// where the second term is summed in fp32.
 // ---------------------------------------------------------------------------
 constexpr int kLinThreads = 128;
 
@@ -658,7 +695,7 @@ struct LqSmem {
     alignas(1024) uint8_t h[2 * kTile];   // H_I^T as [dim e][channel c] bf16 (K-major B of a = F H; MN-major B of H da)
     alignas(1024) uint8_t f[2 * kTile];   // F = phi(Q_I) as [row i][channel c] (K-major A of a; MN-major A of dH)
     alignas(1024) uint8_t da[2 * kTile];  // dA as [row i][dim e] (K-major A of H da; MN-major B of dH)
-    float z[128], db[128];
+    float z[128], db[128], mu[128];
     uint64_t bar_a, bar_d;
     uint32_t tmem_base;
 };
@@ -685,10 +722,21 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         tmem_alloc(&sm.tmem_base, 256);
         tmem_relinquish();
     }
-    // H_I^T row e = tid, and Z_I
+    // Z_I, then row e = tid of the centred H'^T = H_I^T - mu (outer) Z_I
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
-    store_row128(sm.h, kTile, tid, [&](int c) { return __ldg(hrow + (size_t)tid * 128 + c); });
     sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
+    __syncthreads();
+    {
+        const float *he = hrow + (size_t)tid * 128;
+        float zh = 0.0f, zz = 0.0f;
+        for (int c = 0; c < 128; ++c) {
+            zh = fmaf(sm.z[c], __ldg(he + c), zh);
+            zz = fmaf(sm.z[c], sm.z[c], zz);
+        }
+        const float mu = zz > 0.0f ? zh / zz : 0.0f;
+        sm.mu[tid] = mu;
+        store_row128(sm.h, kTile, tid, [&](int c) { return fmaf(-mu, sm.z[c], __ldg(he + c)); });
+    }
     // this thread's Q and dO rows (16-byte units re-read from L1/L2 where they are used)
     const uint4 *qs = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
     const uint4 *ds = reinterpret_cast<const uint4 *>(dout + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
@@ -701,7 +749,6 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
             x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
         }
     };
-    __syncthreads();  // z visible
     // F row (zero past the block's rows) and b = f . Z_I
     float b = 0.0f;
 #pragma unroll
@@ -758,7 +805,7 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
                 for (int e = 0; e < 8; ++e) dot = fmaf(x[e], __uint_as_float(a[8 * uu + e]), dot);
             }
         }
-        db = -(dot * binv) * binv;
+        db = -(dot * binv) * binv;  // db' of the centred state; the true db is db' - da . mu
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t w[32];
@@ -772,7 +819,17 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
             store_row_sw128(sm.da + h * kTile, r, w);
         }
     }
-    sm.db[tid] = db;
+    {
+        float dmu = 0.0f;  // da . mu, for the true db that dZ_I takes
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            float x[8];
+            unit(ds, u, x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dmu = fmaf(x[e] * binv, sm.mu[8 * u + e], dmu);
+        }
+        sm.db[tid] = ok ? db - dmu : 0.0f;
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -852,9 +909,9 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
 
 struct LkSmem {
     alignas(1024) uint8_t g[2 * kTile];   // G_J^T as [dim e][channel c] bf16 (MN-major A of G v; K-major A of G^T phi(k))
-    alignas(1024) uint8_t v[2 * kBox];    // V_J as [key j][dim e] (K-major B of G v)
+    alignas(1024) uint8_t v[2 * kBox];    // V_J - nu as [key j][dim e] (K-major B of G v)
     alignas(1024) uint8_t fk[2 * kBox];   // phi(K_J) as [key j][channel c] (K-major B of G^T phi(k))
-    float gz[128];
+    float gz[128], nu[128], gp[128];      // g_J, the block's mean value row nu, g_J + G_J nu
     uint64_t bar;
     uint32_t tmem_base;
 };
@@ -881,8 +938,16 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
     const float *grow = G + ((size_t)bh * n_kb + J) * kStateCols;
     store_row128(sm.g, kTile, tid, [&](int c) { return __ldg(grow + (size_t)tid * 128 + c); });
     sm.gz[tid] = __ldg(grow + 128 * 128 + tid);
+    // nu = the block's mean value row (dims e = tid), in fp32 from the bf16 rows
     {
-        // thread -> (key row j = tid % 64, half h = tid / 64 of its 128 columns): V and phi(K) rows
+        const int e = tid;
+        float sv = 0.0f;
+        for (int j = 0; j < kv; ++j) sv += __uint_as_float((uint32_t)v[((size_t)bh * N + t0 + j) * 128 + e] << 16);
+        sm.nu[e] = sv / (float)kv;
+    }
+    __syncthreads();
+    {
+        // thread -> (key row j = tid % 64, half h = tid / 64 of its 128 columns): V - nu and phi(K) rows
         const int j = tid & 63, h = tid >> 6;
         const bool ok = j < kv;
         const uint4 *vs = reinterpret_cast<const uint4 *>(v + ((size_t)bh * N + t0 + (ok ? j : 0)) * 128 + 64 * h);
@@ -892,10 +957,13 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         for (int u = 0; u < 8; ++u) {
             const uint4 a = ok ? __ldg(vs + u) : make_uint4(0, 0, 0, 0);
             const uint4 c = ok ? __ldg(ks + u) : make_uint4(0, 0, 0, 0);
-            wv[4 * u] = a.x; wv[4 * u + 1] = a.y; wv[4 * u + 2] = a.z; wv[4 * u + 3] = a.w;
-            const uint32_t cc[4] = {c.x, c.y, c.z, c.w};
+            const uint32_t aa[4] = {a.x, a.y, a.z, a.w}, cc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
+                const int d0 = 64 * h + 8 * u + 2 * e;
+                const float vlo = ok ? __uint_as_float(aa[e] << 16) - sm.nu[d0] : 0.0f;
+                const float vhi = ok ? __uint_as_float(aa[e] & 0xFFFF0000u) - sm.nu[d0 + 1] : 0.0f;
+                wv[4 * u + e] = pack_bf16x2(vlo, vhi);
                 const float lo = ok ? phi_lin(__uint_as_float(cc[e] << 16), phi) : 0.0f;
                 const float hi = ok ? phi_lin(__uint_as_float(cc[e] & 0xFFFF0000u), phi) : 0.0f;
                 wk[4 * u + e] = pack_bf16x2(lo, hi);
@@ -903,6 +971,13 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         }
         store_row_sw128(sm.v + h * kBox, j, wv);
         store_row_sw128(sm.fk + h * kBox, j, wk);
+    }
+    // g' = g_J + G_J nu (fp32): channel c = tid, G_J[c][e] = G_J^T[e][c]
+    {
+        const int c = tid;
+        float gg = sm.gz[c];
+        for (int e = 0; e < 128; ++e) gg = fmaf(__ldg(grow + (size_t)e * 128 + c), sm.nu[e], gg);
+        sm.gp[c] = gg;
     }
     fence_async_smem();
     tc_fence_before();
@@ -936,7 +1011,7 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         for (int j = 0; j < 64; ++j)
             if (j < kv) {
                 const float kc = __uint_as_float((uint32_t)k[base + (size_t)j * 128] << 16);
-                dk[base + (size_t)j * 128] = (__uint_as_float(a[j]) + sm.gz[c]) * dphi_lin(kc, phi);
+                dk[base + (size_t)j * 128] = (__uint_as_float(a[j]) + sm.gp[c]) * dphi_lin(kc, phi);
             }
         tmem_ld64(t_v + lane_off, a);
         tmem_wait_ld();
