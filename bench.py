@@ -501,7 +501,7 @@ def main():
         bwd = {"ms": ms_b, "what": "dq, dk, dv (fp32) of the unquantised forward for a random dout",
                "roofline": {"bound": "tensor", "achieved": ach, "peak": p_bf16, "unit": "TFLOP/s",
                             "frac": ach / p_bf16, "peak_source": f"{peak_kind} bf16 {p_bf16} TFLOP/s (burst)",
-                            "note": "softmax-branch products as tcgen05 bf16 MMAs (fp32 accumulation in tensor memory); the linear branch in fp32 on the CUDA cores"},
+                            "note": "every product (softmax and linear branches) as tcgen05 bf16 MMAs with fp32 accumulation in tensor memory"},
                "flops_per_call": fl_sparse + fl_lin}
         del dout, grads, wsb
 
