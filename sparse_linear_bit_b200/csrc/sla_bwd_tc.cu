@@ -722,20 +722,33 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         tmem_alloc(&sm.tmem_base, 256);
         tmem_relinquish();
     }
-    // Z_I, then row e = tid of the centred H'^T = H_I^T - mu (outer) Z_I
+    // Z_I, then the centred H'^T = H_I^T - mu (outer) Z_I: each warp takes 32 rows e, one coalesced
+    // 512-byte row per load (lane: channels 4 lane .. 4 lane + 3)
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
     sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
     __syncthreads();
     {
-        const float *he = hrow + (size_t)tid * 128;
-        float zh = 0.0f, zz = 0.0f;
-        for (int c = 0; c < 128; ++c) {
-            zh = fmaf(sm.z[c], __ldg(he + c), zh);
-            zz = fmaf(sm.z[c], sm.z[c], zz);
+        const int lane = tid & 31, c0 = 4 * lane;
+        const float4 zc = make_float4(sm.z[c0], sm.z[c0 + 1], sm.z[c0 + 2], sm.z[c0 + 3]);
+        float zz = zc.x * zc.x + zc.y * zc.y + zc.z * zc.z + zc.w * zc.w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
+        float4 hv = __ldg(reinterpret_cast<const float4 *>(hrow + (size_t)(warp * 32) * 128) + lane);
+#pragma unroll 1
+        for (int rr = 0; rr < 32; ++rr) {
+            const int e = warp * 32 + rr;
+            const float4 h = hv;
+            if (rr + 1 < 32) hv = __ldg(reinterpret_cast<const float4 *>(hrow + (size_t)(e + 1) * 128) + lane);
+            float zh = zc.x * h.x + zc.y * h.y + zc.z * h.z + zc.w * h.w;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) zh += __shfl_xor_sync(0xffffffffu, zh, o);
+            const float mu = zz > 0.0f ? zh / zz : 0.0f;
+            if (lane == 0) sm.mu[e] = mu;
+            // channels c0 .. c0 + 3 of row e: box c0 / 64, 16-byte unit (c0 % 64) / 8, half (c0 % 8) / 4
+            uint2 *dst = reinterpret_cast<uint2 *>(sm.h + (c0 >> 6) * kTile + sw128_off(e, (c0 & 63) >> 3) + (c0 & 7) * 2);
+            *dst = make_uint2(pack_bf16x2(fmaf(-mu, zc.x, h.x), fmaf(-mu, zc.y, h.y)),
+                              pack_bf16x2(fmaf(-mu, zc.z, h.z), fmaf(-mu, zc.w, h.w)));
         }
-        const float mu = zz > 0.0f ? zh / zz : 0.0f;
-        sm.mu[tid] = mu;
-        store_row128(sm.h, kTile, tid, [&](int c) { return fmaf(-mu, sm.z[c], __ldg(he + c)); });
     }
     // this thread's Q and dO rows (16-byte units re-read from L1/L2 where they are used)
     const uint4 *qs = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
@@ -936,7 +949,17 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         tmem_relinquish();
     }
     const float *grow = G + ((size_t)bh * n_kb + J) * kStateCols;
-    store_row128(sm.g, kTile, tid, [&](int c) { return __ldg(grow + (size_t)tid * 128 + c); });
+    {
+        // G_J^T rows e: each warp takes 32, one coalesced 512-byte row per load (lane: 4 channels)
+        const int lane = tid & 31, c0 = 4 * lane;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr) {
+            const int e = warp * 32 + rr;
+            const float4 g = __ldg(reinterpret_cast<const float4 *>(grow + (size_t)e * 128) + lane);
+            uint2 *dst = reinterpret_cast<uint2 *>(sm.g + (c0 >> 6) * kTile + sw128_off(e, (c0 & 63) >> 3) + (c0 & 7) * 2);
+            *dst = make_uint2(pack_bf16x2(g.x, g.y), pack_bf16x2(g.z, g.w));
+        }
+    }
     sm.gz[tid] = __ldg(grow + 128 * 128 + tid);
     // nu = the block's mean value row (dims e = tid), in fp32 from the bf16 rows
     {

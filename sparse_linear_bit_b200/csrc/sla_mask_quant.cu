@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_warp_kernel(const double
 // row, the pooled mean that block selection scores with (exact fp64 sums, so the
 // same values as the pooling kernel's).
 template <bool SMOOTH, int BLK, bool FP8>
-__global__ void __launch_bounds__(256, 4) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
+__global__ void __launch_bounds__(256) quant_kernel(const uint4 *__restrict__ x, int N, int nb,
                                                     const float *__restrict__ mean, uint2 *__restrict__ out,
                                                     float *__restrict__ scale, double *__restrict__ bmean)
 {
