@@ -247,8 +247,10 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         named_bar_sync(1, 128);
         const float c = kLog2e * kRsd;
         bool ok = true;
-        // ---- pass 1: row max m, sum l and D = sum p dP (online, in log2 units)
+        // ---- pass 1: row max m, sum l and D = sum p dP (online, in log2 units; m is raised only when
+        // the tile's max exceeds it by more than 2^8, so p stays below 256 and most tiles need no rescale)
         float m = -INFINITY, l = 0.0f, Dt = 0.0f;
+        const uint64_t c2 = f2pack(c, c);
         for (int t = 0; ok && t < k_sel; ++t) {
             const int T = t, b = T & 1;
             const int J = __ldg(sel + t), valid = min(64, N - J * 64);
@@ -260,24 +262,38 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_sdfree[b]);
-            float tmax = -INFINITY;
+            if (valid < 64) {  // the ragged last key block: its missing keys take no part
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < valid) tmax = fmaxf(tmax, __uint_as_float(sv[j]) * c);
-            const float mn = fmaxf(m, tmax);
-            const float alpha = ex2f(m - mn);  // 0 while m = -inf
-            l *= alpha;
-            Dt *= alpha;
-            m = mn;
-            float ls = 0.0f, ds = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const float p = j < valid ? ex2f(__uint_as_float(sv[j]) * c - m) : 0.0f;
-                ls += p;
-                ds = fmaf(p, __uint_as_float(dv[j]), ds);
+                for (int j = 0; j < 64; ++j)
+                    if (j >= valid) sv[j] = __float_as_uint(-INFINITY);
             }
-            l += ls;
-            Dt += ds;
+            float tt[22];
+#pragma unroll
+            for (int j = 0; j < 21; ++j)
+                tt[j] = fmax3f(__uint_as_float(sv[3 * j]), __uint_as_float(sv[3 * j + 1]), __uint_as_float(sv[3 * j + 2]));
+            tt[21] = __uint_as_float(sv[63]);
+#pragma unroll
+            for (int j = 0; j < 7; ++j) tt[j] = fmax3f(tt[3 * j], tt[3 * j + 1], tt[3 * j + 2]);
+            const float tmax =
+                fmax3f(fmax3f(tt[0], tt[1], tt[2]), fmax3f(tt[3], tt[4], tt[5]), fmaxf(tt[6], tt[21])) * c;  // c > 0
+            if (tmax > m + 8.0f) {  // also on the first tile (m = -inf)
+                const float alpha = ex2f(m - tmax);  // 0 while m = -inf
+                l *= alpha;
+                Dt *= alpha;
+                m = tmax;
+            }
+            const uint64_t nm2 = f2pack(-m, -m);
+            uint64_t ls2 = 0, ds2 = 0;
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+                const float2 a = f2unpack(fma2(f2pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2, nm2));
+                const uint64_t p2 = f2pack(ex2f(a.x), ex2f(a.y));  // masked keys: ex2(-inf) = 0
+                ls2 = add2(ls2, p2);
+                ds2 = fma2(p2, f2pack(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), ds2);
+            }
+            const float2 ls = f2unpack(ls2), dsum = f2unpack(ds2);
+            l += ls.x + ls.y;
+            Dt += dsum.x + dsum.y;
         }
         const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
         const float D = Dt * inv_l;
@@ -299,17 +315,26 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_sdfree[b]);
+            if (valid < 64) {  // missing keys of the last block, and rows past the block: dS = 0
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (j >= valid) sv[j] = __float_as_uint(-INFINITY);
+            }
+            // dS = p (dP - D) / sqrt(d) with p = 2^(s c - m) / l, in packed pairs
+            const uint64_t nm2 = f2pack(-m, -m), il2 = f2pack(inv_l * kRsd, inv_l * kRsd), nd2 = f2pack(-D, -D);
             uint32_t w[32];
+            uint64_t sg2 = 0;
 #pragma unroll
             for (int j = 0; j < 64; j += 2) {
-                float g[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float p = (j + h) < valid ? ex2f(__uint_as_float(sv[j + h]) * c - m) * inv_l : 0.0f;
-                    g[h] = p * (__uint_as_float(dv[j + h]) - D) * kRsd;
-                }
-                w[j >> 1] = pack_bf16x2(g[0], g[1]);
-                sigma += __uint_as_float(w[j >> 1] << 16) + __uint_as_float(w[j >> 1] & 0xFFFF0000u);
+                const float2 a = f2unpack(fma2(f2pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2, nm2));
+                const uint64_t p2 = mul2(f2pack(ex2f(a.x), ex2f(a.y)), il2);
+                const float2 g = f2unpack(mul2(p2, add2(f2pack(__uint_as_float(dv[j]), __uint_as_float(dv[j + 1])), nd2)));
+                w[j >> 1] = pack_bf16x2(g.x, g.y);
+                sg2 = add2(sg2, f2pack(__uint_as_float(w[j >> 1] << 16), __uint_as_float(w[j >> 1] & 0xFFFF0000u)));
+            }
+            {
+                const float2 sg = f2unpack(sg2);
+                sigma += sg.x + sg.y;
             }
             if (t >= 2 && !(ok = wait_all(&sm.bar_dsfree[bd], ((t >> 1) - 1) & 1))) break;
             store_row_sw128(sm.ds[bd], r, w);
@@ -722,32 +747,34 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         tmem_alloc(&sm.tmem_base, 256);
         tmem_relinquish();
     }
-    // Z_I, then the centred H'^T = H_I^T - mu (outer) Z_I: each warp takes 32 rows e, one coalesced
-    // 512-byte row per load (lane: channels 4 lane .. 4 lane + 3)
+    // Z_I, then row e = tid of the centred H'^T = H_I^T - mu (outer) Z_I (16-byte loads of the row;
+    // its second pass hits L1)
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
     sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
     __syncthreads();
     {
-        const int lane = tid & 31, c0 = 4 * lane;
-        const float4 zc = make_float4(sm.z[c0], sm.z[c0 + 1], sm.z[c0 + 2], sm.z[c0 + 3]);
-        float zz = zc.x * zc.x + zc.y * zc.y + zc.z * zc.z + zc.w * zc.w;
+        const float4 *he = reinterpret_cast<const float4 *>(hrow + (size_t)tid * 128);
+        float zh = 0.0f, zz = 0.0f;
+#pragma unroll 8
+        for (int u = 0; u < 32; ++u) {
+            const float4 h = __ldg(he + u);
+            zh = fmaf(sm.z[4 * u], h.x, fmaf(sm.z[4 * u + 1], h.y, fmaf(sm.z[4 * u + 2], h.z, fmaf(sm.z[4 * u + 3], h.w, zh))));
+            zz = fmaf(sm.z[4 * u], sm.z[4 * u], fmaf(sm.z[4 * u + 1], sm.z[4 * u + 1],
+                      fmaf(sm.z[4 * u + 2], sm.z[4 * u + 2], fmaf(sm.z[4 * u + 3], sm.z[4 * u + 3], zz))));
+        }
+        const float mu = zz > 0.0f ? zh / zz : 0.0f;
+        sm.mu[tid] = mu;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) zz += __shfl_xor_sync(0xffffffffu, zz, o);
-        float4 hv = __ldg(reinterpret_cast<const float4 *>(hrow + (size_t)(warp * 32) * 128) + lane);
-#pragma unroll 1
-        for (int rr = 0; rr < 32; ++rr) {
-            const int e = warp * 32 + rr;
-            const float4 h = hv;
-            if (rr + 1 < 32) hv = __ldg(reinterpret_cast<const float4 *>(hrow + (size_t)(e + 1) * 128) + lane);
-            float zh = zc.x * h.x + zc.y * h.y + zc.z * h.z + zc.w * h.w;
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t w[32];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) zh += __shfl_xor_sync(0xffffffffu, zh, o);
-            const float mu = zz > 0.0f ? zh / zz : 0.0f;
-            if (lane == 0) sm.mu[e] = mu;
-            // channels c0 .. c0 + 3 of row e: box c0 / 64, 16-byte unit (c0 % 64) / 8, half (c0 % 8) / 4
-            uint2 *dst = reinterpret_cast<uint2 *>(sm.h + (c0 >> 6) * kTile + sw128_off(e, (c0 & 63) >> 3) + (c0 & 7) * 2);
-            *dst = make_uint2(pack_bf16x2(fmaf(-mu, zc.x, h.x), fmaf(-mu, zc.y, h.y)),
-                              pack_bf16x2(fmaf(-mu, zc.z, h.z), fmaf(-mu, zc.w, h.w)));
+            for (int u = 0; u < 16; ++u) {
+                const float4 h = __ldg(he + 16 * hh + u);
+                const int c = 64 * hh + 4 * u;
+                w[2 * u] = pack_bf16x2(fmaf(-mu, sm.z[c], h.x), fmaf(-mu, sm.z[c + 1], h.y));
+                w[2 * u + 1] = pack_bf16x2(fmaf(-mu, sm.z[c + 2], h.z), fmaf(-mu, sm.z[c + 3], h.w));
+            }
+            store_row_sw128(sm.h + hh * kTile, tid, w);
         }
     }
     // this thread's Q and dO rows (16-byte units re-read from L1/L2 where they are used)

@@ -430,6 +430,12 @@ SLA_DEV uint64_t add2(uint64_t a, uint64_t b)
     asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+SLA_DEV uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 
 // byte offset of 16-byte chunk `u` (0..7) of row `r` inside a tile of 128-byte
 // rows stored with the 128-byte swizzle (tile base 1024-byte aligned)
