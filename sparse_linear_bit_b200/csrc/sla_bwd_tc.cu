@@ -717,28 +717,38 @@ SLA_DEV float load_elem128(const uint8_t *tile, uint32_t box, int r, int c)
 }
 
 struct LqSmem {
-    alignas(1024) uint8_t h[2 * kTile];   // H_I^T as [dim e][channel c] bf16 (K-major B of a = F H; MN-major B of H da)
-    alignas(1024) uint8_t f[2 * kTile];   // F = phi(Q_I) as [row i][channel c] (K-major A of a; MN-major A of dH)
-    alignas(1024) uint8_t da[2 * kTile];  // dA as [row i][dim e] (K-major A of H da; MN-major B of dH)
+    alignas(1024) uint8_t hs[4 * kTile];  // H_I^T fp32 as loaded (4 boxes [128 dims x 32 channels]); later dq staging
+    alignas(1024) uint8_t qr[2 * kTile];  // raw Q rows of the query block (bf16, [rows x 64 channels] boxes)
+    alignas(1024) uint8_t da[2 * kTile];  // dO rows as loaded, then dA in place ([row i][dim e]: K-major A of H da,
+                                          // MN-major B of dH)
+    alignas(1024) uint8_t f[2 * kTile];   // F = phi(Q_I) [row i][channel c] (K-major A of a; MN-major A of dH)
+    alignas(1024) uint8_t h[2 * kTile];   // centred H'^T [dim e][channel c] (K-major B of a; MN-major B of H da)
     float z[128], db[128], mu[128];
-    uint64_t bar_a, bar_d;
+    uint64_t bar_ld, bar_a, bar_d;
     uint32_t tmem_base;
 };
 
-// query side: dq (added to the softmax branch's), dH_I and dZ_I (fp32 and bf16)
-__global__ void __launch_bounds__(kLinThreads, 2)
-bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dout, const float *__restrict__ hq,
-                int N, int blk_q, int n_qb, int phi, float *__restrict__ dq, float *__restrict__ dh32,
-                uint16_t *__restrict__ dh16, int *status)
+// byte offset of fp32 element c of row r in a tile of four [rows x 32 fp32] boxes with the 128-byte swizzle
+SLA_DEV uint32_t f32_off(int r, int c) { return (c >> 5) * kTile + sw128_off(r, (c & 31) >> 2) + (c & 3) * 4; }
+
+// query side: dq (added to the softmax branch's), dH_I and dZ_I (fp32 and bf16).  Every operand arrives by
+// TMA (H_I, the Q and dO rows); the dq update goes through shared memory so that its global accesses are
+// whole coalesced rows.
+__global__ void __launch_bounds__(kLinThreads, 1)
+bwd_qlin_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant__ CUtensorMap tm_q,
+                const __grid_constant__ CUtensorMap tm_do, const float *__restrict__ hq, int N, int blk_q, int n_qb,
+                int phi, float *__restrict__ dq, float *__restrict__ dh32, uint16_t *__restrict__ dh16, int *status)
 {
     extern __shared__ uint8_t smem_raw[];
     LqSmem &sm = *reinterpret_cast<LqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int I = blockIdx.x, bh = blockIdx.y;
     const int r = tid, i = I * blk_q + r;
-    const bool row_valid = r < blk_q && i < N;
+    const int rows = min(blk_q, N - I * blk_q);
+    const bool row_valid = r < rows;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     if (tid == 0) {
+        mbar_init(&sm.bar_ld, 1);
         mbar_init(&sm.bar_a, 1);
         mbar_init(&sm.bar_d, 1);
         fence_mbar_init();
@@ -747,41 +757,51 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         tmem_alloc(&sm.tmem_base, 256);
         tmem_relinquish();
     }
-    // Z_I, then row e = tid of the centred H'^T = H_I^T - mu (outer) Z_I (16-byte loads of the row;
-    // its second pass hits L1)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        mbar_expect_tx(&sm.bar_ld, 8 * kTile);
+        for (int c = 0; c < 4; ++c) tma_load_3d(sm.hs + c * kTile, &tm_h, &sm.bar_ld, 32 * c, 0, bh * n_qb + I);
+        for (int c = 0; c < 2; ++c) {
+            tma_load_3d(sm.qr + c * kTile, &tm_q, &sm.bar_ld, 64 * c, I * blk_q, bh);
+            tma_load_3d(sm.da + c * kTile, &tm_do, &sm.bar_ld, 64 * c, I * blk_q, bh);
+        }
+    }
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
     sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
-    __syncthreads();
+    bool ok = __all_sync(0xffffffffu, mbar_wait_quiet(&sm.bar_ld, 0, status));
+    __syncthreads();  // z visible
+    const uint32_t tmem = sm.tmem_base, t_a = tmem, t_d = tmem + 128;  // a then dH at 0; dF at 128
+    // ---- row e = tid of the centred H'^T = H_I^T - mu (outer) Z_I
     {
-        const float4 *he = reinterpret_cast<const float4 *>(hrow + (size_t)tid * 128);
+        const int e = tid;
         float zh = 0.0f, zz = 0.0f;
 #pragma unroll 8
         for (int u = 0; u < 32; ++u) {
-            const float4 h = __ldg(he + u);
+            const float4 h = *reinterpret_cast<const float4 *>(sm.hs + f32_off(e, 4 * u));
             zh = fmaf(sm.z[4 * u], h.x, fmaf(sm.z[4 * u + 1], h.y, fmaf(sm.z[4 * u + 2], h.z, fmaf(sm.z[4 * u + 3], h.w, zh))));
             zz = fmaf(sm.z[4 * u], sm.z[4 * u], fmaf(sm.z[4 * u + 1], sm.z[4 * u + 1],
                       fmaf(sm.z[4 * u + 2], sm.z[4 * u + 2], fmaf(sm.z[4 * u + 3], sm.z[4 * u + 3], zz))));
         }
         const float mu = zz > 0.0f ? zh / zz : 0.0f;
-        sm.mu[tid] = mu;
+        sm.mu[e] = mu;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             uint32_t w[32];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const float4 h = __ldg(he + 16 * hh + u);
                 const int c = 64 * hh + 4 * u;
+                const float4 h = *reinterpret_cast<const float4 *>(sm.hs + f32_off(e, c));
                 w[2 * u] = pack_bf16x2(fmaf(-mu, sm.z[c], h.x), fmaf(-mu, sm.z[c + 1], h.y));
                 w[2 * u + 1] = pack_bf16x2(fmaf(-mu, sm.z[c + 2], h.z), fmaf(-mu, sm.z[c + 3], h.w));
             }
-            store_row_sw128(sm.h + hh * kTile, tid, w);
+            store_row_sw128(sm.h + hh * kTile, e, w);
         }
     }
-    // this thread's Q and dO rows (16-byte units re-read from L1/L2 where they are used)
-    const uint4 *qs = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
-    const uint4 *ds = reinterpret_cast<const uint4 *>(dout + ((size_t)bh * N + (row_valid ? i : 0)) * 128);
-    auto unit = [&](const uint4 *src, int u, float (&x)[8]) {  // channels 8u .. 8u+7 (zeros past the rows)
-        const uint4 w = row_valid ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+    // 8 bf16 channels 8u .. 8u + 7 of row r of a [rows x 128 bf16] tile (two [rows x 64] boxes)
+    auto unit8 = [&](const uint8_t *tile, int u, float (&x)[8]) {
+        const uint4 w = *reinterpret_cast<const uint4 *>(tile + (u >> 3) * kTile + sw128_off(r, u & 7));
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -789,33 +809,32 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
             x[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
         }
     };
-    // F row (zero past the block's rows) and b = f . Z_I
+    // ---- F row (zero past the block's rows) and b = f . Z_I
     float b = 0.0f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int hh = 0; hh < 2; ++hh) {
         uint32_t w[32];
 #pragma unroll
         for (int uu = 0; uu < 8; ++uu) {
             float x[8];
-            unit(qs, 8 * h + uu, x);
+            unit8(sm.qr, 8 * hh + uu, x);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 x[e] = row_valid ? phi_lin(x[e], phi) : 0.0f;
-                b = fmaf(x[e], sm.z[64 * h + 8 * uu + e], b);
+                b = fmaf(x[e], sm.z[64 * hh + 8 * uu + e], b);
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) w[4 * uu + e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
         }
-        store_row_sw128(sm.f + h * kTile, r, w);
+        store_row_sw128(sm.f + hh * kTile, r, w);
     }
     const float binv = (row_valid && b != 0.0f) ? 1.0f / b : 0.0f;
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = sm.tmem_base, t_a = tmem, t_d = tmem + 128;  // a then dH at 0; dF at 128
-    // a = F H_I: M = 128 rows, N = 128 dims, K = 128 channels
-    if (tid == 0) {
+    // a' = F H': M = 128 rows, N = 128 dims, K = 128 channels
+    if (tid == 0 && ok) {
         constexpr uint32_t id = idesc(1, 1, 1, 0, 0, 128, 128);
         const uint64_t fd = sdesc_sw128(smem_u32(sm.f), 16, 1024), hd = sdesc_sw128(smem_u32(sm.h), 16, 1024);
 #pragma unroll
@@ -825,13 +844,12 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         }
         mma_commit(&sm.bar_a);
     }
-    // ol = a / b, db = -(do . ol) / b, da = do / b
-    bool ok = mbar_wait_quiet(&sm.bar_a, 0, status);
-    ok = __all_sync(0xffffffffu, ok);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_quiet(&sm.bar_a, 0, status));
+    // ---- db' = -(do . a') / b^2, dA = do / b (in place of the dO row), and the true db = db' - da . mu
     float db = 0.0f;
     if (ok) {
         tc_fence_after();
-        float dot = 0.0f;
+        float dot = 0.0f, dmu = 0.0f;
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
             uint32_t a[32];
@@ -840,41 +858,36 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
 #pragma unroll
             for (int uu = 0; uu < 4; ++uu) {
                 float x[8];
-                unit(ds, (c0 >> 3) + uu, x);
+                unit8(sm.da, (c0 >> 3) + uu, x);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) dot = fmaf(x[e], __uint_as_float(a[8 * uu + e]), dot);
+                for (int e = 0; e < 8; ++e) {
+                    dot = fmaf(x[e], __uint_as_float(a[8 * uu + e]), dot);
+                    dmu = fmaf(x[e], sm.mu[c0 + 8 * uu + e], dmu);
+                }
             }
         }
-        db = -(dot * binv) * binv;  // db' of the centred state; the true db is db' - da . mu
+        db = -(dot * binv) * binv;  // db' of the centred state
+        sm.db[tid] = db - dmu * binv;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int hh = 0; hh < 2; ++hh) {
             uint32_t w[32];
 #pragma unroll
             for (int uu = 0; uu < 8; ++uu) {
                 float x[8];
-                unit(ds, 8 * h + uu, x);
+                unit8(sm.da, 8 * hh + uu, x);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) w[4 * uu + e] = pack_bf16x2(x[2 * e] * binv, x[2 * e + 1] * binv);
             }
-            store_row_sw128(sm.da + h * kTile, r, w);
+            store_row_sw128(sm.da + hh * kTile, r, w);
         }
-    }
-    {
-        float dmu = 0.0f;  // da . mu, for the true db that dZ_I takes
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            float x[8];
-            unit(ds, u, x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dmu = fmaf(x[e] * binv, sm.mu[8 * u + e], dmu);
-        }
-        sm.db[tid] = ok ? db - dmu : 0.0f;
+    } else {
+        sm.db[tid] = 0.0f;
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // dF = dA H_I^T (N = 128 channels: H_I^T as an MN-major B) and dH = F^T dA (M = 128 channels,
+    // dF = dA H'^T (N = 128 channels: H'^T as an MN-major B) and dH = F^T dA (M = 128 channels,
     // N = 128 dims, K = 128 rows: both operands MN-major), into the dF and a columns
     if (tid == 0 && ok) {
         constexpr uint32_t id_df = idesc(1, 1, 1, 0, 1, 128, 128), id_dh = idesc(1, 1, 1, 1, 1, 128, 128);
@@ -882,43 +895,37 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
         const uint64_t hmn = sdesc_sw128(smem_u32(sm.h), kTile, 1024);
         const uint64_t fmn = sdesc_sw128(smem_u32(sm.f), kTile, 1024), damn = sdesc_sw128(smem_u32(sm.da), kTile, 1024);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // K-step of 16 dims: 32 B of a dA row, 16 rows (2 KB) of H_I^T
+        for (int k = 0; k < 8; ++k) {  // K-step of 16: the two chains alternate
             mma_bf16(t_d, dadd(dad, (k >> 2) * kTile + (k & 3) * 32), dadd(hmn, 2048 * k), id_df, k > 0 ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // K-step of 16 rows
             mma_bf16(t_a, dadd(fmn, 2048 * k), dadd(damn, 2048 * k), id_dh, k > 0 ? 1u : 0u);
+        }
         mma_commit(&sm.bar_d);
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait_quiet(&sm.bar_d, 0, status));
     if (ok) {
         tc_fence_after();
-        // dq_i += (dF + Z_I db) phi'(q_i); the warp-collective TMEM loads run on every lane
-        float *drow = dq + ((size_t)bh * N + (row_valid ? i : 0)) * 128;
+        // dq row delta (dF + Z_I db') phi'(q) into the staging tile (the H_I^T region is free now)
 #pragma unroll 1
         for (int c0 = 0; c0 < 128; c0 += 32) {
             uint32_t a[32];
             tmem_ld32(t_d + lane_off + c0, a);
             tmem_wait_ld();
-            if (row_valid) {
-                float4 *o = reinterpret_cast<float4 *>(drow + c0);
 #pragma unroll
-                for (int uu = 0; uu < 4; ++uu) {
-                    float x[8];
-                    unit(qs, (c0 >> 3) + uu, x);
+            for (int uu = 0; uu < 4; ++uu) {
+                float x[8];
+                unit8(sm.qr, (c0 >> 3) + uu, x);
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int e = 8 * uu + 4 * hh;
-                        float4 v = o[2 * uu + hh];
-                        v.x += fmaf(sm.z[c0 + e], db, __uint_as_float(a[e])) * dphi_lin(x[4 * hh], phi);
-                        v.y += fmaf(sm.z[c0 + e + 1], db, __uint_as_float(a[e + 1])) * dphi_lin(x[4 * hh + 1], phi);
-                        v.z += fmaf(sm.z[c0 + e + 2], db, __uint_as_float(a[e + 2])) * dphi_lin(x[4 * hh + 2], phi);
-                        v.w += fmaf(sm.z[c0 + e + 3], db, __uint_as_float(a[e + 3])) * dphi_lin(x[4 * hh + 3], phi);
-                        o[2 * uu + hh] = v;
-                    }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int e = 8 * uu + 4 * hh, c = c0 + e;
+                    *reinterpret_cast<float4 *>(sm.hs + f32_off(r, c)) = make_float4(
+                        fmaf(sm.z[c], db, __uint_as_float(a[e])) * dphi_lin(x[4 * hh], phi),
+                        fmaf(sm.z[c + 1], db, __uint_as_float(a[e + 1])) * dphi_lin(x[4 * hh + 1], phi),
+                        fmaf(sm.z[c + 2], db, __uint_as_float(a[e + 2])) * dphi_lin(x[4 * hh + 2], phi),
+                        fmaf(sm.z[c + 3], db, __uint_as_float(a[e + 3])) * dphi_lin(x[4 * hh + 3], phi));
                 }
             }
         }
-        // dH (TMEM lane = channel c = tid, column = dim e) stored as dH^T [e][c]; dZ_I[c] = sum_i F[i][c] db_i
+        // dH (TMEM lane = channel c = tid, column = dim e) stored as dH^T [e][c]
         float *d32 = dh32 + ((size_t)bh * n_qb + I) * kStateCols;
         uint16_t *d16 = dh16 + ((size_t)bh * n_qb + I) * kStateCols;
         const int c = tid;
@@ -934,10 +941,24 @@ bwd_qlin_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ dou
                 d16[(size_t)(e0 + e) * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
             }
         }
+        // dZ_I[c] = sum_i F[i][c] db_i
         float dz = 0.0f;
         for (int rr = 0; rr < 128; ++rr) dz = fmaf(load_elem128(sm.f, kTile, rr, c), sm.db[rr], dz);
         d32[128 * 128 + c] = dz;
         d16[128 * 128 + c] = __bfloat16_as_ushort(__float2bfloat16_rn(dz));
+    }
+    __syncthreads();  // the dq deltas are staged
+    if (ok) {
+        // dq += the staged deltas: warp w takes rows 32 w .. 32 w + 31, one coalesced 512-byte row per step
+        for (int rr = 0; rr < 32; ++rr) {
+            const int row = warp * 32 + rr;
+            if (row >= rows) break;
+            float4 *g = reinterpret_cast<float4 *>(dq + ((size_t)bh * N + I * blk_q + row) * 128) + lane;
+            const float4 d = *reinterpret_cast<const float4 *>(sm.hs + f32_off(row, 4 * lane));
+            float4 v = *g;
+            v.x += d.x; v.y += d.y; v.z += d.z; v.w += d.w;
+            *g = v;
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1124,12 +1145,20 @@ cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, c
 cudaError_t launch_bwd_query_linear(const void *q, const void *dout, const float *hq, const Geometry &g, int phi,
                                     float *dq, float *dh32, uint16_t *dh16, int *status, cudaStream_t s)
 {
+    CUtensorMap th, tq, tdo;
+    {
+        // H_I^T of every query block: [BH * n_qb][128 dims][128 channels] fp32 inside rows of kStateCols
+        const uint64_t hd[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)g.BH * g.n_qb};
+        const uint64_t st[2] = {(uint64_t)kD * 4, (uint64_t)kStateCols * 4};
+        const uint32_t bx[3] = {32, 128, 1};
+        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, hd, st, bx)) return cudaErrorInvalidValue;
+    }
+    if (!map_rows(&tq, q, g, 128) || !map_rows(&tdo, dout, g, 128)) return cudaErrorInvalidValue;
     const size_t smem = sizeof(LqSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(bwd_qlin_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_qlin_kernel<<<dim3(g.n_qb, g.BH), kLinThreads, smem, s>>>(static_cast<const uint16_t *>(q),
-                                                                  static_cast<const uint16_t *>(dout), hq, g.N,
-                                                                  g.blk_q, g.n_qb, phi, dq, dh32, dh16, status);
+    bwd_qlin_kernel<<<dim3(g.n_qb, g.BH), kLinThreads, smem, s>>>(th, tq, tdo, hq, g.N, g.blk_q, g.n_qb, phi, dq, dh32,
+                                                                  dh16, status);
     return cudaGetLastError();
 }
 
