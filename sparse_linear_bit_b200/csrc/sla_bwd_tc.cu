@@ -1009,12 +1009,16 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         }
     }
     sm.gz[tid] = __ldg(grow + 128 * 128 + tid);
-    // nu = the block's mean value row (dims e = tid), in fp32 from the bf16 rows
+    // nu = the block's mean value row (dims e = tid), in fp32 from the bf16 rows (the loads are issued
+    // together: a fixed trip count, predicated)
     {
         const int e = tid;
-        float sv = 0.0f;
-        for (int j = 0; j < kv; ++j) sv += __uint_as_float((uint32_t)v[((size_t)bh * N + t0 + j) * 128 + e] << 16);
-        sm.nu[e] = sv / (float)kv;
+        const uint16_t *ve = v + ((size_t)bh * N + t0) * 128 + e;
+        float sv[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+            if (j < kv) sv[j & 7] += __uint_as_float((uint32_t)__ldg(ve + (size_t)j * 128) << 16);
+        sm.nu[e] = (((sv[0] + sv[1]) + (sv[2] + sv[3])) + ((sv[4] + sv[5]) + (sv[6] + sv[7]))) / (float)kv;
     }
     __syncthreads();
     {
@@ -1043,12 +1047,13 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         store_row_sw128(sm.v + h * kBox, j, wv);
         store_row_sw128(sm.fk + h * kBox, j, wk);
     }
-    // g' = g_J + G_J nu (fp32): channel c = tid, G_J[c][e] = G_J^T[e][c]
+    // g' = g_J + G_J nu (fp32): channel c = tid, G_J[c][e] = G_J^T[e][c] (coalesced across the warp)
     {
         const int c = tid;
-        float gg = sm.gz[c];
-        for (int e = 0; e < 128; ++e) gg = fmaf(__ldg(grow + (size_t)e * 128 + c), sm.nu[e], gg);
-        sm.gp[c] = gg;
+        float gg[4] = {sm.gz[c], 0.0f, 0.0f, 0.0f};
+#pragma unroll 32
+        for (int e = 0; e < 128; ++e) gg[e & 3] = fmaf(__ldg(grow + (size_t)e * 128 + c), sm.nu[e], gg[e & 3]);
+        sm.gp[c] = (gg[0] + gg[1]) + (gg[2] + gg[3]);
     }
     fence_async_smem();
     tc_fence_before();
