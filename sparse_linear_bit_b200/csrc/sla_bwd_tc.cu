@@ -743,7 +743,7 @@ bwd_qlin_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant_
     LqSmem &sm = *reinterpret_cast<LqSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int I = blockIdx.x, bh = blockIdx.y;
-    const int r = tid, i = I * blk_q + r;
+    const int r = tid;
     const int rows = min(blk_q, N - I * blk_q);
     const bool row_valid = r < rows;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;

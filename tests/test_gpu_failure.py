@@ -11,6 +11,12 @@ waits from its start until the last key block is done -- so the call must:
 * return (no hang), with sla_check reporting SLA_ERR_TIMEOUT;
 * leave the context usable: a following call on the SAME workspace with the default
   budget reports SLA_OK and matches the oracle (cosine >= 0.999, relative L2 <= 2e-2).
+
+The same holds for the backward, whose tensor-core kernels (the forward's states and
+state reduction, and the softmax branch's query and key sides) wait the same bounded
+way: with a one-cycle budget sla_backward must report SLA_ERR_TIMEOUT and return, and a
+following call on the same workspace must match the oracle's gradients (relative L2
+<= 5e-3, the backward's bar).
 """
 from __future__ import annotations
 
@@ -54,6 +60,32 @@ def test_short_wait_budget_times_out_cleanly_and_the_workspace_recovers():
     ref = oracle.forward(q, k, v, blk_q, 64, float(np.float32(topk)), phi=0, quant=1)
     r, c = rel_l2(got, ref), cosine(got, ref)
     assert r <= 2e-2 and c >= 0.999, (r, c)
+
+
+def test_short_wait_budget_in_the_backward_times_out_cleanly_and_recovers():
+    B, H, grid, blk_q, topk = 1, 2, (8, 16, 16), 128, 0.25  # N = 2048: 8 selected of 32 key blocks
+    q, k, v = synth.make_qkv(B, H, grid, seed=93)
+    dout = synth.make_qkv(B, H, grid, seed=94)[0]
+    N, d = q.shape[2], q.shape[3]
+    qd, kd, vd, dod = (to_dev(x, torch) for x in (q, k, v, dout))
+    grads = [torch.zeros(B, H, N, d, dtype=torch.float32, device="cuda") for _ in range(3)]
+    ws = sla.backward_workspace(B, H, N, d, blk_q, 64, topk)
+    sla.sla_set_wait_budget(1)
+    try:
+        sla.sla_backward(qd, kd, vd, dod, *grads, blk_q, 64, topk, 0, ws)
+        with pytest.raises(sla.SlaError) as err:
+            sla.sla_check(ws)
+        assert sla.sla_status_string(err.value.code) == "SLA_ERR_TIMEOUT"
+    finally:
+        sla.sla_set_wait_budget(0)
+    torch.cuda.synchronize()
+
+    sla.sla_backward(qd, kd, vd, dod, *grads, blk_q, 64, topk, 0, ws)
+    sla.sla_check(ws)
+    ref = oracle.backward(q, k, v, dout, blk_q, 64, float(np.float32(topk)), phi=0)
+    for g, r in zip(grads, ref):
+        err = rel_l2(g.cpu().numpy().astype(np.float64), r)
+        assert err <= 5e-3, err
 
 
 def test_wait_budget_argument_checks():
