@@ -26,9 +26,11 @@
 //   the results are added to dk, dv, which the linear branch's key side has
 //   written before.
 //
-// Roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// warps 2-5 one row per thread (query rows; in bwdk's epilogue, dims).  All
-// products take bf16 operands with fp32 accumulation.  Every wait is bounded
+// Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, then the row
+// warps: in bwdq (192 threads) warps 2-5, one query row per thread; in bwdk (320
+// threads) warps 2-9, two threads per query row, each with half of the tile's 64
+// keys (in bwdk's epilogue, one dim or channel per pair, half of the keys each).
+// All products take bf16 operands with fp32 accumulation.  Every wait is bounded
 // (see sla_ptx.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,6 +45,7 @@ namespace sla {
 namespace {
 
 constexpr int kBwThreads = 192;
+constexpr int kBkThreads = 320;
 constexpr uint32_t kBox = 64 * 128;    // [64 rows x 128 B]
 constexpr uint32_t kTile = 128 * 128;  // [128 rows x 128 B]
 constexpr int kBqStages = 3;
@@ -410,7 +413,7 @@ struct BitWalk {
     }
 };
 
-__global__ void __launch_bounds__(kBwThreads, 1)
+__global__ void __launch_bounds__(kBkThreads, 1)
 bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
             const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
             const uint32_t *__restrict__ selT, int n_awT, const float *__restrict__ st_m,
@@ -441,8 +444,8 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         mbar_init(&sm.bar_kv, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.bar_sd[b], 1);
-            mbar_init(&sm.bar_sdfree[b], 128);
-            mbar_init(&sm.bar_pd[b], 128);
+            mbar_init(&sm.bar_sdfree[b], 256);
+            mbar_init(&sm.bar_pd[b], 256);
             mbar_init(&sm.bar_pdfree[b], 1);
         }
         mbar_init(&sm.bar_acc, 1);
@@ -504,9 +507,7 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const uint64_t kd = sdesc_sw128(smem_u32(sm.k), 16, 1024), vd = sdesc_sw128(smem_u32(sm.v), 16, 1024);
         bool ok = mbar_wait_warp(&sm.bar_kv, 0, status, abort_flag);
         auto issue_sd = [&](int t) {
-            const int s = t % kBkStages, b = t & 1;
-            if (!(ok = mbar_wait_warp(&sm.full[s], (t / kBkStages) & 1, status, abort_flag))) return;
-            if (t >= 2 && !(ok = mbar_wait_warp(&sm.bar_sdfree[b], ((t >> 1) - 1) & 1, status, abort_flag))) return;
+            const int s = t % kBkStages, b = t & 1;  // both phases were seen complete by the poll
             tc_fence_after();
             if (elect_one()) {
                 issue_s_dp(tmem + 128 * b, tmem + 128 * b + 64, sdesc_sw128(smem_u32(sm.qd[s]), 16, 1024),
@@ -516,8 +517,7 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             __syncwarp();
         };
         auto issue_acc = [&](int t) {
-            const int s = t % kBkStages, b = t & 1;
-            if (!(ok = mbar_wait_warp(&sm.bar_pd[b], (t >> 1) & 1, status, abort_flag))) return;
+            const int s = t % kBkStages, b = t & 1;  // the phase was seen complete by the poll
             tc_fence_after();
             if (elect_one()) {
                 const uint64_t qmn = sdesc_sw128(smem_u32(sm.qd[s]), kTile, 1024);
@@ -573,7 +573,8 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         __syncwarp();
     } else {
         // ------------------------------------------------------------ rows (query rows; dims at the end)
-        const int quarter = warp & 3;
+        // warps 2-5 take keys 0-31 of their rows, warps 6-9 keys 32-63
+        const int quarter = warp & 3, half = (warp - 2) >> 2, j0 = 32 * half;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         auto wait_all = [&](uint64_t *bar, uint32_t par) {
@@ -606,27 +607,38 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int valid = row_valid ? kv : 0;
             if (!(ok = wait_all(&sm.bar_sd[b], (t >> 1) & 1))) break;
             tc_fence_after();
-            uint32_t sv[64], dpv[64];
-            tmem_ld64(tmem + 128 * b + lane_off, sv);
-            tmem_ld64(tmem + 128 * b + 64 + lane_off, dpv);
+            uint32_t sv[32], dpv[32];
+            tmem_ld32(tmem + 128 * b + j0 + lane_off, sv);
+            tmem_ld32(tmem + 128 * b + 64 + j0 + lane_off, dpv);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&sm.bar_sdfree[b]);
-            uint32_t wp[32], wd[32];
+            uint32_t wp[16], wd[16];
+            if (valid < j0 + 32) {  // keys past the block's end (the ragged last block), or a row that takes no part
 #pragma unroll
-            for (int j = 0; j < 64; j += 2) {
-                float p[2], g[2];
+                for (int j = 0; j < 32; ++j)
+                    if (j0 + j >= valid) sv[j] = __float_as_uint(-INFINITY);
+            }
+            const uint64_t c2 = f2pack(c, c), nm2 = f2pack(-m, -m), il2 = f2pack(il, il), nd2 = f2pack(-D, -D);
+            const uint64_t rs2 = f2pack(kRsd, kRsd);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    p[h] = (j + h) < valid ? ex2f(__uint_as_float(sv[j + h]) * c - m) * il : 0.0f;
-                    g[h] = p[h] * (__uint_as_float(dpv[j + h]) - D) * kRsd;
-                }
-                wp[j >> 1] = pack_bf16x2(p[0], p[1]);
-                wd[j >> 1] = pack_bf16x2(g[0], g[1]);
+            for (int j = 0; j < 32; j += 2) {
+                const float2 a = f2unpack(fma2(f2pack(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), c2, nm2));
+                const uint64_t p2 = mul2(f2pack(ex2f(a.x), ex2f(a.y)), il2);
+                const uint64_t g2 = mul2(mul2(p2, add2(f2pack(__uint_as_float(dpv[j]), __uint_as_float(dpv[j + 1])), nd2)), rs2);
+                const float2 p = f2unpack(p2), g = f2unpack(g2);
+                wp[j >> 1] = pack_bf16x2(p.x, p.y);
+                wd[j >> 1] = pack_bf16x2(g.x, g.y);
             }
             if (t >= 2 && !(ok = wait_all(&sm.bar_pdfree[b], ((t >> 1) - 1) & 1))) break;
-            store_row_sw128(sm.p[b], r, wp);
-            store_row_sw128(sm.ds[b], r, wd);
+            // this thread's 64 bytes of row r: 16-byte units 4 half .. 4 half + 3
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                *reinterpret_cast<uint4 *>(sm.p[b] + sw128_off(r, 4 * half + u)) =
+                    make_uint4(wp[4 * u], wp[4 * u + 1], wp[4 * u + 2], wp[4 * u + 3]);
+                *reinterpret_cast<uint4 *>(sm.ds[b] + sw128_off(r, 4 * half + u)) =
+                    make_uint4(wd[4 * u], wd[4 * u + 1], wd[4 * u + 2], wd[4 * u + 3]);
+            }
             fence_async_smem();
             mbar_arrive(&sm.bar_pd[b]);
         }
@@ -634,19 +646,19 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (ok) ok = wait_all(&sm.bar_acc, 0);
         if (ok) {
             tc_fence_after();
-            uint32_t a[64];
-            tmem_ld64(t_dv + lane_off, a);
+            uint32_t a[32];
+            tmem_ld32(t_dv + j0 + lane_off, a);
             tmem_wait_ld();
-            float *pv = dv + ((size_t)bh * N + t0) * 128 + r;
+            float *pv = dv + ((size_t)bh * N + t0 + j0) * 128 + r;
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < kv) pv[(size_t)j * 128] += __uint_as_float(a[j]);
-            tmem_ld64(t_dk + lane_off, a);
+            for (int j = 0; j < 32; ++j)
+                if (j0 + j < kv) pv[(size_t)j * 128] += __uint_as_float(a[j]);
+            tmem_ld32(t_dk + j0 + lane_off, a);
             tmem_wait_ld();
-            float *pk = dk + ((size_t)bh * N + t0) * 128 + r;
+            float *pk = dk + ((size_t)bh * N + t0 + j0) * 128 + r;
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (j < kv) pk[(size_t)j * 128] += __uint_as_float(a[j]);
+            for (int j = 0; j < 32; ++j)
+                if (j0 + j < kv) pk[(size_t)j * 128] += __uint_as_float(a[j]);
         }
     }
     tc_fence_before();
@@ -1142,7 +1154,7 @@ cudaError_t launch_bwd_key_sparse(const void *q, const void *k, const void *v, c
     const size_t smem = sizeof(BkSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(bwdk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwdk_kernel<<<dim3(g.n_kb, g.BH), kBwThreads, smem, s>>>(tq, tdo, tk, tv, selT, n_awT, st_m, st_l, st_D, g.N,
+    bwdk_kernel<<<dim3(g.n_kb, g.BH), kBkThreads, smem, s>>>(tq, tdo, tk, tv, selT, n_awT, st_m, st_l, st_D, g.N,
                                                              g.blk_q, g.n_qb, g.n_kb, dk, dv, status);
     return cudaGetLastError();
 }
