@@ -365,85 +365,54 @@ def main():
     ops = dense_equiv_ops(wl.B, wl.H, wl.N, wl.d)  # this rank's share
     value = ops_job / (ms * 1e-3) / 1e12
 
-    # ---- end to end through the public call: pinned host Q/K/V in, bf16 out back to pinned host.
-    # Every (batch, head) is an independent problem, so a step runs the workload as chunks of
-    # consecutive heads on three streams: the copy-in of chunk c+1 and the copy-out of chunk c-1
-    # overlap sla_forward on chunk c.  The step's result equals one call over the whole workload.
+    # ---- end to end through the C-ABI call that takes HOST buffers (sla_forward_host): pinned host
+    # Q/K/V in, bf16 output back to pinned host memory, every copy inside the timed region.  The call
+    # runs the (batch, head) problems in chunks of consecutive heads on three streams of its own, so
+    # that the copy-in of chunk c+1 and the copy-out of chunk c-1 overlap the forward of chunk c; its
+    # result equals one device call over the whole workload.
     e2e = None
     if not a.no_e2e:
         hq_, hk_, hv_ = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in (q, k, v))
         hout = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
         steps_e2e = max(2, min(a.steps, 5))
-        BHn = wl.B * wl.H
-        n_chunks = min(8, BHn)
-        bounds = [(BHn * c) // n_chunks for c in range(n_chunks + 1)]
-        flat = lambda t: t.reshape(BHn, wl.N, wl.d)
-        s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ws_chunk = sla.workspace(1, max(bounds[c + 1] - bounds[c] for c in range(n_chunks)), wl.N, wl.d, wl.blk_q,
-                                 wl.blk_k, a.topk, a.quant, device=dev)
-
-        # per chunk: its inputs landed (in), its forward done (done), its output copied out (out);
-        # the next step's copy-in of a chunk waits for this step's forward on it, and the next
-        # step's forward for this step's copy-out, so buffers are reused in order
-        ev = {nm: [None] * n_chunks for nm in ("in", "done", "out")}
+        n_chunks = min(8, wl.B * wl.H)
+        chunk_heads = -(-(wl.B * wl.H) // n_chunks)
+        dev_host = sla.host_workspace(wl.B, wl.H, wl.N, wl.d, wl.blk_q, wl.blk_k, a.topk, a.quant, chunk_heads,
+                                      device=dev)
+        s_e2e = torch.cuda.current_stream(dev)
 
         def e2e_step():
-            for c in range(n_chunks):
-                h0, h1 = bounds[c], bounds[c + 1]
-                if ev["done"][c] is not None:
-                    s_in.wait_event(ev["done"][c])
-                with torch.cuda.stream(s_in):
-                    for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_)):
-                        flat(dst)[h0:h1].copy_(flat(src)[h0:h1], non_blocking=True)
-                ev["in"][c] = torch.cuda.Event()
-                ev["in"][c].record(s_in)
-            for c in range(n_chunks):
-                h0, h1 = bounds[c], bounds[c + 1]
-                s_cmp.wait_event(ev["in"][c])
-                if ev["out"][c] is not None:
-                    s_cmp.wait_event(ev["out"][c])
-                view = lambda t: flat(t)[h0:h1].reshape(1, h1 - h0, wl.N, wl.d)
-                sla.sla_forward(view(qd), view(kd), view(vd), view(out), wl.blk_q, wl.blk_k, a.topk, a.phi, a.quant,
-                                ws_chunk, stream=s_cmp)
-                ev["done"][c] = torch.cuda.Event()
-                ev["done"][c].record(s_cmp)
-            for c in range(n_chunks):
-                h0, h1 = bounds[c], bounds[c + 1]
-                s_out.wait_event(ev["done"][c])
-                with torch.cuda.stream(s_out):
-                    flat(hout)[h0:h1].copy_(flat(out)[h0:h1], non_blocking=True)
-                ev["out"][c] = torch.cuda.Event()
-                ev["out"][c].record(s_out)
+            sla.sla_forward_host(hq_, hk_, hv_, hout, wl.blk_q, wl.blk_k, a.topk, a.phi, a.quant, chunk_heads,
+                                 dev_host, stream=s_e2e)
 
         def timed(nsteps):
             f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize(dev)
-            f0.record(s_in)
-            s_cmp.wait_event(f0)
-            s_out.wait_event(f0)
+            f0.record(s_e2e)
             for _ in range(nsteps):
                 e2e_step()
-            s_in.wait_stream(s_out)
-            f1.record(s_in)
+            f1.record(s_e2e)
             torch.cuda.synchronize(dev)
             return f0.elapsed_time(f1) / nsteps
 
         timed(1)
-        # the chunked step gives, bit for bit, the output of one call over the whole workload
+        sla.sla_check(dev_host, stream=s_e2e)
+        # the chunked host call gives, bit for bit, the output of one device call over the workload
         fwd()
         torch.cuda.synchronize(dev)
         same = bool(torch.equal(hout.view(torch.int16), out.cpu().view(torch.int16)))
         if world > 1:
             dist.barrier()
         ms_e2e = max_over_ranks(timed(steps_e2e), dev, world)
-        sla.sla_check(ws_chunk, stream=s_cmp)
+        sla.sla_check(dev_host, stream=s_e2e)
         nbytes = qd.numel() * 2
         e2e = {"value": ops_job / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "chunks": n_chunks,
+               "h2d_bytes_per_step": 3 * nbytes, "d2h_bytes_per_step": nbytes, "chunks": -(-(wl.B * wl.H) // chunk_heads),
                "output_equals_single_call": same,
-               "note": ("host->device copy of Q, K, V from pinned memory, sla_forward, output copied back; "
-                        f"{n_chunks} chunks of consecutive heads pipelined over copy-in, compute and copy-out "
-                        "streams")}
+               "note": ("sla_forward_host: Q, K, V copied in from pinned host memory and the output copied back "
+                        f"inside the call, {chunk_heads} heads per chunk pipelined over copy-in, compute and "
+                        "copy-out streams")}
+        del dev_host
 
     # ---- roofline of the dominant kernel (attention), against the measured peaks
     peaks, peak_kind = load_peaks()

@@ -48,7 +48,8 @@
  * Only d = 128, blk_k = 64 and blk_q in {64, 128} are supported.
  *
  * Memory: every pointer is caller-owned device memory (q, k, v, out, outputs
- * and the workspace), 16-byte aligned.  The library allocates nothing and
+ * and the workspace), 16-byte aligned, except the host buffers of
+ * sla_forward_host.  The library allocates nothing and
  * keeps no per-call global state; calls on different workspaces may run
  * concurrently on different streams.  Calls that share one workspace must be
  * ordered (same stream or explicit events).
@@ -142,6 +143,50 @@ SLA_API sla_status sla_quantize_qk_fp8(const void *q_bf16, const void *k_bf16, i
 SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* The forward of sla_forward for callers whose Q, K, V and output are in HOST
+ * memory.  The pages have no counterpart: this is a deployment variant of
+ * sla_forward that keeps the host-device copies off the critical path.
+ *
+ * q_host, k_host, v_host: bf16 [B, H, N, d] in host memory; out_host: bf16
+ * [B, H, N, d] in host memory, written.  Page-locked buffers (cudaHostAlloc,
+ * cudaHostRegister) let the copies overlap the compute; pageable buffers give
+ * the same result with the copies serialised by the driver.
+ *
+ * The B*H (batch, head) problems are independent.  The call takes them in
+ * chunks of chunk_heads consecutive problems (the last chunk may be smaller)
+ * and, for each chunk, copies its Q, K, V in on one stream, runs the forward
+ * on a second and copies its output back on a third, so that the copy-in of
+ * chunk c+1 and the copy-out of chunk c-1 overlap the forward of chunk c.
+ * The output equals, bit for bit, that of one sla_forward over the whole
+ * problem.
+ *
+ * dev: device memory of at least sla_forward_host_bytes(...) bytes, 16-byte
+ * aligned, owned by the caller: the workspace of one chunk's forward at offset
+ * 0, then two staging slots of Q, K, V and output for one chunk each.  The
+ * status word is the workspace's: sla_check(dev, stream) reports the call.
+ * The first chunk clears it, and later chunks keep an error an earlier chunk
+ * recorded (they then exit early; the output is undefined).
+ *
+ * Ordering: the call's device work starts after the work already queued on
+ * `stream`, and work queued on `stream` after the call starts after the last
+ * copy-out, so out_host is complete once `stream` has been synchronised
+ * (sla_check does that).  The host buffers must stay valid until then.  The
+ * call creates its own three streams and 1 + 3*ceil(B*H/chunk_heads) events
+ * and releases them before it returns (CUDA frees them when their work is
+ * done); it allocates no memory.
+ *
+ * Errors: the shape checks of sla_forward; SLA_ERR_INVALID_ARG for a null host
+ * pointer, chunk_heads < 1 or a null or misaligned dev; SLA_ERR_WORKSPACE when
+ * dev_bytes is below sla_forward_host_bytes; SLA_ERR_CUDA when a stream, an
+ * event or a copy cannot be created or queued (the call then waits for
+ * whatever it had queued before returning).  sla_forward_host_bytes returns 0
+ * for arguments that sla_forward_host would reject before any work. */
+SLA_API size_t sla_forward_host_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant,
+                                      int chunk_heads);
+SLA_API sla_status sla_forward_host(const void *q_host, const void *k_host, const void *v_host, void *out_host,
+                                    int B, int H, int N, int d, int blk_q, int blk_k, float topk, int phi,
+                                    int quant, int chunk_heads, void *dev, size_t dev_bytes, void *stream);
 
 /* sla_block_mask for callers that cannot allocate device memory (for example
  * code inside a framework that owns the whole device-memory budget and hands

@@ -60,6 +60,10 @@ lib.sla_quantize_qk_fp8.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, 
 lib.sla_quantize_qk_fp8.restype = _I
 lib.sla_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P]
 lib.sla_forward.restype = _I
+lib.sla_forward_host_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _F, _I, _I]
+lib.sla_forward_host_bytes.restype = _SZ
+lib.sla_forward_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P, _SZ, _P]
+lib.sla_forward_host.restype = _I
 lib.sla_forward_profile.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _SZ, _P,
                                     ctypes.POINTER(ctypes.c_float)]
 lib.sla_forward_profile.restype = _I
@@ -199,6 +203,31 @@ def sla_forward(q, k, v, out, blk_q, blk_k, topk, phi, quant, ws, stream=None) -
     B, H, N, d = _bhnd(q)
     _ok(lib.sla_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk), int(phi),
                         int(quant), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "sla_forward")
+
+
+def sla_forward_host_bytes(B, H, N, d, blk_q, blk_k, topk, quant, chunk_heads) -> int:
+    return int(lib.sla_forward_host_bytes(B, H, N, d, blk_q, blk_k, float(topk), quant, chunk_heads))
+
+
+def host_workspace(B, H, N, d, blk_q, blk_k, topk, quant, chunk_heads, device=None):
+    """Allocate the device memory (uint8 CUDA tensor) of sla_forward_host."""
+    import torch
+    n = sla_forward_host_bytes(B, H, N, d, blk_q, blk_k, topk, quant, chunk_heads)
+    if n == 0:
+        raise SlaError(1, "sla_forward_host_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def sla_forward_host(q, k, v, out, blk_q, blk_k, topk, phi, quant, chunk_heads, dev, stream=None) -> None:
+    """sla_forward from and to host memory: q, k, v, out are contiguous bf16 CPU tensors (page-locked for
+    overlap); the copies run inside the call, chunk_heads (batch, head) problems at a time."""
+    B, H, N, d = _bhnd(q)
+    for t in (q, k, v, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("sla_forward_host takes contiguous host tensors")
+    _ok(lib.sla_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, blk_q, blk_k, float(topk), int(phi),
+                             int(quant), int(chunk_heads), _ptr(dev), dev.numel() * dev.element_size(),
+                             _stream(stream)), "sla_forward_host")
 
 
 def sla_backward_workspace_bytes(B, H, N, d, blk_q, blk_k, topk) -> int:

@@ -8,8 +8,10 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "../../include/sla.h"
+
 #include "sla_internal.h"
 
 namespace sla {
@@ -242,7 +244,7 @@ namespace {
 constexpr int kProfStages = 7;  // pool, scores+top-k, quantise, states, state reduce, attention, total
 sla_status run_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
                        int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, cudaStream_t s,
-                       cudaEvent_t *ev)
+                       cudaEvent_t *ev, bool reset_status = true)
 {
     sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
     if (st != SLA_OK) return st;
@@ -273,7 +275,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     int e = 0;
     auto mark = [&]() { if (ev) cudaEventRecord(ev[e++], s); };
 
-    SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
+    if (reset_status) SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
     mark();
     // (1) Q: INT8 codes and scales, with the pooled block means as a by-product
     //     (without quantisation: the pooled means alone)
@@ -305,9 +307,129 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     return SLA_OK;
 }
 
+// Device memory of sla_forward_host: the workspace of one chunk's forward at offset 0, then two
+// staging slots, each holding Q, K, V and the output of one chunk.
+struct HostPlan {
+    int hc;              // (batch, head) problems per chunk
+    size_t ws;           // workspace bytes (a multiple of 256)
+    size_t tensor;       // bytes of one staged tensor of a chunk (a multiple of 256)
+    size_t total;
+};
+
+bool host_plan(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant, int chunk_heads, HostPlan &p)
+{
+    if (check_shape(B, H, N, d, blk_q, blk_k, topk) != SLA_OK || quant < 0 || quant > 2 || chunk_heads < 1)
+        return false;
+    p.hc = chunk_heads < B * H ? chunk_heads : B * H;
+    p.ws = align256(make_layout(make_geometry(1, p.hc, N, d, blk_q, blk_k, topk, quant)).total);
+    p.tensor = align256((size_t)p.hc * N * d * sizeof(uint16_t));
+    p.total = p.ws + 2 * 4 * p.tensor;
+    return true;
+}
+
+// Streams and events of one sla_forward_host call; released when the call returns (CUDA frees
+// them once the work queued on them has completed).
+struct HostPipe {
+    cudaStream_t st[3] = {nullptr, nullptr, nullptr};  // copy-in, compute, copy-out
+    std::vector<cudaEvent_t> ev;
+    ~HostPipe()
+    {
+        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+        for (cudaStream_t x : st)
+            if (x) cudaStreamDestroy(x);
+    }
+    bool make(int n_events)
+    {
+        for (cudaStream_t &x : st)
+            if (cudaStreamCreateWithFlags(&x, cudaStreamNonBlocking) != cudaSuccess) return false;
+        ev.reserve(n_events);
+        for (int i = 0; i < n_events; ++i) {
+            cudaEvent_t e;
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+            ev.push_back(e);
+        }
+        return true;
+    }
+};
+
 }  // namespace
 
 extern "C" {
+
+size_t sla_forward_host_bytes(int B, int H, int N, int d, int blk_q, int blk_k, float topk, int quant,
+                              int chunk_heads)
+{
+    HostPlan p;
+    return host_plan(B, H, N, d, blk_q, blk_k, topk, quant, chunk_heads, p) ? p.total : 0;
+}
+
+sla_status sla_forward_host(const void *q_host, const void *k_host, const void *v_host, void *out_host, int B, int H,
+                            int N, int d, int blk_q, int blk_k, float topk, int phi, int quant, int chunk_heads,
+                            void *dev, size_t dev_bytes, void *stream)
+{
+    sla_status st = check_shape(B, H, N, d, blk_q, blk_k, topk);
+    if (st != SLA_OK) return st;
+    if (phi != SLA_PHI_ELU1 && phi != SLA_PHI_RELU) return SLA_ERR_INVALID_ARG;
+    if (quant < 0 || quant > 2 || chunk_heads < 1) return SLA_ERR_INVALID_ARG;
+    if (!q_host || !k_host || !v_host || !out_host || !aligned16(dev)) return SLA_ERR_INVALID_ARG;
+    HostPlan p;
+    if (!host_plan(B, H, N, d, blk_q, blk_k, topk, quant, chunk_heads, p)) return SLA_ERR_INVALID_ARG;
+    if (dev_bytes < p.total) return SLA_ERR_WORKSPACE;
+
+    const int BH = B * H, n_chunks = (BH + p.hc - 1) / p.hc;
+    const size_t head_bytes = (size_t)N * d * sizeof(uint16_t);
+    char *base = static_cast<char *>(dev);
+    void *ws = base;  // status word at offset 0: sla_check(dev, stream) reads the call's status
+    auto staged = [&](int c, int t) { return base + p.ws + ((size_t)(c & 1) * 4 + t) * p.tensor; };
+    const char *host_in[3] = {static_cast<const char *>(q_host), static_cast<const char *>(k_host),
+                              static_cast<const char *>(v_host)};
+    char *host_out = static_cast<char *>(out_host);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // events: [0] the caller's stream at entry; per chunk c: inputs landed (1 + 3c), forward done
+    // (2 + 3c), output copied out (3 + 3c)
+    HostPipe pipe;
+    if (!pipe.make(1 + 3 * n_chunks)) return SLA_ERR_CUDA;
+    cudaStream_t s_in = pipe.st[0], s_cmp = pipe.st[1], s_out = pipe.st[2];
+    auto ev_in = [&](int c) { return pipe.ev[1 + 3 * c]; };
+    auto ev_done = [&](int c) { return pipe.ev[2 + 3 * c]; };
+    auto ev_out = [&](int c) { return pipe.ev[3 + 3 * c]; };
+    SLA_TRY(cudaEventRecord(pipe.ev[0], s));
+    for (cudaStream_t x : pipe.st) SLA_TRY(cudaStreamWaitEvent(x, pipe.ev[0], 0));
+
+    // Chunk c uses slot c % 2.  Its copy-in waits for the forward of chunk c - 2 (which read the
+    // slot's inputs), its forward for its copy-in and for the copy-out of chunk c - 2 (which read
+    // the slot's output).  Every event is recorded before a wait on it is queued.
+    auto enqueue = [&]() -> sla_status {
+        for (int c = 0; c < n_chunks; ++c) {
+            const int h0 = c * p.hc, nh = (c + 1) * p.hc <= BH ? p.hc : BH - h0;
+            const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)nh * head_bytes;
+            if (c >= 2) SLA_TRY(cudaStreamWaitEvent(s_in, ev_done(c - 2), 0));
+            for (int t = 0; t < 3; ++t)
+                SLA_TRY(cudaMemcpyAsync(staged(c, t), host_in[t] + off, bytes, cudaMemcpyHostToDevice, s_in));
+            SLA_TRY(cudaEventRecord(ev_in(c), s_in));
+
+            SLA_TRY(cudaStreamWaitEvent(s_cmp, ev_in(c), 0));
+            if (c >= 2) SLA_TRY(cudaStreamWaitEvent(s_cmp, ev_out(c - 2), 0));
+            // the first chunk clears the status word; later chunks keep an error recorded before them
+            st = run_forward(staged(c, 0), staged(c, 1), staged(c, 2), staged(c, 3), 1, nh, N, d, blk_q, blk_k, topk,
+                             phi, quant, ws, p.ws, s_cmp, nullptr, c == 0);
+            if (st != SLA_OK) return st;
+            SLA_TRY(cudaEventRecord(ev_done(c), s_cmp));
+
+            SLA_TRY(cudaStreamWaitEvent(s_out, ev_done(c), 0));
+            SLA_TRY(cudaMemcpyAsync(host_out + off, staged(c, 3), bytes, cudaMemcpyDeviceToHost, s_out));
+            SLA_TRY(cudaEventRecord(ev_out(c), s_out));
+        }
+        // the caller's stream continues after the last copy-out (which follows every other step)
+        SLA_TRY(cudaStreamWaitEvent(s, ev_out(n_chunks - 1), 0));
+        return SLA_OK;
+    };
+    st = enqueue();
+    if (st != SLA_OK)  // nothing queued by this call outlives it
+        for (cudaStream_t x : pipe.st) cudaStreamSynchronize(x);
+    return st;
+}
 
 sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
                        int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, void *stream)

@@ -102,6 +102,38 @@ def test_forward_host_validation():
     assert fwd(ws_bytes=need - 1) == 3
 
 
+def fwd_host(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, B=1, H=3, N=2048, d=128, blk_q=64, blk_k=64, topk=0.1, phi=0,
+             quant=1, chunk=2, dev=FAKE, dev_bytes=0, stream=None)
+    a.update(kw)
+    return L.sla_forward_host(a["q"], a["k"], a["v"], a["out"], a["B"], a["H"], a["N"], a["d"], a["blk_q"],
+                              a["blk_k"], a["topk"], a["phi"], a["quant"], a["chunk"], a["dev"], a["dev_bytes"],
+                              a["stream"])
+
+
+def test_forward_from_host_buffers_validation():
+    assert fwd_host(q=None) == 1 and fwd_host(out=None) == 1 and fwd_host(dev=None) == 1
+    assert fwd_host(dev=FAKE + 8) == 1                 # misaligned device memory
+    assert fwd_host(chunk=0) == 1 and fwd_host(chunk=-3) == 1
+    assert fwd_host(B=0) == 1 and fwd_host(topk=2.0) == 1 and fwd_host(phi=5) == 1 and fwd_host(quant=3) == 1
+    assert fwd_host(d=64) == 2 and fwd_host(blk_q=32) == 2
+    assert fwd_host(dev_bytes=0) == 3                  # device memory too small (everything else valid)
+    need = sla.sla_forward_host_bytes(1, 3, 2048, 128, 64, 64, 0.1, 1, 2)
+    assert fwd_host(dev_bytes=need - 1) == 3
+
+
+def test_forward_from_host_buffers_bytes():
+    # the workspace of one chunk's forward, then two slots of Q, K, V and output of one chunk
+    for (B, H, N, quant, chunk) in ((1, 40, 75600, 1, 5), (1, 3, 2048, 0, 2), (2, 3, 585, 2, 4), (1, 2, 210, 1, 9)):
+        hc = min(chunk, B * H)
+        ws = sla.sla_workspace_bytes(1, hc, N, 128, 64, 64, 0.1, quant)
+        tensor = -(-hc * N * 128 * 2 // 256) * 256
+        assert sla.sla_forward_host_bytes(B, H, N, 128, 64, 64, 0.1, quant, chunk) == -(-ws // 256) * 256 + 8 * tensor
+    assert sla.sla_forward_host_bytes(1, 3, 2048, 128, 64, 64, 0.1, 1, 0) == 0     # chunk_heads
+    assert sla.sla_forward_host_bytes(1, 3, 2048, 128, 64, 64, 0.1, 3, 2) == 0     # quant
+    assert sla.sla_forward_host_bytes(1, 3, 2048, 64, 64, 64, 0.1, 1, 2) == 0      # d
+
+
 def bwd(**kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1, H=2, N=2048, d=128, blk_q=64,
              blk_k=64, topk=0.1, phi=0, ws=FAKE, ws_bytes=0, stream=None)
