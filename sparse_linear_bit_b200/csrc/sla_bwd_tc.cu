@@ -48,7 +48,7 @@ constexpr int kBwThreads = 192;
 constexpr int kBkThreads = 320;
 constexpr uint32_t kBox = 64 * 128;    // [64 rows x 128 B]
 constexpr uint32_t kTile = 128 * 128;  // [128 rows x 128 B]
-constexpr int kBqStages = 3;
+constexpr int kBqStages = 4;
 constexpr int kBkStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRsd = 0.08838834764831845f;  // 1 / sqrt(128)
@@ -196,10 +196,9 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         constexpr uint32_t id_dq = idesc(1, 1, 1, 0, 1, 128, 128);  // A = dS K-major, B = K MN-major
         const uint64_t qd = sdesc_sw128(smem_u32(sm.q), 16, 1024), dod = sdesc_sw128(smem_u32(sm.dO), 16, 1024);
         bool ok = k_sel == 0 || mbar_wait_warp(&sm.bar_qdo, 0, status, abort_flag);
+        // both issue steps run once the poll below has seen their barriers' phases complete
         auto issue_sd = [&](int T) {
             const int s = T % kBqStages, b = T & 1;
-            if (!(ok = mbar_wait_warp(&sm.full[s], (T / kBqStages) & 1, status, abort_flag))) return;
-            if (T >= 2 && !(ok = mbar_wait_warp(&sm.bar_sdfree[b], ((T >> 1) - 1) & 1, status, abort_flag))) return;
             tc_fence_after();
             if (elect_one()) {
                 issue_s_dp(tmem + 128 * b, tmem + 128 * b + 64, qd, dod, sdesc_sw128(smem_u32(sm.kv[s][0]), 16, 1024),
@@ -211,7 +210,6 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         };
         auto issue_dq = [&](int t) {  // pass-2 tile t
             const int T = k_sel + t, s = T % kBqStages, b = t & 1;
-            if (!(ok = mbar_wait_warp(&sm.bar_ds[b], (t >> 1) & 1, status, abort_flag))) return;
             tc_fence_after();
             if (elect_one()) {
                 const uint64_t dsd = sdesc_sw128(smem_u32(sm.ds[b]), 16, 1024);
@@ -225,11 +223,36 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             }
             __syncwarp();
         };
-        for (int T = 0; ok && T < nT; ++T) {
-            issue_sd(T);
-            if (ok && T - 1 >= k_sel) issue_dq(T - 1 - k_sel);
+        // dQ of a pass-2 tile is issued as soon as its dS is in shared memory (it frees a K/V stage
+        // and a dS buffer); S/dP of the next tile as soon as its stage has landed and its TMEM
+        // buffer is free
+        int n_sd = 0, n_dq = 0;
+        long long t0c = clock64();
+        const long long budget = wait_budget();
+        while (ok && n_dq < k_sel) {
+            const bool can_dq = n_dq < n_sd - k_sel && mbar_test(&sm.bar_ds[n_dq & 1], (n_dq >> 1) & 1);
+            if (__any_sync(0xffffffffu, can_dq)) {
+                issue_dq(n_dq++);
+                t0c = clock64();
+                continue;
+            }
+            const bool can_sd = n_sd < nT && mbar_test(&sm.full[n_sd % kBqStages], (n_sd / kBqStages) & 1) &&
+                                (n_sd < 2 || mbar_test(&sm.bar_sdfree[n_sd & 1], ((n_sd >> 1) - 1) & 1));
+            if (__any_sync(0xffffffffu, can_sd)) {
+                issue_sd(n_sd++);
+                t0c = clock64();
+                continue;
+            }
+            if (clock64() - t0c > budget) {  // neither came: the same bounded-wait rule as mbar_wait
+                if (elect_one()) record_error(status, kStatusTimeout);
+                *abort_flag = 1;
+                ok = false;
+            } else if (global_failed(status) || *abort_flag) {
+                *abort_flag = 1;
+                ok = false;
+            }
+            ok = __all_sync(0xffffffffu, ok);
         }
-        if (ok && k_sel > 0) issue_dq(k_sel - 1);
         if (elect_one()) {
             mma_commit(&sm.drain);
             mbar_wait_quiet(&sm.drain, 0, status);  // this thread's MMAs retired before TMEM is released
