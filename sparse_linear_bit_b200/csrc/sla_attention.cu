@@ -261,13 +261,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             tma_prefetch_desc(&tm_h);
             tma_prefetch_desc(&tm_qr);
             // the linear epilogue's operands into L2 now, so that their loads at the end do not wait on HBM
-            for (int c = 0; c < 4; ++c) tma_prefetch_l2_3d(&tm_h, 32 * c, 0, bh * n_qb + I);
+            tma_prefetch_l2_4d(&tm_h, 0, 0, 0, bh * n_qb + I);
             if (QUANT) {
-                for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_qr, 64 * c, I * blk_q, bh);
+                tma_prefetch_l2_4d(&tm_qr, 0, I * blk_q, 0, bh);
             } else {  // the bf16 Q tile: A operand of Q.K^T, and the raw Q of phi at the end
                 mbar_expect_tx(&sm.bar_q, 2 * kQRowsBox);
-                for (int c = 0; c < 2; ++c)
-                    tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_q, 64 * c, I * blk_q, bh);
+                tma_load_4d(qraw_s, &tm_qr, &sm.bar_q, 0, I * blk_q, 0, bh);
             }
         }
         __syncwarp();
@@ -280,11 +279,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
             const int J = __ldg(sel + t);
             if (elect_one()) {
                 mbar_expect_tx(&sm.full[s], Cfg::kStageBytes);
-                // K: one 128-channel int8 box, or two 64-channel bf16 boxes; V: dims 0-63, then 64-127
-                tma_load_3d(st, &tm_k, &sm.full[s], 0, J * 64, bh);
-                if (!QUANT) tma_load_3d(st + kBox, &tm_k, &sm.full[s], 64, J * 64, bh);
-                tma_load_3d(st + Cfg::kKBytes, &tm_v, &sm.full[s], 0, J * 64, bh);
-                tma_load_3d(st + Cfg::kKBytes + kBox, &tm_v, &sm.full[s], 64, J * 64, bh);
+                // K: one 128-channel int8 box, or the two 64-channel halves of the bf16 rows; V: the two
+                // halves of its rows (dims 0-63, then 64-127).  One copy each: a copy costs the issuing
+                // CTA about the same whatever its size
+                if (QUANT) tma_load_3d(st, &tm_k, &sm.full[s], 0, J * 64, bh);
+                else tma_load_4d(st, &tm_k, &sm.full[s], 0, J * 64, 0, bh);
+                tma_load_4d(st + Cfg::kKBytes, &tm_v, &sm.full[s], 0, J * 64, 0, bh);
             }
             __syncwarp();
             issued = t + 1;
@@ -297,11 +297,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CU
         }
         if (ok && elect_one()) {
             mbar_expect_tx(&sm.bar_h, 4 * kQRowsBox);
-            for (int c = 0; c < 4; ++c) tma_load_3d(h_s + c * kQRowsBox, &tm_h, &sm.bar_h, 32 * c, 0, bh * n_qb + I);
+            tma_load_4d(h_s, &tm_h, &sm.bar_h, 0, 0, 0, bh * n_qb + I);
             if (QUANT) {
                 mbar_expect_tx(&sm.bar_qr, 2 * kQRowsBox);
-                for (int c = 0; c < 2; ++c)
-                    tma_load_3d(qraw_s + c * kQRowsBox, &tm_qr, &sm.bar_qr, 64 * c, I * blk_q, bh);
+                tma_load_4d(qraw_s, &tm_qr, &sm.bar_qr, 0, I * blk_q, 0, bh);
             }
         }
         __syncwarp();
@@ -573,28 +572,30 @@ cudaError_t launch_attn_t(const void *q, const void *k, const void *v, const int
         const uint64_t st[2] = {(uint64_t)kD, (uint64_t)g.N * kD};
         const uint32_t bk[3] = {128, 64, 1};
         if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, k8, dims, st, bk)) return cudaErrorInvalidValue;
-    } else {
-        const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
-        const uint32_t bk[3] = {64, 64, 1};
-        if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, st, bk)) return cudaErrorInvalidValue;
     }
+    // 16-bit rows of 128 as [64 elements, rows (256 B apart), 2 halves (128 B apart), BH]: a box of
+    // {64, 64, 2, 1} lands as the two [64 rows x 128 B] half-tiles one after the other
+    const uint64_t dims_h[4] = {64, (uint64_t)g.N, 2, (uint64_t)g.BH};
+    const uint64_t st_h[3] = {(uint64_t)kD * 2, 128, (uint64_t)g.N * kD * 2};
+    const uint32_t box_h[4] = {64, 64, 2, 1};
+    if (!QUANT && !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims_h, st_h, box_h))
+        return cudaErrorInvalidValue;
     {
-        const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
-        const uint32_t bv[3] = {64, 64, 1};
         const CUtensorMapDataType vt = QUANT ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-        if (!encode_tmap(&tv, vt, 3, v, dims, st, bv)) return cudaErrorInvalidValue;
+        if (!encode_tmap(&tv, vt, 4, v, dims_h, st_h, box_h)) return cudaErrorInvalidValue;
     }
     {
-        const uint64_t hd[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)g.BH * g.n_qb};
-        const uint64_t st[2] = {(uint64_t)kD * 4, (uint64_t)kStateCols * 4};
-        const uint32_t bh[3] = {32, 128, 1};
-        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, hd, st, bh)) return cudaErrorInvalidValue;
+        // H_I^T [128 dims][128 channels] fp32 in rows of kStateCols, viewed as [32 channels, 128 dims
+        // (512 B apart), 4 quarters (128 B apart), BH * n_qb]: one box, the four quarter-tiles in order
+        const uint64_t hd[4] = {32, (uint64_t)kD, 4, (uint64_t)g.BH * g.n_qb};
+        const uint64_t st[3] = {(uint64_t)kD * 4, 128, (uint64_t)kStateCols * 4};
+        const uint32_t bh[4] = {32, 128, 4, 1};
+        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, hq, hd, st, bh)) return cudaErrorInvalidValue;
     }
     {
-        // raw Q rows of a query block: [BH, N, 128] bf16, boxes of 64 channels x 128 rows
-        const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
-        const uint32_t bq[3] = {64, 128, 1};
-        if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, dims, st, bq)) return cudaErrorInvalidValue;
+        // raw Q rows of a query block: both 64-channel halves of 128 rows in one box
+        const uint32_t bq[4] = {64, 128, 2, 1};
+        if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q, dims_h, st_h, bq)) return cudaErrorInvalidValue;
     }
     const size_t smem = sizeof(AttnSmem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attn_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

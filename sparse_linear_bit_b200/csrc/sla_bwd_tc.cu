@@ -162,10 +162,8 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             mbar_expect_tx(&sm.bar_qdo, 4 * kTile);
-            for (int c = 0; c < 2; ++c) {
-                tma_load_3d(sm.q + c * kTile, &tm_q, &sm.bar_qdo, 64 * c, I * blk_q, bh);
-                tma_load_3d(sm.dO + c * kTile, &tm_do, &sm.bar_qdo, 64 * c, I * blk_q, bh);
-            }
+            tma_load_4d(sm.q, &tm_q, &sm.bar_qdo, 0, I * blk_q, 0, bh);
+            tma_load_4d(sm.dO, &tm_do, &sm.bar_qdo, 0, I * blk_q, 0, bh);
         }
         __syncwarp();
         int issued = 0;
@@ -176,10 +174,8 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const int J = __ldg(sel + (T < k_sel ? T : T - k_sel));
             if (elect_one()) {
                 mbar_expect_tx(&sm.full[s], 4 * kBox);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_3d(sm.kv[s][c], &tm_k, &sm.full[s], 64 * c, J * 64, bh);
-                    tma_load_3d(sm.kv[s][2 + c], &tm_v, &sm.full[s], 64 * c, J * 64, bh);
-                }
+                tma_load_4d(sm.kv[s][0], &tm_k, &sm.full[s], 0, J * 64, 0, bh);
+                tma_load_4d(sm.kv[s][2], &tm_v, &sm.full[s], 0, J * 64, 0, bh);
             }
             __syncwarp();
             issued = T + 1;
@@ -493,10 +489,8 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             mbar_expect_tx(&sm.bar_kv, 4 * kBox);
-            for (int c = 0; c < 2; ++c) {
-                tma_load_3d(sm.k + c * kBox, &tm_k, &sm.bar_kv, 64 * c, t0, bh);
-                tma_load_3d(sm.v + c * kBox, &tm_v, &sm.bar_kv, 64 * c, t0, bh);
-            }
+            tma_load_4d(sm.k, &tm_k, &sm.bar_kv, 0, t0, 0, bh);
+            tma_load_4d(sm.v, &tm_v, &sm.bar_kv, 0, t0, 0, bh);
         }
         __syncwarp();
         BitWalk walk(bits, words);
@@ -508,10 +502,8 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             if (u > 0 && !(ok = mbar_wait_warp(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
             if (elect_one()) {
                 mbar_expect_tx(&sm.full[s], 4 * kTile);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_3d(sm.qd[s] + c * kTile, &tm_q, &sm.full[s], 64 * c, I * blk_q, bh);
-                    tma_load_3d(sm.qd[s] + (2 + c) * kTile, &tm_do, &sm.full[s], 64 * c, I * blk_q, bh);
-                }
+                tma_load_4d(sm.qd[s], &tm_q, &sm.full[s], 0, I * blk_q, 0, bh);
+                tma_load_4d(sm.qd[s] + 2 * kTile, &tm_do, &sm.full[s], 0, I * blk_q, 0, bh);
             }
             __syncwarp();
             issued = t + 1;
@@ -797,11 +789,9 @@ bwd_qlin_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant_
     tc_fence_after();
     if (tid == 0) {
         mbar_expect_tx(&sm.bar_ld, 8 * kTile);
-        for (int c = 0; c < 4; ++c) tma_load_3d(sm.hs + c * kTile, &tm_h, &sm.bar_ld, 32 * c, 0, bh * n_qb + I);
-        for (int c = 0; c < 2; ++c) {
-            tma_load_3d(sm.qr + c * kTile, &tm_q, &sm.bar_ld, 64 * c, I * blk_q, bh);
-            tma_load_3d(sm.da + c * kTile, &tm_do, &sm.bar_ld, 64 * c, I * blk_q, bh);
-        }
+        tma_load_4d(sm.hs, &tm_h, &sm.bar_ld, 0, 0, 0, bh * n_qb + I);
+        tma_load_4d(sm.qr, &tm_q, &sm.bar_ld, 0, I * blk_q, 0, bh);
+        tma_load_4d(sm.da, &tm_do, &sm.bar_ld, 0, I * blk_q, 0, bh);
     }
     const float *hrow = hq + ((size_t)bh * n_qb + I) * kStateCols;
     sm.z[tid] = __ldg(hrow + 128 * 128 + tid);
@@ -1138,13 +1128,16 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
     }
 }
 
-// 3-D map [BH, N, 128] of a bf16 tensor, boxes of 64 channels x `rows` rows
+// Map of a bf16 tensor [BH, N, 128] viewed as [64 elements, N rows (256 B apart), 2 halves (128 B
+// apart), BH]: one box of {64, rows, 2, 1} lands as the two [rows x 128 B] half-tiles (channels 0-63,
+// then 64-127) one after the other.  One copy per tile instead of two: a copy costs the issuing CTA
+// about the same whatever its size.
 bool map_rows(CUtensorMap *m, const void *base, const Geometry &g, uint32_t rows)
 {
-    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
-    const uint64_t st[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
-    const uint32_t box[3] = {64, rows, 1};
-    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, st, box);
+    const uint64_t dims[4] = {64, (uint64_t)g.N, 2, (uint64_t)g.BH};
+    const uint64_t st[3] = {(uint64_t)kD * 2, 128, (uint64_t)g.N * kD * 2};
+    const uint32_t box[4] = {64, rows, 2, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, st, box);
 }
 
 }  // namespace
@@ -1187,11 +1180,13 @@ cudaError_t launch_bwd_query_linear(const void *q, const void *dout, const float
 {
     CUtensorMap th, tq, tdo;
     {
-        // H_I^T of every query block: [BH * n_qb][128 dims][128 channels] fp32 inside rows of kStateCols
-        const uint64_t hd[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)g.BH * g.n_qb};
-        const uint64_t st[2] = {(uint64_t)kD * 4, (uint64_t)kStateCols * 4};
-        const uint32_t bx[3] = {32, 128, 1};
-        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, hq, hd, st, bx)) return cudaErrorInvalidValue;
+        // H_I^T of every query block: [BH * n_qb][128 dims][128 channels] fp32 inside rows of kStateCols,
+        // viewed as [32 channels, 128 dims (512 B apart), 4 quarters (128 B apart), BH * n_qb]: one box
+        // lands as the four [128 x 128 B] quarter-tiles one after the other
+        const uint64_t hd[4] = {32, (uint64_t)kD, 4, (uint64_t)g.BH * g.n_qb};
+        const uint64_t st[3] = {(uint64_t)kD * 4, 128, (uint64_t)kStateCols * 4};
+        const uint32_t bx[4] = {32, 128, 4, 1};
+        if (!encode_tmap(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, hq, hd, st, bx)) return cudaErrorInvalidValue;
     }
     if (!map_rows(&tq, q, g, 128) || !map_rows(&tdo, dout, g, 128)) return cudaErrorInvalidValue;
     const size_t smem = sizeof(LqSmem) + 1024;

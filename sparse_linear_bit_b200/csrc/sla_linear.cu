@@ -123,10 +123,8 @@ __global__ void __launch_bounds__(kStatesThreads, 1) states_kernel(const __grid_
                     const int s = j % kStStages, u = j / kStStages, row = (Jbeg + jj) * 64;
                     if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
                     mbar_expect_tx(&sm.full[s], 4 * kTileBytes);
-                    tma_load_3d(sm.kv[s][0], &tm_k, &sm.full[s], 0, row, bh);
-                    tma_load_3d(sm.kv[s][1], &tm_k, &sm.full[s], 64, row, bh);
-                    tma_load_3d(sm.kv[s][2], &tm_v, &sm.full[s], 0, row, bh);
-                    tma_load_3d(sm.kv[s][3], &tm_v, &sm.full[s], 64, row, bh);
+                    tma_load_4d(sm.kv[s][0], &tm_k, &sm.full[s], 0, row, 0, bh);  // both halves of K
+                    tma_load_4d(sm.kv[s][2], &tm_v, &sm.full[s], 0, row, 0, bh);  // both halves of V
                 }
             }
             if (!ok) {  // loads in flight land before the CTA exits
@@ -455,9 +453,7 @@ __global__ void __launch_bounds__(kRedThreads, 1) reduce_kernel(const uint32_t *
                 const int s = kc % kRedBStages, u = kc / kRedBStages;
                 if (u > 0 && !(ok = mbar_wait(&sm.empty[s], (u - 1) & 1, status, abort_flag))) break;
                 mbar_expect_tx(&sm.full[s], kRedB);
-#pragma unroll
-                for (int g = 0; g < 3; ++g)
-                    tma_load_3d(sm.b[s] + g * kTileBytes, &tm_s, &sm.full[s], n0 + 64 * g, kt * 64, bh);
+                tma_load_4d(sm.b[s], &tm_s, &sm.full[s], n0, kt * 64, 0, bh);  // the three 64-column groups
             }
         }
         if (!ok) {  // let in-flight loads land before the CTA exits
@@ -618,11 +614,13 @@ cudaError_t launch_states(const void *k, const void *v, const Geometry &g, int p
                           uint16_t *v16, int *status, cudaStream_t s)
 {
     CUtensorMap tk, tv, to;
-    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)g.N, (uint64_t)g.BH};
-    const uint64_t strides[2] = {(uint64_t)kD * 2, (uint64_t)g.N * kD * 2};
-    const uint32_t box[3] = {64, 64, 1};
-    if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, v, dims, strides, box)) return cudaErrorInvalidValue;
+    // K and V [BH, N, 128] viewed as [64 elements, N rows (256 B apart), 2 halves (128 B apart), BH]:
+    // one box per key block lands as its two [64 rows x 128 B] half-tiles, one after the other
+    const uint64_t dims[4] = {64, (uint64_t)g.N, 2, (uint64_t)g.BH};
+    const uint64_t strides[3] = {(uint64_t)kD * 2, 128, (uint64_t)g.N * kD * 2};
+    const uint32_t box[4] = {64, 64, 2, 1};
+    if (!encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, strides, box)) return cudaErrorInvalidValue;
     {
         // h_J^T of every key block: [BH * n_kb][128 dims][128 channels] inside rows of kStateCols
         const uint64_t od[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)g.BH * g.n_kb};
@@ -663,10 +661,15 @@ cudaError_t launch_state_reduce(const uint32_t *amask, const uint16_t *states, c
             return cudaErrorInvalidValue;
     }
     {
-        const uint64_t dims[3] = {(uint64_t)kStateCols, (uint64_t)g.n_kb, (uint64_t)g.BH};
-        const uint64_t strides[2] = {(uint64_t)kStateCols * 2, (uint64_t)g.n_kb * kStateCols * 2};
-        const uint32_t box[3] = {64, 64, 1};
-        if (!encode_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, states, dims, strides, box))
+        // states [BH][n_kb][kStateCols] bf16 viewed as [columns, key blocks, 3 column groups (128 B
+        // apart), BH]: a box of {64, 64, 3, 1} at column n0 holds columns n0 + 64 g + (0..63) for g < 3,
+        // landing as the three [64 key blocks x 128 B] tiles of a k-step one after the other (the
+        // group dimension overlaps the column dimension; the box never leaves the row: n0 + 191 <
+        // kStateCols)
+        const uint64_t dims[4] = {(uint64_t)kStateCols, (uint64_t)g.n_kb, 3, (uint64_t)g.BH};
+        const uint64_t strides[3] = {(uint64_t)kStateCols * 2, 128, (uint64_t)g.n_kb * kStateCols * 2};
+        const uint32_t box[4] = {64, 64, 3, 1};
+        if (!encode_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, states, dims, strides, box))
             return cudaErrorInvalidValue;
     }
     const size_t smem = sizeof(ReduceSmem) + 1024;
