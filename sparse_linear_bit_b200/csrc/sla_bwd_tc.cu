@@ -657,23 +657,33 @@ bwdk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             fence_async_smem();
             mbar_arrive(&sm.bar_pd[b]);
         }
-        // ---- epilogue: TMEM lane r = dim / channel r; column j = key t0 + j.  Added to the linear part.
-        if (ok) ok = wait_all(&sm.bar_acc, 0);
+        // ---- epilogue: TMEM lane r = dim / channel r; column j = key t0 + j.  Added to the linear part,
+        // whose values are all loaded first (while the last accumulation runs), so that the 64
+        // read-modify-writes of a thread do not wait on one another's loads
+        float *pv = dv + ((size_t)bh * N + t0 + j0) * 128 + r;
+        float *pk = dk + ((size_t)bh * N + t0 + j0) * 128 + r;
+        float lv[32], lk[32];
+        if (ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                lv[j] = j0 + j < kv ? __ldcg(pv + (size_t)j * 128) : 0.0f;
+                lk[j] = j0 + j < kv ? __ldcg(pk + (size_t)j * 128) : 0.0f;
+            }
+            ok = wait_all(&sm.bar_acc, 0);
+        }
         if (ok) {
             tc_fence_after();
             uint32_t a[32];
             tmem_ld32(t_dv + j0 + lane_off, a);
             tmem_wait_ld();
-            float *pv = dv + ((size_t)bh * N + t0 + j0) * 128 + r;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (j0 + j < kv) pv[(size_t)j * 128] += __uint_as_float(a[j]);
+                if (j0 + j < kv) pv[(size_t)j * 128] = lv[j] + __uint_as_float(a[j]);
             tmem_ld32(t_dk + j0 + lane_off, a);
             tmem_wait_ld();
-            float *pk = dk + ((size_t)bh * N + t0 + j0) * 128 + r;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                if (j0 + j < kv) pk[(size_t)j * 128] += __uint_as_float(a[j]);
+                if (j0 + j < kv) pk[(size_t)j * 128] = lk[j] + __uint_as_float(a[j]);
         }
     }
     tc_fence_before();
@@ -974,15 +984,26 @@ bwd_qlin_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant_
     }
     __syncthreads();  // the dq deltas are staged
     if (ok) {
-        // dq += the staged deltas: warp w takes rows 32 w .. 32 w + 31, one coalesced 512-byte row per step
-        for (int rr = 0; rr < 32; ++rr) {
-            const int row = warp * 32 + rr;
-            if (row >= rows) break;
-            float4 *g = reinterpret_cast<float4 *>(dq + ((size_t)bh * N + I * blk_q + row) * 128) + lane;
-            const float4 d = *reinterpret_cast<const float4 *>(sm.hs + f32_off(row, 4 * lane));
-            float4 v = *g;
-            v.x += d.x; v.y += d.y; v.z += d.z; v.w += d.w;
-            *g = v;
+        // dq += the staged deltas: warp w takes rows 32 w .. 32 w + 31, one coalesced 512-byte row per
+        // step, eight rows' loads issued before their stores
+#pragma unroll 1
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+            float4 v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int row = warp * 32 + r0 + q;
+                if (row < rows)
+                    v[q] = __ldcg(reinterpret_cast<const float4 *>(dq + ((size_t)bh * N + I * blk_q + row) * 128) + lane);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int row = warp * 32 + r0 + q;
+                if (row < rows) {
+                    const float4 d = *reinterpret_cast<const float4 *>(sm.hs + f32_off(row, 4 * lane));
+                    v[q].x += d.x; v[q].y += d.y; v[q].z += d.z; v[q].w += d.w;
+                    reinterpret_cast<float4 *>(dq + ((size_t)bh * N + I * blk_q + row) * 128)[lane] = v[q];
+                }
+            }
         }
     }
     tc_fence_before();
