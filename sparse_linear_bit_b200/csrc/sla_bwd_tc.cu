@@ -273,9 +273,11 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // the tile's max exceeds it by more than 2^8, so p stays below 256 and most tiles need no rescale)
         float m = -INFINITY, l = 0.0f, Dt = 0.0f;
         const uint64_t c2 = f2pack(c, c);
+        int J_next = k_sel > 0 ? __ldg(sel) : 0;  // the selected blocks, loaded one tile ahead of use
         for (int t = 0; ok && t < k_sel; ++t) {
             const int T = t, b = T & 1;
-            const int J = __ldg(sel + t), valid = min(64, N - J * 64);
+            const int J = J_next, valid = min(64, N - J * 64);
+            J_next = __ldg(sel + (t + 1 < k_sel ? t + 1 : 0));
             if (!(ok = wait_all(&sm.bar_sd[b], (T >> 1) & 1))) break;
             tc_fence_after();
             uint32_t sv[64], dv[64];
@@ -326,9 +328,11 @@ bwdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         // ---- pass 2: dS (bf16) into shared memory for dQ += dS K
         float sigma = 0.0f;  // fp32 sum of the rounded dS of this row
+        J_next = k_sel > 0 ? __ldg(sel) : 0;
         for (int t = 0; ok && t < k_sel; ++t) {
             const int T = k_sel + t, b = T & 1, bd = t & 1;
-            const int J = __ldg(sel + t), valid = row_valid ? min(64, N - J * 64) : 0;
+            const int J = J_next, valid = row_valid ? min(64, N - J * 64) : 0;
+            J_next = __ldg(sel + (t + 1 < k_sel ? t + 1 : 0));
             if (!(ok = wait_all(&sm.bar_sd[b], (T >> 1) & 1))) break;
             tc_fence_after();
             uint32_t sv[64], dv[64];
@@ -1130,11 +1134,16 @@ bwd_klin_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, 
         tmem_wait_ld();
         const size_t base = ((size_t)bh * N + t0) * 128 + c;
 #pragma unroll
-        for (int j = 0; j < 64; ++j)
-            if (j < kv) {
-                const float kc = __uint_as_float((uint32_t)k[base + (size_t)j * 128] << 16);
-                dk[base + (size_t)j * 128] = (__uint_as_float(a[j]) + sm.gp[c]) * dphi_lin(kc, phi);
-            }
+        for (int j0 = 0; j0 < 64; j0 += 32) {  // 32 keys' loads issued before their stores
+            uint16_t kb[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) kb[j] = j0 + j < kv ? __ldg(k + base + (size_t)(j0 + j) * 128) : (uint16_t)0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j0 + j < kv)
+                    dk[base + (size_t)(j0 + j) * 128] =
+                        (__uint_as_float(a[j0 + j]) + sm.gp[c]) * dphi_lin(__uint_as_float((uint32_t)kb[j] << 16), phi);
+        }
         tmem_ld64(t_v + lane_off, a);
         tmem_wait_ld();
 #pragma unroll
