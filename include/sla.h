@@ -139,7 +139,12 @@ SLA_API sla_status sla_quantize_qk_fp8(const void *q_bf16, const void *k_bf16, i
                                float *k_scale, float *k_mean, void *ws, size_t ws_bytes, void *stream);
 
 /* The whole forward, steps 1-6.  quant: 0 = none, 1 = INT8, 2 = FP8 e4m3.
- * out: bf16 [B, H, N, d]. */
+ * out: bf16 [B, H, N, d].  Stream-ordered on `stream`: its work starts after the
+ * work queued there before the call and ends before the work queued after it.
+ * Inside, the K side (K's block means, the linear states, K's smoothing mean and
+ * codes) runs on a second stream that the call creates and releases, beside the Q
+ * side and the block selection; not while `stream` is being captured into a
+ * graph, where every step runs on `stream`. */
 SLA_API sla_status sla_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N,
                        int d, int blk_q, int blk_k, float topk, int phi, int quant, void *ws,
                        size_t ws_bytes, void *stream);

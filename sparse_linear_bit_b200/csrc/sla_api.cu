@@ -239,8 +239,33 @@ sla_status sla_quantize_qk_fp8(const void *q, const void *k, int B, int H, int N
 
 namespace {
 
+// A second stream and two events for one forward call; released when the call returns (CUDA frees
+// them once the work queued on them has completed).
+struct ForkK {
+    cudaStream_t st = nullptr;
+    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, K block means ready, K side done
+    bool make()
+    {
+        if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return false;
+        for (cudaEvent_t &e : ev)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+        return true;
+    }
+    ~ForkK()
+    {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+        if (st) cudaStreamDestroy(st);
+    }
+};
+
 // The forward's launch sequence.  When `ev` is non-null, an event is recorded
-// before the first stage and after each of the kStages stages (on `s`).
+// before the first stage and after each of the kStages stages (on `s`), and every
+// stage runs on `s` in order.  Otherwise the K side (K's block means and partial
+// sums, the linear states and the global state, K's smoothing mean and codes)
+// runs on a second stream beside the Q side and the block selection, which need
+// from it only the K block means; the two meet before the state reduction.  The
+// selection's fp64 scores and top-k then overlap the K side's memory traffic.
 constexpr int kProfStages = 7;  // pool, scores+top-k, quantise, states, state reduce, attention, total
 sla_status run_forward(const void *q, const void *k, const void *v, void *out, int B, int H, int N, int d, int blk_q,
                        int blk_k, float topk, int phi, int quant, void *ws, size_t ws_bytes, cudaStream_t s,
@@ -276,27 +301,53 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     auto mark = [&]() { if (ev) cudaEventRecord(ev[e++], s); };
 
     if (reset_status) SLA_TRY(cudaMemsetAsync(status, 0, sizeof(int), s));
-    mark();
-    // (1) Q: INT8 codes and scales, with the pooled block means as a by-product
-    //     (without quantisation: the pooled means alone)
-    if (quant) SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, qbar, quant == 2, s));
-    else SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
-    mark();
-    // (2) pooled block means of K (and its partial sums for the smoothing mean),
-    //     per-key-block linear states and the global state
-    SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, quant ? kpart : nullptr, s));
-    SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, s));
-    SLA_TRY(launch_htot(partials, g, htot, s));
-    mark();
-    // (3) scores + top-k selection
-    SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
-    SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
-    mark();
-    // (4) K: smoothing mean, INT8 codes and scales
-    if (quant) {
-        SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), kmean, s));
-        SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, nullptr, quant == 2, s));
+    // (not while `s` is being captured into a graph: the second stream is destroyed when the call
+    // returns, before the capture ends)
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    SLA_TRY(cudaStreamIsCapturing(s, &cap));
+    ForkK fk;
+    const bool fork = ev == nullptr && cap == cudaStreamCaptureStatusNone && fk.make();
+    cudaStream_t sk = fork ? fk.st : s;  // the K side's stream
+    if (fork) {
+        SLA_TRY(cudaEventRecord(fk.ev[0], s));
+        SLA_TRY(cudaStreamWaitEvent(sk, fk.ev[0], 0));
     }
+    mark();
+    // The stages up to the join.  On an error the K side is still joined below, so that nothing
+    // this call queued outlives the caller's stream.
+    auto until_join = [&]() -> sla_status {
+        // (1) Q: INT8 codes and scales, with the pooled block means as a by-product
+        //     (without quantisation: the pooled means alone)
+        if (quant) SLA_TRY(launch_quant(q, g.BH, N, blk_q, g.n_qb, nullptr, q8, qscale, qbar, quant == 2, s));
+        else SLA_TRY(launch_pool(q, g.BH, N, blk_q, g.n_qb, qbar, nullptr, s));
+        mark();
+        // (2) pooled block means of K (and its partial sums for the smoothing mean),
+        //     per-key-block linear states and the global state
+        SLA_TRY(launch_pool(k, g.BH, N, blk_k, g.n_kb, kbar, quant ? kpart : nullptr, sk));
+        if (fork) SLA_TRY(cudaEventRecord(fk.ev[1], sk));
+        SLA_TRY(launch_states(k, v, g, phi, states, partials, v16, status, sk));
+        SLA_TRY(launch_htot(partials, g, htot, sk));
+        mark();
+        // (3) scores + top-k selection
+        if (fork) SLA_TRY(cudaStreamWaitEvent(s, fk.ev[1], 0));
+        SLA_TRY(launch_scores(qbar, kbar, g, scores, s));
+        SLA_TRY(launch_topk(scores, g, idx, nullptr, amask, s));
+        mark();
+        // (4) K: smoothing mean, INT8 codes and scales
+        if (quant) {
+            SLA_TRY(launch_kmean(kpart, g.BH, N, pool_parts(g.n_kb), kmean, sk));
+            SLA_TRY(launch_quant(k, g.BH, N, blk_k, g.n_kb, kmean, k8, kscale, nullptr, quant == 2, sk));
+        }
+        return SLA_OK;
+    };
+    st = until_join();
+    if (fork) {  // the join: the state reduction and attention need the K side
+        if (cudaEventRecord(fk.ev[2], sk) != cudaSuccess || cudaStreamWaitEvent(s, fk.ev[2], 0) != cudaSuccess) {
+            cudaStreamSynchronize(sk);
+            return SLA_ERR_CUDA;
+        }
+    }
+    if (st != SLA_OK) return st;
     mark();
     // (5) per-query-block state
     SLA_TRY(launch_state_reduce(amask, states, htot, g, hq, status, s));
