@@ -758,7 +758,7 @@ SLA_DEV float load_elem128(const uint8_t *tile, uint32_t box, int r, int c)
 }
 
 struct LqSmem {
-    alignas(1024) uint8_t hs[4 * kTile];  // H_I^T fp32 as loaded (4 boxes [128 dims x 32 channels]); later dq staging
+    alignas(1024) uint8_t hs[4 * kTile];  // H_I^T fp32: four [128 dims x 32 channels] tiles; later dq staging
     alignas(1024) uint8_t qr[2 * kTile];  // raw Q rows of the query block (bf16, [rows x 64 channels] boxes)
     alignas(1024) uint8_t da[2 * kTile];  // dO rows as loaded, then dA in place ([row i][dim e]: K-major A of H da,
                                           // MN-major B of dH)
