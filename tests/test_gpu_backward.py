@@ -10,8 +10,8 @@ tf32 (2^-11), and the state gradients entering G = A^T dH as bf16 (2^-9).  So
 either branch's part of a gradient carries up to ~2 x 2^-9 ~ 4e-3 relative
 error, and the whole gradient less.
 Every element must also be finite, and two calls must give identical bytes.
-At the full 14B-720P size, dq of sampled rows and dk, dv of sampled key blocks are
-compared with the oracle, which evaluates exactly those rows / blocks.
+At the full 14B-720P and 1.3B-480P sizes, dq of sampled rows and dk, dv of sampled key
+blocks are compared with the oracle, which evaluates exactly those rows / blocks.
 """
 from __future__ import annotations
 
@@ -146,3 +146,34 @@ def test_backward_full_size_sampled_dkdv():
     ek, ev = rel_l2(gk, rk), rel_l2(gv, rv)
     print(f"\nfull-size sampled key blocks: dk rel_l2={ek:.3e} dv rel_l2={ev:.3e}")
     assert ek <= TOL and ev <= TOL, (ek, ev)
+
+
+def test_backward_480p_sampled():
+    """1.3B-480P shape (B=1, H=12, N=32760: its last query block holds 120 rows and its last key block
+    56 keys), one call: dq of sampled rows of 3 heads, and dk, dv of the first, a middle and the ragged
+    last key block of 3 heads, against the oracle."""
+    w = synth.WORKLOADS["wan1.3b-480p"]
+    q, k, v = workload_qkv("wan1.3b-480p")
+    dout = workload_qkv("wan1.3b-480p", seed_offset=1)[0]
+    dq, dk, dv = run_backward(q, k, v, dout, w.blk_q, 0.1, 0)
+    topk = float(np.float32(0.1))
+    rows = synth.sample_rows(w.B, w.H, w.N, n_heads=3, rows_per_head=32)
+    got = dq.cpu().numpy().reshape(w.B * w.H, w.N, 128)[rows[:, 0], rows[:, 1]].astype(np.float64)
+    ref = oracle.backward_dq_rows(q, k, v, dout, w.blk_q, w.blk_k, topk, rows, phi=0)
+    eq = rel_l2(got, ref)
+    n_kb = -(-w.N // w.blk_k)
+    blocks = np.array([[0, 0], [5, n_kb // 2], [11, n_kb - 1]], dtype=np.int64)
+    ref_k, ref_v = oracle.backward_dkdv_blocks(q, k, v, dout, w.blk_q, w.blk_k, topk, blocks, phi=0)
+    dk_h, dv_h = dk.view(w.B * w.H, w.N, 128), dv.view(w.B * w.H, w.N, 128)
+    gk, gv, rk, rv = [], [], [], []
+    for b, (bh, J) in enumerate(blocks.tolist()):
+        n = min(64, w.N - 64 * J)
+        gk.append(dk_h[bh, 64 * J:64 * J + n].cpu().numpy().astype(np.float64))
+        gv.append(dv_h[bh, 64 * J:64 * J + n].cpu().numpy().astype(np.float64))
+        rk.append(ref_k[b, :n])
+        rv.append(ref_v[b, :n])
+    gk, gv, rk, rv = (np.concatenate(x) for x in (gk, gv, rk, rv))
+    assert np.isfinite(got).all() and np.isfinite(gk).all() and np.isfinite(gv).all()
+    ek, ev = rel_l2(gk, rk), rel_l2(gv, rv)
+    print(f"\n480P sampled: dq rel_l2={eq:.3e} dk rel_l2={ek:.3e} dv rel_l2={ev:.3e}")
+    assert eq <= TOL and ek <= TOL and ev <= TOL, (eq, ek, ev)

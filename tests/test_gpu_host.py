@@ -103,3 +103,15 @@ def test_host_forward_rejects_device_tensors():
     dev = sla.host_workspace(1, 1, 256, 128, 64, 64, 0.1, 1, 1)
     with pytest.raises(ValueError):
         sla.sla_forward_host(qd, qd, qd, qd, 64, 64, 0.1, 0, 1, 1, dev)
+
+
+def test_host_forward_at_480p_shape_equals_device_forward():
+    """The 1.3B-480P workload (B=1, H=12, N=32760) in chunks of 5 heads (5 + 5 + 2), INT8: the same
+    bytes as one device call."""
+    from gpu_helpers import workload_qkv
+
+    w = synth.WORKLOADS["wan1.3b-480p"]
+    q, k, v = workload_qkv("wan1.3b-480p")
+    ref = device_forward(q, k, v, w.blk_q, w.topk, 0, 1)
+    got, _ = host_forward(q, k, v, w.blk_q, w.topk, 0, 1, 5)
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
