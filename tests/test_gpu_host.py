@@ -16,7 +16,7 @@ import pytest
 
 import oracle
 import synth
-from gpu_helpers import bf16_to_f64, cosine, rel_l2, to_dev
+from gpu_helpers import bf16_to_f64, cosine, rel_l2, to_dev, workload_qkv
 
 pytestmark = pytest.mark.gpu
 
@@ -108,8 +108,6 @@ def test_host_forward_rejects_device_tensors():
 def test_host_forward_at_480p_shape_equals_device_forward():
     """The 1.3B-480P workload (B=1, H=12, N=32760) in chunks of 5 heads (5 + 5 + 2), INT8: the same
     bytes as one device call."""
-    from gpu_helpers import workload_qkv
-
     w = synth.WORKLOADS["wan1.3b-480p"]
     q, k, v = workload_qkv("wan1.3b-480p")
     ref = device_forward(q, k, v, w.blk_q, w.topk, 0, 1)
