@@ -307,6 +307,8 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     SLA_TRY(cudaStreamIsCapturing(s, &cap));
     ForkK fk;
     const bool fork = ev == nullptr && cap == cudaStreamCaptureStatusNone && fk.make();
+    if (ev == nullptr && cap == cudaStreamCaptureStatusNone && !fork)
+        cudaGetLastError();  // no second stream: run in order on `s`, and keep the failure from the launch checks
     cudaStream_t sk = fork ? fk.st : s;  // the K side's stream
     if (fork) {
         SLA_TRY(cudaEventRecord(fk.ev[0], s));
