@@ -442,7 +442,10 @@ sla_status sla_forward_host(const void *q_host, const void *k_host, const void *
     // events: [0] the caller's stream at entry; per chunk c: inputs landed (1 + 3c), forward done
     // (2 + 3c), output copied out (3 + 3c)
     HostPipe pipe;
-    if (!pipe.make(1 + 3 * n_chunks)) return SLA_ERR_CUDA;
+    if (!pipe.make(1 + 3 * n_chunks)) {
+        cudaGetLastError();  // reported here; later calls' launch checks do not see it
+        return SLA_ERR_CUDA;
+    }
     cudaStream_t s_in = pipe.st[0], s_cmp = pipe.st[1], s_out = pipe.st[2];
     auto ev_in = [&](int c) { return pipe.ev[1 + 3 * c]; };
     auto ev_done = [&](int c) { return pipe.ev[2 + 3 * c]; };
