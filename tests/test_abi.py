@@ -35,6 +35,18 @@ def test_every_declared_symbol_is_exported():
         assert hasattr(lib, n), n
 
 
+def test_every_exported_symbol_is_declared():
+    # the library's dynamic symbol table (default visibility) holds the header's calls and nothing else
+    import shutil
+    import subprocess
+
+    if shutil.which("nm") is None:
+        pytest.skip("nm not available")
+    out = subprocess.run(["nm", "-D", "--defined-only", sla.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = sorted({line.split()[-1] for line in out.stdout.splitlines() if line.split()[-1].startswith("sla_")})
+    assert exported == declared_symbols()
+
+
 def test_library_links_no_torch():
     with open(sla.LIB_PATH, "rb") as f:
         blob = f.read()
