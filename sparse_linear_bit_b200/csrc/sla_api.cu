@@ -239,8 +239,8 @@ sla_status sla_quantize_qk_fp8(const void *q, const void *k, int B, int H, int N
 
 namespace {
 
-// A second stream and two events for one forward call; released when the call returns (CUDA frees
-// them once the work queued on them has completed).
+// A second stream and three events for one forward call; released when the call returns (CUDA
+// frees them once the work queued on them has completed).
 struct ForkK {
     cudaStream_t st = nullptr;
     cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // fork, K block means ready, K side done
@@ -308,7 +308,7 @@ sla_status run_forward(const void *q, const void *k, const void *v, void *out, i
     ForkK fk;
     const bool fork = ev == nullptr && cap == cudaStreamCaptureStatusNone && fk.make();
     if (ev == nullptr && cap == cudaStreamCaptureStatusNone && !fork)
-        cudaGetLastError();  // no second stream: run in order on `s`, and keep the failure from the launch checks
+        cudaGetLastError();  // no second stream: run in order on `s`; the failure stays out of the launch checks
     cudaStream_t sk = fork ? fk.st : s;  // the K side's stream
     if (fork) {
         SLA_TRY(cudaEventRecord(fk.ev[0], s));
