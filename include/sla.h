@@ -49,10 +49,11 @@
  *
  * Memory: every pointer is caller-owned device memory (q, k, v, out, outputs
  * and the workspace), 16-byte aligned, except the host buffers of
- * sla_forward_host.  The library allocates nothing and
- * keeps no per-call global state; calls on different workspaces may run
- * concurrently on different streams.  Calls that share one workspace must be
- * ordered (same stream or explicit events).
+ * sla_forward_host.  The library allocates no memory and keeps no per-call
+ * global state (sla_forward and sla_forward_host create a few streams and
+ * events of their own and release them before they return); calls on different
+ * workspaces may run concurrently on different streams.  Calls that share one
+ * workspace must be ordered (same stream or explicit events).
  *
  * Errors: arguments are validated before anything is enqueued; a bad argument
  * returns SLA_ERR_INVALID_ARG (null/misaligned pointer, negative size, topk
